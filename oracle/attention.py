@@ -1,0 +1,161 @@
+"""Plain fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path (the CUDA library
+``libfa_b200.so`` and the Python binding in ``exact_attention_136_b200``)
+imports, calls or links this module, and this module imports nothing from the
+product package.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` use it.
+
+What it computes
+----------------
+"Standard attention" as the Flash Attention skill pages write it out
+(Flash Attention | Hermes Skill, Workflow 1, Step 2 "Replace standard
+attention"; the same step on the Russian mirror "Flash Attention - Fast
+Memory-Efficient Attention"): the softmax over keys of the scaled
+query-key dot products, multiplied by the values.  The explainer page
+(FlashAttention, aiunderstanding.org, "Overview"/"Deep dive") states that
+the tiled method reaches exactly the same attention, so the plain definition
+written out here *is* the oracle:
+
+    S_ij   = scale * sum_d Q[b,i,h,d] * K[b,j,h,d]          (all (i, j))
+    S_ij   = -inf  where key j is not visible to query i
+    m_i    = max_j S_ij
+    l_i    = sum_j exp(S_ij - m_i)
+    P_ij   = exp(S_ij - m_i) / l_i
+    O_i    = sum_j P_ij V[b,j,h,:]
+    LSE_i  = m_i + ln(l_i)            (natural log of sum_j exp(S_ij))
+
+Rows that see no key at all get O_i = 0 and LSE_i = -inf.
+
+Visibility (the "mask" of the pages' ``causal=True`` and ``window_size``
+arguments; Flash Attention | Hermes Skill, Workflow 2, Steps 2-3):
+    causal:               key j visible to query i only if j <= i
+    window_left = w >= 0: key j visible to query i only if j >= i - w
+    window_left = -1:     no window (the pages' ``(-1, -1)``)
+Indices are absolute (top-left aligned) also when N_q != N_k; this is the
+plainest reading, since the pages only show N_q == N_k.
+
+Layouts follow the pages' flash_attn_func layout ``[batch, seqlen, nheads,
+headdim]`` for Q, K, V and O (Workflow 2, Step 2), and ``[batch, heads,
+N_q]`` for LSE (the pages print no LSE layout; this is our reading).
+
+Everything is float64.  Inputs are the exact dtype-rounded (or dequantised
+FP8) values, upcast.  Matrix products use numpy's BLAS matmul, which is the
+only library primitive used; there is no tiling, fusion or online softmax.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Iterable
+
+import numpy as np
+
+__all__ = [
+    "visibility",
+    "attention_ref",
+    "attention_bruteforce",
+]
+
+
+def visibility(rows: Iterable[int], n_k: int, causal: bool, window_left: int) -> np.ndarray:
+    """Boolean [len(rows), n_k] table: True where key j is visible to query i.
+
+    Follows the pages' flash_attn_func arguments (Flash Attention | Hermes
+    Skill, Workflow 2, Step 2 ``causal=True`` and Step 3 ``window_size=(left,
+    right)``): causal hides keys after the query, a left window of ``w`` hides
+    keys more than ``w`` positions before it, ``-1`` means unlimited.
+    """
+    i = np.asarray(list(rows) if not isinstance(rows, np.ndarray) else rows, dtype=np.int64)[:, None]
+    j = np.arange(n_k, dtype=np.int64)[None, :]
+    vis = np.ones((i.shape[0], n_k), dtype=bool)
+    if causal:
+        vis &= j <= i
+    if window_left >= 0:
+        vis &= j >= i - window_left
+    return vis
+
+
+def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
+                  rows=None, return_probs: bool = False):
+    """Exact attention forward in float64 (definition in the module docstring).
+
+    q: [B, N_q, H, D]; k, v: [B, N_k, H, D] (any real dtype; upcast to fp64).
+    rows: optional 1-D array of query indices; only those rows are computed
+          (used for long sequences where the full N_q x N_k matrix is large).
+    Returns (O [B, R, H, D], LSE [B, H, R]) with R = len(rows) (or N_q), and
+    with ``return_probs`` also P [B, H, R, N_k].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("q, k, v must be [batch, seqlen, heads, headdim]")
+    B, n_q, H, D = q.shape
+    n_k = k.shape[1]
+    if k.shape != (B, n_k, H, D) or v.shape != (B, n_k, H, D):
+        raise ValueError("k and v must be [B, N_k, H, D] matching q")
+    rows = np.arange(n_q, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    R = rows.shape[0]
+    vis = visibility(rows, n_k, causal, window_left)
+    seen = vis.any(axis=1)
+
+    out = np.zeros((B, R, H, D), dtype=np.float64)
+    lse = np.full((B, H, R), -np.inf, dtype=np.float64)
+    probs = np.zeros((B, H, R, n_k), dtype=np.float64) if return_probs else None
+    for b in range(B):
+        for h in range(H):
+            # scores of every selected query against every key
+            s = scale * (q[b, rows, h, :] @ k[b, :, h, :].T)
+            s = np.where(vis, s, -np.inf)
+            m = np.where(seen, s.max(axis=1, initial=-np.inf), 0.0)
+            e = np.where(vis, np.exp(s - m[:, None]), 0.0)
+            l = e.sum(axis=1)
+            p = e / np.where(seen, l, 1.0)[:, None]
+            out[b, :, h, :] = p @ v[b, :, h, :]
+            lse[b, h, :] = np.where(seen, m + np.log(np.where(seen, l, 1.0)), -np.inf)
+            if return_probs:
+                probs[b, h] = p
+    if return_probs:
+        return out, lse, probs
+    return out, lse
+
+
+def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_left: int = -1):
+    """Pure-Python triple loop over (query, key, dim), for tiny shapes only.
+
+    Written independently of ``attention_ref``: nested lists, ``math.exp``, no
+    max subtraction, and the visibility rule spelled out inline.  Used only to
+    pin ``attention_ref``.  Returns (O, LSE) as nested Python lists shaped like
+    ``attention_ref``'s outputs.
+    """
+    B = len(q)
+    n_q = len(q[0])
+    H = len(q[0][0])
+    D = len(q[0][0][0])
+    n_k = len(k[0])
+    O = [[[[0.0] * D for _ in range(H)] for _ in range(n_q)] for _ in range(B)]
+    L = [[[float("-inf")] * n_q for _ in range(H)] for _ in range(B)]
+    for b in range(B):
+        for h in range(H):
+            for i in range(n_q):
+                weights = []
+                for j in range(n_k):
+                    if causal and j > i:
+                        continue
+                    if window_left != -1 and i - j > window_left:
+                        continue
+                    dot = 0.0
+                    for d in range(D):
+                        dot += float(q[b][i][h][d]) * float(k[b][j][h][d])
+                    weights.append((j, math.exp(scale * dot)))
+                total = sum(w for _, w in weights)
+                if not weights:
+                    continue
+                L[b][h][i] = math.log(total)
+                for d in range(D):
+                    acc = 0.0
+                    for j, w in weights:
+                        acc += w * float(v[b][j][h][d])
+                    O[b][i][h][d] = acc / total
+    return O, L

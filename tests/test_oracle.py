@@ -1,0 +1,302 @@
+"""Pins for the fp64 oracle, independent of the oracle's own code.
+
+Each check fixes the oracle against something other than itself: a
+pure-Python brute force written separately, closed forms (constant V, Q = 0,
+causal row 0, a two-key window, one-hot scores), invariants (row sums, shift
+and key-permutation invariance), scipy's softmax / logsumexp, and the literal
+window rule "i - w <= j <= i".  The last tests plant plausible mistakes in the
+oracle (on the CPU) and require that at least one pin catches each of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle.attention as oa
+from oracle import attention_bruteforce, attention_ref, visibility
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_values.json")
+MODES = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 3), (False, 2), (True, 100)]
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# --------------------------------------------------------------------------
+# pin functions: each takes an attention function with attention_ref's
+# signature and raises AssertionError when it disagrees with the pin
+# --------------------------------------------------------------------------
+
+def pin_bruteforce(fn):
+    for (n_q, n_k, D) in [(1, 1, 1), (2, 2, 4), (3, 3, 8), (7, 7, 4), (17, 17, 8), (5, 9, 4), (9, 5, 4)]:
+        for causal, wl in MODES:
+            q = _rand((2, n_q, 2, D), 10 + n_q)
+            k = _rand((2, n_k, 2, D), 20 + n_k)
+            v = _rand((2, n_k, 2, D), 30 + D)
+            scale = 0.37
+            o, l = fn(q, k, v, scale, causal, wl)
+            ob, lb = attention_bruteforce(q.tolist(), k.tolist(), v.tolist(), scale, causal, wl)
+            np.testing.assert_allclose(o, np.array(ob), rtol=0, atol=1e-12)
+            lb = np.array(lb)
+            assert np.array_equal(np.isinf(l), np.isinf(lb))
+            fin = np.isfinite(lb)
+            np.testing.assert_allclose(l[fin], lb[fin], rtol=0, atol=1e-12)
+
+
+def pin_constant_v(fn):
+    q, k = _rand((1, 33, 3, 8), 1), _rand((1, 33, 3, 8), 2)
+    row = _rand((8,), 3)
+    v = np.broadcast_to(row, (1, 33, 3, 8)).copy()
+    for causal, wl in MODES:
+        o, _ = fn(q, k, v, 0.9, causal, wl)
+        np.testing.assert_allclose(o, np.broadcast_to(row, o.shape), rtol=0, atol=1e-12)
+
+
+def pin_zero_query_mean(fn):
+    n = 40
+    k, v = _rand((2, n, 2, 4), 4), _rand((2, n, 2, 4), 5)
+    q = np.zeros((2, n, 2, 4))
+    for causal, wl in MODES:
+        o, l = fn(q, k, v, 1.3, causal, wl)
+        for i in range(n):
+            lo = 0 if wl < 0 else max(0, i - wl)
+            hi = i if causal else n - 1
+            mean = v[:, lo:hi + 1].mean(axis=1)
+            np.testing.assert_allclose(o[:, i], mean, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(l[:, :, i], math.log(hi - lo + 1), rtol=0, atol=1e-12)
+
+
+def pin_scale_zero_mean(fn):
+    n = 24
+    q, k, v = _rand((1, n, 2, 4), 6), _rand((1, n, 2, 4), 7), _rand((1, n, 2, 4), 8)
+    o, l = fn(q, k, v, 0.0, True, -1)
+    for i in range(n):
+        np.testing.assert_allclose(o[:, i], v[:, :i + 1].mean(axis=1), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l[:, :, i], math.log(i + 1), rtol=0, atol=1e-12)
+
+
+def pin_causal_row0(fn):
+    q, k, v = _rand((2, 16, 3, 8), 9), _rand((2, 16, 3, 8), 10), _rand((2, 16, 3, 8), 11)
+    scale = 0.25
+    o, l = fn(q, k, v, scale, True, -1)
+    np.testing.assert_allclose(o[:, 0], v[:, 0], rtol=0, atol=1e-12)
+    dot0 = np.einsum("bhd,bhd->bh", q[:, 0], k[:, 0])
+    np.testing.assert_allclose(l[:, :, 0], scale * dot0, rtol=0, atol=1e-12)
+
+
+def pin_window_zero(fn):
+    """causal with a left window of 0: each query sees only its own key."""
+    q, k, v = _rand((1, 20, 2, 8), 12), _rand((1, 20, 2, 8), 13), _rand((1, 20, 2, 8), 14)
+    scale = 0.5
+    o, l = fn(q, k, v, scale, True, 0)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l, scale * np.einsum("bnhd,bnhd->bhn", q, k), rtol=0, atol=1e-12)
+
+
+def pin_two_key_window(fn):
+    """causal, window 1: query i >= 1 sees keys i-1 and i; closed-form sigmoid weights."""
+    q, k, v = _rand((1, 12, 1, 4), 15), _rand((1, 12, 1, 4), 16), _rand((1, 12, 1, 4), 17)
+    scale = 0.7
+    o, l = fn(q, k, v, scale, True, 1)
+    for i in range(1, 12):
+        a = scale * float(q[0, i, 0] @ k[0, i, 0])
+        b = scale * float(q[0, i, 0] @ k[0, i - 1, 0])
+        w_self = 1.0 / (1.0 + math.exp(b - a))
+        expect = w_self * v[0, i, 0] + (1.0 - w_self) * v[0, i - 1, 0]
+        np.testing.assert_allclose(o[0, i, 0], expect, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l[0, 0, i], math.log(math.exp(a) + math.exp(b)), rtol=0, atol=1e-12)
+
+
+def pin_scipy(fn):
+    """softmax weights and LSE against scipy.special on the full score matrix."""
+    q, k, v = _rand((1, 30, 2, 6), 18), _rand((1, 30, 2, 6), 19), _rand((1, 30, 2, 6), 20)
+    scale = 0.8
+    for causal, wl in MODES:
+        o, l = fn(q, k, v, scale, causal, wl)
+        for h in range(2):
+            s = scale * np.einsum("id,jd->ij", q[0, :, h], k[0, :, h])
+            i = np.arange(30)[:, None]
+            j = np.arange(30)[None, :]
+            keep = np.ones((30, 30), bool)
+            if causal:
+                keep &= ~(j > i)
+            if wl >= 0:
+                keep &= ~(i - j > wl)
+            s = np.where(keep, s, -np.inf)
+            p = scipy.special.softmax(s, axis=1)
+            np.testing.assert_allclose(o[0, :, h], p @ v[0, :, h], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(l[0, h], scipy.special.logsumexp(s, axis=1), rtol=0, atol=1e-12)
+
+
+def pin_shift_invariance(fn):
+    """A constant added to every score of a row leaves O and moves LSE by it."""
+    q, k, v = _rand((1, 25, 2, 5), 21), _rand((1, 25, 2, 5), 22), _rand((1, 25, 2, 5), 23)
+    c, scale = 3.25, 0.6
+    q2 = np.concatenate([q, np.ones((1, 25, 2, 1))], axis=-1)
+    k2 = np.concatenate([k, np.full((1, 25, 2, 1), c)], axis=-1)
+    for causal, wl in MODES:
+        o1, l1 = fn(q, k, v, scale, causal, wl)
+        v2 = np.concatenate([v, np.zeros((1, 25, 2, 1))], axis=-1)  # values padded with 0
+        o2, l2 = fn(q2, k2, v2, scale, causal, wl)
+        np.testing.assert_allclose(o2[..., :5], o1, rtol=0, atol=1e-12)
+        assert np.all(o2[..., 5] == 0.0)
+        np.testing.assert_allclose(l2, l1 + scale * c, rtol=0, atol=1e-12)
+
+
+def pin_key_permutation(fn):
+    q, k, v = _rand((1, 19, 2, 4), 24), _rand((1, 31, 2, 4), 25), _rand((1, 31, 2, 4), 26)
+    perm = np.random.default_rng(27).permutation(31)
+    o1, l1 = fn(q, k, v, 0.45, False, -1)
+    o2, l2 = fn(q, k[:, perm], v[:, perm], 0.45, False, -1)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-12)
+
+
+def pin_wide_window_is_causal(fn):
+    q, k, v = _rand((1, 37, 2, 4), 28), _rand((1, 37, 2, 4), 29), _rand((1, 37, 2, 4), 30)
+    o1, l1 = fn(q, k, v, 0.5, True, -1)
+    for wl in (36, 37, 1000):
+        o2, l2 = fn(q, k, v, 0.5, True, wl)
+        np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-12)
+
+
+def pin_one_hot_large_scores(fn):
+    """Q = K = 30 * identity rows: score 900 on the diagonal, 0 elsewhere; no overflow."""
+    n = 16
+    eye = np.zeros((1, n, 1, n))
+    for i in range(n):
+        eye[0, i, 0, i] = 30.0
+    v = _rand((1, n, 1, n), 31)
+    o, l = fn(eye, eye, v, 1.0, False, -1)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(l))
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l, 900.0, rtol=0, atol=1e-12)
+
+
+def pin_empty_rows(fn):
+    """With N_q > N_k + w, late queries see no key: O = 0, LSE = -inf."""
+    q, k, v = _rand((1, 12, 1, 4), 32), _rand((1, 4, 1, 4), 33), _rand((1, 4, 1, 4), 34)
+    o, l = fn(q, k, v, 1.0, True, 2)
+    # query i sees keys max(0, i-2) .. min(i, 3); empty once i - 2 > 3
+    for i in range(12):
+        if i - 2 > 3:
+            assert np.all(o[0, i] == 0.0) and l[0, 0, i] == -np.inf
+        else:
+            assert np.isfinite(l[0, 0, i])
+
+
+PINS = [pin_bruteforce, pin_constant_v, pin_zero_query_mean, pin_scale_zero_mean, pin_causal_row0,
+        pin_window_zero, pin_two_key_window, pin_scipy, pin_shift_invariance, pin_key_permutation,
+        pin_wide_window_is_causal, pin_one_hot_large_scores, pin_empty_rows]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_oracle_pin(pin):
+    pin(attention_ref)
+
+
+def test_rows_sum_to_one_and_nonnegative():
+    q, k, v = _rand((2, 29, 2, 4), 40), _rand((2, 29, 2, 4), 41), _rand((2, 29, 2, 4), 42)
+    for causal, wl in MODES:
+        _, _, p = attention_ref(q, k, v, 1.1, causal, wl, return_probs=True)
+        assert np.all(p >= 0)
+        np.testing.assert_allclose(p.sum(axis=-1), 1.0, rtol=0, atol=1e-12)
+        vis = visibility(np.arange(29), 29, causal, wl)
+        assert np.all(p[..., ~vis] == 0)
+
+
+def test_sampled_rows_match_full():
+    q, k, v = _rand((1, 50, 2, 4), 43), _rand((1, 50, 2, 4), 44), _rand((1, 50, 2, 4), 45)
+    rows = np.array([0, 3, 17, 49])
+    o, l = attention_ref(q, k, v, 0.3, True, 5)
+    os_, ls = attention_ref(q, k, v, 0.3, True, 5, rows=rows)
+    np.testing.assert_array_equal(os_, o[:, rows])
+    np.testing.assert_array_equal(ls, l[:, :, rows])
+
+
+def test_visibility_literal_window_rule():
+    """The sliding-window workload's rule, written literally: visible iff i - w <= j <= i."""
+    rng = np.random.default_rng(46)
+    for _ in range(200):
+        n = int(rng.integers(1, 60))
+        w = int(rng.integers(0, 70))
+        vis = visibility(np.arange(n), n, True, w)
+        for i in range(n):
+            for j in range(n):
+                assert vis[i, j] == (i - w <= j <= i)
+
+
+def test_pages_auto_scale_reading():
+    """The pages divide D=64 scores by 8.0 and call the default 'auto-scale'; 1/sqrt(64) == 1/8."""
+    g = json.load(open(GOLDEN))
+    acc = g["accuracy_check"]
+    assert 1.0 / math.sqrt(acc["headdim"]) == 1.0 / acc["score_divisor"]
+    assert g["no_window"]["window_size"] == [-1, -1]
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each plausible slip in the oracle must fail >= 1 pin
+# --------------------------------------------------------------------------
+
+def _caught(fn):
+    for pin in PINS:
+        try:
+            pin(fn)
+        except AssertionError:
+            return True
+    return False
+
+
+def _mut_dropped_scale(q, k, v, scale, causal=False, wl=-1, **kw):
+    return attention_ref(q, k, v, 1.0, causal, wl, **kw)
+
+
+def _mut_swapped_kv(q, k, v, scale, causal=False, wl=-1, **kw):
+    return attention_ref(q, v, k, scale, causal, wl, **kw)
+
+
+def _mut_log2_lse(q, k, v, scale, causal=False, wl=-1, **kw):
+    o, l = attention_ref(q, k, v, scale, causal, wl, **kw)
+    return o, l / math.log(2.0)
+
+
+def _mut_unnormalised(q, k, v, scale, causal=False, wl=-1, **kw):
+    o, l = attention_ref(q, k, v, scale, causal, wl, **kw)
+    return o * 1.0001, l
+
+
+def _mut_transposed_heads(q, k, v, scale, causal=False, wl=-1, **kw):
+    # k read with batch and head roles crossed
+    return attention_ref(q, np.ascontiguousarray(k[:, :, ::-1]), v, scale, causal, wl, **kw)
+
+
+def _mut_negated_scores(q, k, v, scale, causal=False, wl=-1, **kw):
+    return attention_ref(q, k, v, -scale, causal, wl, **kw)
+
+
+@pytest.mark.parametrize("mut", [_mut_dropped_scale, _mut_swapped_kv, _mut_log2_lse,
+                                 _mut_unnormalised, _mut_transposed_heads, _mut_negated_scores])
+def test_planted_mistake_is_caught(mut):
+    assert _caught(mut)
+
+
+@pytest.mark.parametrize("bad", ["strict_causal", "window_off_by_one", "window_ignored", "causal_ignored"])
+def test_planted_mask_mistake_is_caught(monkeypatch, bad):
+    def mutated(rows, n_k, causal, window_left):
+        i = np.asarray(rows, dtype=np.int64)[:, None]
+        j = np.arange(n_k)[None, :]
+        vis = np.ones((i.shape[0], n_k), bool)
+        if causal and bad != "causal_ignored":
+            vis &= (j < i) if bad == "strict_causal" else (j <= i)
+        if window_left >= 0 and bad != "window_ignored":
+            vis &= (j > i - window_left) if bad == "window_off_by_one" else (j >= i - window_left)
+        return vis
+
+    monkeypatch.setattr(oa, "visibility", mutated)
+    assert _caught(oa.attention_ref)

@@ -1,1 +1,12 @@
-"""Exact attention forward for NVIDIA B200 (sm_100a)."""
+"""Exact attention forward for NVIDIA B200 (sm_100a).
+
+    from exact_attention_136_b200 import forward
+    out, lse = forward(q, k, v, causal=True)      # [batch, seqlen, heads, headdim]
+
+The computation runs in libfa_b200.so (hand-written sm_100a CUDA, C ABI in
+include/fa.h); this package only marshals arguments.
+"""
+
+from .api import device_status, forward, forward_fp8, forward_host, set_wait_limit_ns, wait_probe
+
+__all__ = ["forward", "forward_fp8", "forward_host", "device_status", "set_wait_limit_ns", "wait_probe"]

@@ -1,0 +1,146 @@
+"""Python entry points over the C ABI (argument marshalling only).
+
+Tensors use the pages' flash_attn_func layout [batch, seqlen, nheads,
+headdim] (Flash Attention | Hermes Skill, Workflow 2, Step 2).  PyTorch only
+allocates outputs and supplies the current CUDA stream; every step of the
+computation runs in libfa_b200.so.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float16: _lib.FA_FP16, torch.bfloat16: _lib.FA_BF16, torch.float8_e4m3fn: _lib.FA_E4M3}
+
+
+def _check_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [batch, seqlen, heads, headdim]")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _DT:
+        raise ValueError("q, k, v must share one dtype: float16, bfloat16 or float8_e4m3fn")
+    B, n_q, H, D = q.shape
+    if k.shape[0] != B or k.shape[2:] != (H, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, N_k, H, D] with q's B, H, D")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
+    return B, n_q, k.shape[1], H, D
+
+
+def _outputs(q, B, n_q, H, D, out, lse, want_lse):
+    out_dtype = torch.float16 if q.dtype == torch.float16 else torch.bfloat16
+    if out is None:
+        out = torch.empty((B, n_q, H, D), dtype=out_dtype, device=q.device)
+    elif out.shape != (B, n_q, H, D) or out.dtype != out_dtype or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {out_dtype} tensor of shape {(B, n_q, H, D)}")
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, n_q), dtype=torch.float32, device=q.device)
+    elif lse is not None and (lse.shape != (B, H, n_q) or lse.dtype != torch.float32
+                              or not lse.is_contiguous()):
+        raise ValueError(f"lse must be a contiguous float32 tensor of shape {(B, H, n_q)}")
+    return out, lse
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+            causal: bool = False, window_left: int = -1, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None, return_lse: bool = True,
+            stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Exact attention forward; returns (out, lse).
+
+    scale=None means 1/sqrt(headdim), the pages' auto scale (Workflow 2,
+    Step 2).  window_left=-1 means no window.  For float8_e4m3fn inputs all
+    descales are 1; use forward_fp8 to pass per-tensor scales.
+    """
+    B, n_q, n_k, H, D = _check_inputs(q, k, v)
+    if q.dtype == torch.float8_e4m3fn:
+        return forward_fp8(q, k, v, 1.0, 1.0, 1.0, scale, causal, window_left, out, lse, return_lse, stream)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out, lse = _outputs(q, B, n_q, H, D, out, lse, return_lse)
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        rc = _lib.lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, D, scale,
+                               int(bool(causal)), int(window_left), _DT[q.dtype], s.cuda_stream)
+    _lib.check(rc, "fa_fwd")
+    return out, lse
+
+
+def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale: float, k_descale: float,
+                v_descale: float, scale: Optional[float] = None, causal: bool = False,
+                window_left: int = -1, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                return_lse: bool = True, stream: Optional[torch.cuda.Stream] = None):
+    """FP8 e4m3 forward with per-tensor descales; out is bfloat16."""
+    B, n_q, n_k, H, D = _check_inputs(q8, k8, v8)
+    if q8.dtype != torch.float8_e4m3fn:
+        raise ValueError("forward_fp8 takes float8_e4m3fn tensors")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out, lse = _outputs(q8, B, n_q, H, D, out, lse, return_lse)
+    with torch.cuda.device(q8.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q8.device)
+        rc = _lib.lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, D, scale,
+                                   int(bool(causal)), int(window_left), float(q_descale), float(k_descale),
+                                   float(v_descale), s.cuda_stream)
+    _lib.check(rc, "fa_fwd_fp8")
+    return out, lse
+
+
+def forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, staging, scale: float, causal: bool = False,
+                 window_left: int = -1, descales=(1.0, 1.0, 1.0), out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Forward on HOST tensors through fa_fwd_host.
+
+    q, k, v are CPU tensors (pinned for asynchronous copies); `staging` is a
+    dict of device tensors "q", "k", "v", "out", "lse" that the call copies
+    through.  Returns the host (out, lse).
+    """
+    B, n_q, H, D = q.shape
+    n_k = k.shape[1]
+    dt = _DT[q.dtype]
+    out_dtype = torch.float16 if q.dtype == torch.float16 else torch.bfloat16
+    if out is None:
+        out = torch.empty((B, n_q, H, D), dtype=out_dtype, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, H, n_q), dtype=torch.float32, pin_memory=True)
+    dev = staging["q"].device
+    with torch.cuda.device(dev):
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        rc = _lib.lib().fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                    staging["q"].data_ptr(), staging["k"].data_ptr(), staging["v"].data_ptr(),
+                                    staging["out"].data_ptr(), staging["lse"].data_ptr(), B, n_q, n_k, H, D,
+                                    float(scale), int(bool(causal)), int(window_left), dt,
+                                    float(descales[0]), float(descales[1]), float(descales[2]),
+                                    s.cuda_stream)
+    _lib.check(rc, "fa_fwd_host")
+    return out, lse
+
+
+def device_status(stream: Optional[torch.cuda.Stream] = None, device=None) -> Tuple[int, int]:
+    """(status, flags) of the device status word; synchronises the stream and clears the word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        flags = ctypes.c_int(0)
+        rc = _lib.lib().fa_device_status(s.cuda_stream, ctypes.byref(flags))
+    return rc, flags.value
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    _lib.lib().fa_set_wait_limit_ns(int(limit_ns))
+
+
+def wait_probe(limit_ns: int, stream: Optional[torch.cuda.Stream] = None, device=None) -> None:
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        _lib.check(_lib.lib().fa_wait_probe(int(limit_ns), s.cuda_stream), "fa_wait_probe")

@@ -1,0 +1,229 @@
+// C ABI of the attention library (declared in include/fa.h): argument
+// validation, TMA tensor-map encoding, persistent-grid sizing and launch.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_fwd_kernel.cuh"
+#include "tmap.h"
+
+namespace fa {
+
+__device__ int g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool init = false;
+  int num_sms = 0;
+  int* status = nullptr;     // device address of g_status_word
+  unsigned attr_set = 0;     // bit per kernel instantiation
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+unsigned long long g_wait_limit_ns = 2000000000ull;
+
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  DeviceState& s = g_dev[dev];
+  if (!s.init) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!s.init) {
+      if (cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return FA_ERR_CUDA;
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.status), g_status_word) != cudaSuccess)
+        return FA_ERR_CUDA;
+      s.init = true;
+    }
+  }
+  *out = &s;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D, int DT>
+int launch(const void* q, const void* k, const void* v, const FwdParams& base, cudaStream_t stream,
+           DeviceState* ds, int bit) {
+  using C = Cfg<D, DT>;
+  FwdParams p = base;
+  const CUtensorMapDataType tdt = DT == DT_FP16   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                  : DT == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUtensorMap mq, mk, mv;
+  if (encode_bnhd(&mq, q, tdt, C::ES, p.B, p.Nq, p.H, D, C::BOX_INNER, BLOCK_M) ||
+      encode_bnhd(&mk, k, tdt, C::ES, p.B, p.Nk, p.H, D, C::BOX_INNER, BLOCK_N) ||
+      encode_bnhd(&mv, v, tdt, C::ES, p.B, p.Nk, p.H, D, C::BOX_INNER, BLOCK_N))
+    return FA_ERR_CUDA;
+  if (!(ds->attr_set & (1u << bit))) {
+    if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return FA_ERR_CUDA;
+    ds->attr_set |= (1u << bit);
+  }
+  const int grid = p.num_units < ds->num_sms ? p.num_units : ds->num_sms;
+  fa_fwd_kernel<D, DT><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int validate(const void* q, const void* k, const void* v, void* out, int B, int Nq, int Nk, int H,
+             int D, float scale, int causal, int window_left, int dtype) {
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 0) return FA_ERR_ARG;
+  // q / out may be NULL only when there are no queries, k / v only when there are no keys
+  if ((Nq > 0 && (!q || !out)) || (Nk > 0 && (!k || !v))) return FA_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_ARG;
+  if (window_left < -1) return FA_ERR_ARG;
+  if (dtype != FA_FP16 && dtype != FA_BF16 && dtype != FA_E4M3) return FA_ERR_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_E4M3 && D != 128) return FA_ERR_UNSUPPORTED;
+  // TMA coordinates are 32-bit; keep every index well inside int range
+  const int64_t rows_q = static_cast<int64_t>(B) * Nq * H;
+  const int64_t rows_k = static_cast<int64_t>(B) * Nk * H;
+  if (rows_q > (int64_t(1) << 31) || rows_k > (int64_t(1) << 31)) return FA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FA_ERR_ALIGN;
+  return FA_OK;
+}
+
+int forward(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Nq, int Nk,
+            int H, int D, float scale, int causal, int window_left, int dtype, float qd, float kd,
+            float vd, cudaStream_t stream) {
+  int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype);
+  if (rc != FA_OK) return rc;
+  if (!(qd > 0.f) || !std::isfinite(qd) || !(kd > 0.f) || !std::isfinite(kd) || !(vd > 0.f) ||
+      !std::isfinite(vd))
+    return FA_ERR_ARG;
+  if (Nq == 0) return FA_OK;
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if (Nk == 0) {
+    const int threads = 256;
+    const int64_t rows = static_cast<int64_t>(B) * Nq * H;
+    const int blocks = static_cast<int>(rows / threads + 1 < 4096 ? rows / threads + 1 : 4096);
+    if (D == 64) fa_empty_kernel<64, 2><<<blocks, threads, 0, stream>>>(out, lse, B, Nq, H);
+    else fa_empty_kernel<128, 2><<<blocks, threads, 0, stream>>>(out, lse, B, Nq, H);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  }
+  FwdParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.H = H;
+  p.causal = causal;
+  p.window_left = window_left;
+  p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
+                                     static_cast<double>(qd) * static_cast<double>(kd));
+  p.out_scale = vd;
+  p.pairs = (Nq + 2 * BLOCK_M - 1) / (2 * BLOCK_M);
+  const int64_t units = static_cast<int64_t>(p.pairs) * B * H;
+  if (units > 0x7fffffff) return FA_ERR_ARG;
+  p.num_units = static_cast<int>(units);
+  p.wait_limit_ns = g_wait_limit_ns;
+  p.status = ds->status;
+  switch (dtype * 2 + (D == 128 ? 1 : 0)) {
+    case FA_FP16 * 2 + 0: return launch<64, DT_FP16>(q, k, v, p, stream, ds, 0);
+    case FA_FP16 * 2 + 1: return launch<128, DT_FP16>(q, k, v, p, stream, ds, 1);
+    case FA_BF16 * 2 + 0: return launch<64, DT_BF16>(q, k, v, p, stream, ds, 2);
+    case FA_BF16 * 2 + 1: return launch<128, DT_BF16>(q, k, v, p, stream, ds, 3);
+    case FA_E4M3 * 2 + 1: return launch<128, DT_E4M3>(q, k, v, p, stream, ds, 4);
+    default: return FA_ERR_UNSUPPORTED;
+  }
+}
+
+size_t elem_bytes(int dtype) { return dtype == FA_E4M3 ? 1 : 2; }
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q, int N_k,
+           int H, int D, float scale, int causal, int window_left, int dtype, fa_stream_t stream) {
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, D, scale, causal, window_left, dtype, 1.f, 1.f,
+                     1.f, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q,
+               int N_k, int H, int D, float scale, int causal, int window_left, float q_descale,
+               float k_descale, float v_descale, fa_stream_t stream) {
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, D, scale, causal, window_left, FA_E4M3,
+                     q_descale, k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,
+                void* dv, void* dout, float* dlse, int B, int N_q, int N_k, int H, int D, float scale,
+                int causal, int window_left, int dtype, float q_descale, float k_descale,
+                float v_descale, fa_stream_t stream) {
+  if (!q || !k || !v || !out) return FA_ERR_ARG;
+  int rc = fa::validate(dq, dk, dv, dout, B, N_q, N_k, H, D, scale, causal, window_left, dtype);
+  if (rc != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = fa::elem_bytes(dtype);
+  const size_t nq = static_cast<size_t>(B) * N_q * H * D;
+  const size_t nk = static_cast<size_t>(B) * N_k * H * D;
+  if (cudaMemcpyAsync(dq, q, nq * es, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k, nk * es, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v, nk * es, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return FA_ERR_CUDA;
+  rc = fa::forward(dq, dk, dv, dout, dlse, B, N_q, N_k, H, D, scale, causal, window_left, dtype,
+                   q_descale, k_descale, v_descale, s);
+  if (rc != FA_OK) return rc;
+  if (cudaMemcpyAsync(out, dout, nq * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (lse && dlse &&
+      cudaMemcpyAsync(lse, dlse, static_cast<size_t>(B) * H * N_q * sizeof(float), cudaMemcpyDeviceToHost,
+                      s) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_device_status(fa_stream_t stream, int* flags) {
+  fa::DeviceState* ds = nullptr;
+  int rc = fa::device_state(&ds);
+  if (rc != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, ds->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  const int zero = 0;
+  if (word != 0 && cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (flags) *flags = word;
+  return word == 0 ? FA_OK : FA_ERR_TIMEOUT;
+}
+
+void fa_set_wait_limit_ns(unsigned long long limit_ns) {
+  fa::g_wait_limit_ns = limit_ns > 0 ? limit_ns : 1ull;
+}
+
+int fa_wait_probe(unsigned long long limit_ns, fa_stream_t stream) {
+  fa::DeviceState* ds = nullptr;
+  int rc = fa::device_state(&ds);
+  if (rc != FA_OK) return rc;
+  fa::fa_wait_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, ds->status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported head dim / dtype";
+    case FA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case FA_ERR_CUDA: return "CUDA runtime error";
+    case FA_ERR_TIMEOUT: return "kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* fa_version(void) { return "0.1.0"; }
+
+}  // extern "C"

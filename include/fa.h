@@ -1,0 +1,128 @@
+/*
+ * fa.h -- C ABI of libfa_b200.so: exact attention forward on NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation is the pages' "standard attention" (Flash Attention | Hermes
+ * Skill, Workflow 1, Step 2): for every batch b, head h and query row i
+ *
+ *     S_ij   = scale * sum_d Q[b,i,h,d] * K[b,j,h,d]
+ *     O[b,i,h,:] = sum_j softmax_j(S_ij over visible j) * V[b,j,h,:]
+ *     LSE[b,h,i] = ln sum_{visible j} exp(S_ij)
+ *
+ * computed tile by tile with an online softmax so the N_q x N_k scores never
+ * reach device memory (FlashAttention explainer, aiunderstanding.org,
+ * "Technical insight").  Visibility follows the flash_attn_func arguments
+ * shown on the pages (Workflow 2, Steps 2-3): with `causal`, key j is visible
+ * to query i only if j <= i; with window_left = w >= 0, only if j >= i - w;
+ * window_left = -1 means no window (the pages' window_size=(-1,-1)).  Query
+ * and key indices are absolute (top-left aligned) also when N_q != N_k.  A
+ * row that sees no key gets O = 0 and LSE = -inf.
+ *
+ * Layouts (the pages' flash_attn_func layout [batch, seqlen, nheads,
+ * headdim], Workflow 2, Step 2), all contiguous, row-major:
+ *     q, out : [B, N_q, H, D]      k, v : [B, N_k, H, D]
+ *     lse    : [B, H, N_q] float32 (may be NULL: not written)
+ * Element types: FA_FP16 -> q/k/v/out fp16; FA_BF16 -> q/k/v/out bf16;
+ * FA_E4M3 -> q/k/v e4m3 (OCP FP8, 1 byte), out bf16.
+ *
+ * Ownership: the caller allocates and owns every buffer; the library
+ * allocates no device memory and keeps no pointer after a call returns.
+ * Calls are asynchronous on `stream` (NULL = the legacy default stream);
+ * outputs are ready when the stream's work completes.
+ *
+ * Errors: every entry point returns FA_OK (0) or a negative fa_status and
+ * never aborts.  Argument errors are detected before any GPU work is queued.
+ * Wait timeouts inside a running kernel are recorded on the device and
+ * reported by fa_device_status().
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1, FA_E4M3 = 2 } fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_ARG = -1,         /* bad size, flag, scale or NULL pointer          */
+  FA_ERR_UNSUPPORTED = -2, /* head dim / dtype combination not built          */
+  FA_ERR_ALIGN = -3,       /* q, k, v or out not 16-byte aligned              */
+  FA_ERR_CUDA = -4,        /* CUDA runtime error (no device, launch failure)  */
+  FA_ERR_TIMEOUT = -5      /* a kernel wait ran past its limit (see below)    */
+} fa_status;
+
+/*
+ * fa_fwd -- attention forward for fp16 / bf16 inputs (dtype FA_E4M3 is
+ * accepted too and means all descales are 1).
+ *   B, H >= 1; N_q, N_k >= 0; D in {64, 128} (FA_E4M3: D = 128).
+ *   scale: finite and > 0 (the pages' default is 1/sqrt(D)).
+ *   causal: 0 or 1.  window_left: -1 (none) or >= 0.
+ * q and out may be NULL when N_q = 0, k and v when N_k = 0 (N_q = 0 is a
+ * no-op; N_k = 0 writes O = 0 and LSE = -inf).
+ * Returns FA_ERR_ARG / FA_ERR_UNSUPPORTED / FA_ERR_ALIGN without touching
+ * the GPU, FA_ERR_CUDA when the launch fails, else FA_OK.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+           int B, int N_q, int N_k, int H, int D, float scale, int causal,
+           int window_left, int dtype, fa_stream_t stream);
+
+/*
+ * fa_fwd_fp8 -- FP8 e4m3 forward with per-tensor scales (the FP8 forward the
+ * pages describe for FlashAttention-3, Flash Attention | Hermes Skill,
+ * Workflow 3).  The true inputs are q_descale * q, k_descale * k and
+ * v_descale * v; out is bf16.  Softmax probabilities are quantised to e4m3
+ * (after a power-of-two shift into e4m3's range) for the P*V product; all
+ * accumulation is fp32.  Descales must be finite and > 0.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
+               int B, int N_q, int N_k, int H, int D, float scale, int causal,
+               int window_left, float q_descale, float k_descale, float v_descale,
+               fa_stream_t stream);
+
+/*
+ * fa_fwd_host -- the same forward on HOST buffers: copies q, k, v from host
+ * to the caller's device buffers dq, dk, dv, runs fa_fwd / fa_fwd_fp8 into
+ * dout / dlse, and copies out (and lse, when both lse and dlse are non-NULL)
+ * back to host, all on `stream`.  Host buffers should be pinned for
+ * asynchronous copies.  Synchronises `stream` before returning.
+ */
+int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse,
+                void* dq, void* dk, void* dv, void* dout, float* dlse,
+                int B, int N_q, int N_k, int H, int D, float scale, int causal,
+                int window_left, int dtype, float q_descale, float k_descale,
+                float v_descale, fa_stream_t stream);
+
+/*
+ * fa_device_status -- synchronises `stream`, then reads and clears the
+ * device status word that kernels set when a wait times out.  Returns FA_OK,
+ * FA_ERR_TIMEOUT (and the raw flag bits in *flags when flags != NULL) or
+ * FA_ERR_CUDA.
+ */
+int fa_device_status(fa_stream_t stream, int* flags);
+
+/* Upper bound of every in-kernel wait, in nanoseconds (default 2e9). */
+void fa_set_wait_limit_ns(unsigned long long limit_ns);
+
+/*
+ * fa_wait_probe -- launches one CTA whose wait nothing completes, with the
+ * given limit; used to check that waits end and report FA_ERR_TIMEOUT
+ * through fa_device_status instead of hanging.
+ */
+int fa_wait_probe(unsigned long long limit_ns, fa_stream_t stream);
+
+/* Static description of a status code. */
+const char* fa_status_string(int status);
+
+/* Library version, e.g. "0.1.0". */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

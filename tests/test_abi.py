@@ -1,0 +1,102 @@
+"""C-ABI library: loads, exports every declared symbol, rejects bad arguments
+on the host before touching a GPU (no compute calls here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_136_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_fwd_fp8", "fa_fwd_host", "fa_device_status", "fa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(_lib.SIGNATURES), "binding misses a declared entry point"
+
+
+def test_status_strings_and_version():
+    assert _lib.status_string(0) == "ok"
+    for code in (-1, -2, -3, -4, -5):
+        assert _lib.status_string(code) != "unknown status"
+    assert _lib.lib().fa_version().decode().count(".") == 2
+
+
+# a fake, 16-byte aligned address: validation must reject before any use
+A = 1 << 20
+MIS = A + 8
+
+
+def fwd(q=A, k=A, v=A, out=A, lse=None, B=1, nq=128, nk=128, H=1, D=64, scale=0.125, causal=0,
+        wl=-1, dt=_lib.FA_FP16):
+    return _lib.lib().fa_fwd(q, k, v, out, lse, B, nq, nk, H, D, scale, causal, wl, dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), _lib.FA_ERR_ARG),
+    (dict(k=None), _lib.FA_ERR_ARG),
+    (dict(out=None), _lib.FA_ERR_ARG),
+    (dict(B=0), _lib.FA_ERR_ARG),
+    (dict(H=0), _lib.FA_ERR_ARG),
+    (dict(nq=-1), _lib.FA_ERR_ARG),
+    (dict(nk=-5), _lib.FA_ERR_ARG),
+    (dict(scale=0.0), _lib.FA_ERR_ARG),
+    (dict(scale=-1.0), _lib.FA_ERR_ARG),
+    (dict(scale=float("inf")), _lib.FA_ERR_ARG),
+    (dict(scale=float("nan")), _lib.FA_ERR_ARG),
+    (dict(causal=2), _lib.FA_ERR_ARG),
+    (dict(wl=-2), _lib.FA_ERR_ARG),
+    (dict(dt=7), _lib.FA_ERR_ARG),
+    (dict(D=96), _lib.FA_ERR_UNSUPPORTED),
+    (dict(D=256), _lib.FA_ERR_UNSUPPORTED),
+    (dict(D=64, dt=_lib.FA_E4M3), _lib.FA_ERR_UNSUPPORTED),
+    (dict(q=MIS), _lib.FA_ERR_ALIGN),
+    (dict(v=MIS), _lib.FA_ERR_ALIGN),
+    (dict(out=MIS), _lib.FA_ERR_ALIGN),
+    (dict(B=1 << 16, H=1 << 8, nq=1 << 16), _lib.FA_ERR_ARG),
+])
+def test_invalid_arguments_rejected_on_host(kw, expect):
+    assert fwd(**kw) == expect
+
+
+def test_empty_query_is_a_no_op():
+    # N_q = 0: nothing to compute, returns before touching the GPU
+    assert fwd(nq=0) == _lib.FA_OK
+
+
+def test_fp8_descales_validated():
+    f = _lib.lib().fa_fwd_fp8
+    assert f(A, A, A, A, None, 1, 128, 128, 1, 128, 0.1, 0, -1, 0.0, 1.0, 1.0, None) == _lib.FA_ERR_ARG
+    assert f(A, A, A, A, None, 1, 128, 128, 1, 128, 0.1, 0, -1, 1.0, float("nan"), 1.0, None) == _lib.FA_ERR_ARG
+    assert f(A, A, A, A, None, 1, 128, 128, 1, 64, 0.1, 0, -1, 1.0, 1.0, 1.0, None) == _lib.FA_ERR_UNSUPPORTED
+
+
+def test_host_entry_rejects_null_host_buffers():
+    f = _lib.lib().fa_fwd_host
+    rc = f(None, A, A, A, None, A, A, A, A, None, 1, 128, 128, 1, 64, 0.1, 0, -1, 0, 1.0, 1.0, 1.0, None)
+    assert rc == _lib.FA_ERR_ARG
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    from exact_attention_136_b200 import forward
+    x = torch.zeros(1, 4, 1, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        forward(x, x, x)

@@ -1,0 +1,215 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small and ragged shapes are compared element by element on every output;
+the full-size workloads (in the launch configuration bench.py times) are
+compared on sampled query rows of every (batch, head).
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_136_b200 import forward, forward_fp8, forward_host, device_status, wait_probe
+from exact_attention_136_b200 import inputs, workloads as W
+from exact_attention_136_b200 import _lib
+from tests.oracle_cmp import TOL_LSE, TOL_O, compare, oracle
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_values.json")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    _lib.lib()  # fails loudly when the library is missing
+
+
+def run(qkv, scale, causal, wl, want_lse=True, stream=None):
+    dev = torch.device("cuda", 0)
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    if q.dtype == torch.float8_e4m3fn:
+        out, lse = forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, scale, causal, wl,
+                               return_lse=want_lse, stream=stream)
+    else:
+        out, lse = forward(q, k, v, scale, causal, wl, return_lse=want_lse, stream=stream)
+    torch.cuda.synchronize()
+    rc, flags = device_status()
+    assert rc == 0, f"device status {rc} flags {flags}"
+    return out, lse
+
+
+def check(qkv, dtype, scale, causal, wl, rows=None):
+    out, lse = run(qkv, scale, causal, wl)
+    ref_o, ref_l = oracle(qkv, scale, causal, wl, rows=rows)
+    d_o, d_l = compare(out, lse, ref_o, ref_l, rows=rows)
+    assert d_o <= TOL_O[dtype], f"max|dO| {d_o:.3e} > {TOL_O[dtype]}"
+    assert d_l <= TOL_LSE, f"max|dLSE| {d_l:.3e} > {TOL_LSE}"
+    return d_o, d_l
+
+
+# (B, N_q, N_k, H, D, dtype, causal, window_left)
+SMALL = [
+    (1, 128, 128, 1, 64, "fp16", False, -1),
+    (1, 128, 128, 1, 128, "bf16", True, -1),
+    (2, 256, 256, 3, 64, "bf16", False, -1),
+    (2, 256, 256, 3, 128, "fp16", True, -1),
+    (1, 1, 1, 2, 128, "bf16", False, -1),
+    (1, 7, 7, 2, 64, "fp16", True, -1),
+    (1, 127, 127, 2, 128, "bf16", True, -1),
+    (1, 129, 129, 2, 64, "bf16", True, -1),
+    (1, 255, 255, 1, 128, "fp16", False, -1),
+    (1, 257, 257, 1, 128, "bf16", True, -1),
+    (2, 300, 300, 2, 64, "fp16", True, -1),
+    (1, 1000, 1000, 2, 128, "bf16", True, -1),
+    (1, 100, 300, 2, 128, "bf16", False, -1),
+    (1, 100, 300, 2, 64, "fp16", True, -1),
+    (1, 300, 100, 2, 128, "bf16", True, -1),
+    (1, 513, 1025, 1, 128, "fp16", True, -1),
+    (1, 1025, 513, 1, 64, "bf16", False, -1),
+    (1, 600, 600, 2, 128, "bf16", True, 0),
+    (1, 600, 600, 2, 128, "bf16", True, 1),
+    (1, 600, 600, 1, 64, "fp16", True, 127),
+    (1, 600, 600, 1, 128, "bf16", True, 128),
+    (1, 600, 600, 1, 128, "fp16", True, 129),
+    (2, 1000, 1000, 2, 128, "bf16", True, 300),
+    (1, 700, 700, 2, 64, "bf16", False, 200),
+    (1, 600, 100, 2, 128, "bf16", True, 50),   # rows >= 151 see no key
+    (1, 1000, 40, 1, 64, "fp16", True, 10),    # whole tiles with no key
+    (1, 512, 512, 1, 128, "e4m3", False, -1),
+    (2, 300, 300, 2, 128, "e4m3", True, -1),
+    (1, 1000, 1000, 1, 128, "e4m3", True, 200),
+    (1, 200, 333, 2, 128, "e4m3", True, -1),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[
+    f"B{c[0]}_q{c[1]}_k{c[2]}_H{c[3]}_D{c[4]}_{c[5]}_{'c' if c[6] else 'nc'}_w{c[7]}" for c in SMALL])
+def test_small_exact_parity(case):
+    B, nq, nk, H, D, dt, causal, wl = case
+    qkv = inputs.make_qkv(B, nq, nk, H, D, dt, seeds=(11 + nq, 12 + nk, 13 + D))
+    check(qkv, dt, 1.0 / math.sqrt(D), causal, wl)
+
+
+@pytest.mark.parametrize("dt,D", [("fp16", 64), ("bf16", 128), ("e4m3", 128)])
+@pytest.mark.parametrize("mult", [4.0, 12.0])
+def test_large_scores_exercise_rescaling(dt, D, mult):
+    """Scores of tens to hundreds (log2 units): the max rises often, O is rescaled in place."""
+    qkv = inputs.make_qkv(1, 700, 700, 2, D, "bf16" if dt == "e4m3" else dt, seeds=(21, 22, 23))
+    if dt == "e4m3":
+        q8, sq = inputs.quantize_e4m3(qkv.q.float() * mult)
+        k8, sk = inputs.quantize_e4m3(qkv.k.float())
+        v8, sv = inputs.quantize_e4m3(qkv.v.float())
+        qkv = inputs.QKV(q8, k8, v8, sq, sk, sv)
+    else:
+        qkv = inputs.QKV((qkv.q.float() * mult).to(qkv.q.dtype), qkv.k, qkv.v)
+    for causal in (False, True):
+        check(qkv, dt, 1.0 / math.sqrt(D), causal, -1)
+
+
+def test_many_units_per_cta():
+    """More work units than SMs: barrier phases carry across units of one CTA."""
+    qkv = inputs.make_qkv(4, 1024, 1024, 32, 64, "fp16", seeds=(31, 32, 33))
+    rows = np.array([0, 1, 127, 128, 255, 256, 511, 700, 1023])
+    for causal in (False, True):
+        check(qkv, "fp16", 0.125, causal, -1, rows=rows)
+
+
+def test_pages_accuracy_check_bound():
+    """The pages' check (B1 H8 N512 D64 fp16, scores / 8) expects max diff < 1e-3."""
+    g = json.load(open(GOLDEN))["accuracy_check"]
+    w = W.WORKLOADS["pr1_b1h8n512d64_fp16"]
+    assert (w.B, w.H, w.n_q, w.D) == (g["batch"], g["heads"], g["seqlen"], g["headdim"])
+    assert w.scale == 1.0 / g["score_divisor"]
+    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=w.seeds)
+    d_o, d_l = check(qkv, "fp16", w.scale, w.causal, w.window_left)
+    assert d_o < g["max_abs_diff_bound"]
+
+
+@pytest.mark.parametrize("name", W.ORDER)
+def test_full_workload_sampled_rows(name):
+    """Every workload at full size; all rows finite, sampled rows of every head vs the oracle."""
+    w = W.WORKLOADS[name]
+    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=w.seeds)
+    rows = W.sample_rows(w, count=64 if w.n_q > 4096 else 256)
+    out, lse = run(qkv, w.scale, w.causal, w.window_left)
+    assert bool(torch.isfinite(out).all()) and bool(torch.isfinite(lse).all())
+    ref_o, ref_l = oracle(qkv, w.scale, w.causal, w.window_left, rows=rows)
+    d_o, d_l = compare(out, lse, ref_o, ref_l, rows=rows)
+    assert d_o <= TOL_O[w.dtype] and d_l <= TOL_LSE, (d_o, d_l)
+
+
+def test_no_keys_gives_zero_and_neg_inf():
+    qkv = inputs.make_qkv(2, 300, 1, 2, 64, "bf16", seeds=(41, 42, 43))
+    dev = torch.device("cuda", 0)
+    k0 = torch.empty((2, 0, 2, 64), dtype=torch.bfloat16, device=dev)
+    out, lse = forward(qkv.q.to(dev), k0, k0.clone(), 0.125)
+    torch.cuda.synchronize()
+    assert bool((out == 0).all()) and bool(torch.isneginf(lse).all())
+
+
+def test_lse_optional_and_guard_regions():
+    """Writes stay inside out / lse: sentinels around both are untouched; lse=NULL works."""
+    dev = torch.device("cuda", 0)
+    B, n, H, D = 1, 333, 3, 128
+    qkv = inputs.make_qkv(B, n, n, H, D, "bf16", seeds=(51, 52, 53))
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    pad = 4096
+    obuf = torch.full((pad + B * n * H * D + pad,), 7.0, dtype=torch.bfloat16, device=dev)
+    lbuf = torch.full((pad + B * H * n + pad,), 7.0, dtype=torch.float32, device=dev)
+    out = obuf[pad:pad + B * n * H * D].view(B, n, H, D)
+    lse = lbuf[pad:pad + B * H * n].view(B, H, n)
+    forward(q, k, v, 1 / math.sqrt(D), True, -1, out=out, lse=lse)
+    out2, none = forward(q, k, v, 1 / math.sqrt(D), True, -1, return_lse=False)
+    torch.cuda.synchronize()
+    assert none is None
+    assert bool((obuf[:pad] == 7).all()) and bool((obuf[-pad:] == 7).all())
+    assert bool((lbuf[:pad] == 7).all()) and bool((lbuf[-pad:] == 7).all())
+    assert torch.equal(out, out2)
+    ref_o, ref_l = oracle(qkv, 1 / math.sqrt(D), True, -1)
+    d_o, d_l = compare(out, lse, ref_o, ref_l)
+    assert d_o <= TOL_O["bf16"] and d_l <= TOL_LSE
+
+
+def test_side_stream_and_determinism():
+    dev = torch.device("cuda", 0)
+    qkv = inputs.make_qkv(2, 777, 777, 4, 128, "fp16", seeds=(61, 62, 63))
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a, la = forward(q, k, v, None, True)
+    b, lb = forward(q, k, v, None, True, stream=s)
+    s.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_host_buffer_entry_point_matches_device_entry():
+    dev = torch.device("cuda", 0)
+    B, n, H, D = 1, 640, 4, 128
+    qkv = inputs.make_qkv(B, n, n, H, D, "bf16", seeds=(71, 72, 73))
+    staging = {"q": torch.empty_like(qkv.q, device=dev), "k": torch.empty_like(qkv.k, device=dev),
+               "v": torch.empty_like(qkv.v, device=dev),
+               "out": torch.empty((B, n, H, D), dtype=torch.bfloat16, device=dev),
+               "lse": torch.empty((B, H, n), dtype=torch.float32, device=dev)}
+    ho, hl = forward_host(qkv.q.pin_memory(), qkv.k.pin_memory(), qkv.v.pin_memory(), staging, 0.09, True)
+    do, dl = forward(qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev), 0.09, True)
+    torch.cuda.synchronize()
+    assert torch.equal(ho, do.cpu()) and torch.equal(hl, dl.cpu())
+
+
+def test_wait_timeout_reports_status_and_context_survives():
+    """A wait that nothing completes ends after its limit with FA_ERR_TIMEOUT; later calls still work."""
+    rc, _ = device_status()
+    assert rc == 0
+    wait_probe(2_000_000)  # 2 ms
+    rc, flags = device_status()
+    assert rc == _lib.FA_ERR_TIMEOUT and flags != 0
+    rc, _ = device_status()
+    assert rc == 0  # the word was cleared
+    qkv = inputs.make_qkv(1, 256, 256, 2, 64, "fp16", seeds=(81, 82, 83))
+    check(qkv, "fp16", 0.125, True, -1)

@@ -1,0 +1,364 @@
+"""Benchmark: exact attention forward TFLOP/s on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one forward over the whole workload (default: causal B4 H32 N8192
+D128 bf16).  `value` is the whole-job TFLOP/s (4*B*H*N_q*N_k*D times the
+fraction of 128x128 blocks with a visible pair, per step, summed over ranks,
+divided by the slowest rank's CUDA-event time for K steps).  Inputs are
+resident in HBM and larger than L2.  `e2e` measures the same metric through
+fa_fwd_host with pinned host buffers, host<->device copies inside the timed
+region.  With N > 1 each rank runs its own batch of the workload (weak
+scaling; the work units are independent, so there is no collective on the
+data path).
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from exact_attention_136_b200 import workloads as W  # noqa: E402
+from exact_attention_136_b200 import inputs  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s and % of dense tensor peak (1×B200) vs CPU oracle"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_TFLOPS = {"fp16": 2250.0, "bf16": 2250.0, "e4m3": 4500.0}
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = ["exact_attention_136_b200/csrc/fa_fwd_kernel.cuh", "exact_attention_136_b200/csrc/sm100.cuh",
+                  "exact_attention_136_b200/csrc/fa_api.cu", "exact_attention_136_b200/csrc/tmap.h"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks(dtype: str):
+    """(peak TF/s for the kernel timed alone, source string, sustained) from MEASURED_PEAKS.json."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    ratio = 2.0 if dtype == "e4m3" else 1.0
+    try:
+        with open(path) as f:
+            mp = json.load(f)
+        return mp["bf16_tflops"] * ratio, "measured", mp.get("bf16_tflops_sustained", None)
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS * ratio, "fallback", None
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel."""
+    path = os.path.join(PROFILE_DIR, "fa_fwd_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = rec.get(workload)
+    if not entry or entry.get("kernel_hash") != kernel_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            text, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            text, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(text)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def oracle_rows_tflops(w: W.Workload, qkv, rows_per_head: int, heads=None):
+    """Time the fp64 oracle on `rows_per_head` sampled rows of each selected (b, h).
+
+    Returns (TFLOP/s-equivalent, seconds, rows, threads).  The FLOP credited per
+    row is the workload's average per row, 4 * N_k * D * block_fraction.
+    """
+    from oracle import attention_ref
+    rows = W.sample_rows(w, count=rows_per_head)
+    heads = heads if heads is not None else [(b, h) for b in range(w.B) for h in range(w.H)]
+    t0 = time.perf_counter()
+    for b, h in heads:
+        q = (qkv.q[b:b + 1, :, h:h + 1].to(torch.float64) * qkv.q_descale).numpy()
+        k = (qkv.k[b:b + 1, :, h:h + 1].to(torch.float64) * qkv.k_descale).numpy()
+        v = (qkv.v[b:b + 1, :, h:h + 1].to(torch.float64) * qkv.v_descale).numpy()
+        attention_ref(q, k, v, w.scale, w.causal, w.window_left, rows=rows)
+    dt = time.perf_counter() - t0
+    per_row = 4.0 * w.n_k * w.D * W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left)
+    n_rows = len(rows) * len(heads)
+    return per_row * n_rows / dt / 1e12, dt, n_rows, blas_threads()
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle, timed on this host's cores."""
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=w.seeds)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    rows_per_step = args.reference_rows
+    for i in range(args.warmup):
+        oracle_rows_tflops(w, qkv, rows_per_step, heads=[heads[i % len(heads)]])
+    total_t = 0.0
+    total_rows = 0
+    t_all = time.perf_counter()
+    for i in range(args.steps):
+        _, dt, n, threads = oracle_rows_tflops(w, qkv, rows_per_step, heads=[heads[i % len(heads)]])
+        total_t += dt
+        total_rows += n
+    wall = time.perf_counter() - t_all
+    per_row = 4.0 * w.n_k * w.D * W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left)
+    value = per_row * total_rows / total_t / 1e12
+    # one full forward of the workload at this throughput
+    ms_per_step = W.flops(w) / (value * 1e12) * 1e3
+    sample = (f"each step: fp64 oracle on {rows_per_step} sampled query rows of one (batch, head), "
+              f"cycling over the {len(heads)} heads; {args.steps} steps took {wall:.1f} s")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "desc": w.desc, "rows_per_step": rows_per_step,
+                   "ms_per_step_note": "one full forward of the workload at the sampled throughput"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=W.HEADLINE, choices=W.ORDER)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-rows", type=int, default=128, help="oracle rows per (batch, head) for cpu_baseline")
+    ap.add_argument("--reference-rows", type=int, default=256, help="oracle rows per step in --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling cases)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_info()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    from exact_attention_136_b200 import _lib, device_status, forward, forward_fp8, forward_host
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    lib = _lib.lib()  # loud failure when the CUDA library is missing
+
+    w = W.WORKLOADS[args.workload]
+    if args.batch is not None:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name}@B{args.batch}")
+    seeds = tuple(s + 7919 * rank for s in w.seeds)   # each rank: its own batch
+    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=seeds)
+    hq, hk, hv = qkv.q.pin_memory(), qkv.k.pin_memory(), qkv.v.pin_memory()
+    q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
+    out_dtype = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+    out = torch.empty((w.B, w.n_q, w.H, w.D), dtype=out_dtype, device=dev)
+    lse = torch.empty((w.B, w.H, w.n_q), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if w.dtype == "e4m3":
+            forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, w.scale, w.causal, w.window_left,
+                        out=out, lse=lse, stream=stream)
+        else:
+            forward(q, k, v, w.scale, w.causal, w.window_left, out=out, lse=lse, stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc, flags = device_status(device=dev)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} flags {flags} after warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    rc, flags = device_status(device=dev)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} flags {flags} in the timed region")
+    if not bool(torch.isfinite(out).all()):
+        raise RuntimeError("non-finite output")
+
+    flops = W.flops(w)
+    ms_per_step = ms / args.steps
+    value = world * flops * args.steps / (ms / 1e3) / 1e12
+    per_launch_tflops = flops / (ms_per_step / 1e3) / 1e12
+
+    # end to end through the host-buffer entry point: H2D inputs, kernel, D2H out + lse
+    ho = torch.empty((w.B, w.n_q, w.H, w.D), dtype=out_dtype, pin_memory=True)
+    hl = torch.empty((w.B, w.H, w.n_q), dtype=torch.float32, pin_memory=True)
+    staging = {"q": q, "k": k, "v": v, "out": out, "lse": lse}
+    desc = (qkv.q_descale, qkv.k_descale, qkv.v_descale)
+    for _ in range(2):
+        forward_host(hq, hk, hv, staging, w.scale, w.causal, w.window_left, desc, ho, hl, stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        forward_host(hq, hk, hv, staging, w.scale, w.causal, w.window_left, desc, ho, hl, stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ems = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ems], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = world * flops * args.e2e_steps / (ems / 1e3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    peak, peak_src, sustained = measured_peaks(w.dtype)
+    traffic = recorded_traffic(w.name)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, dt, n_rows, threads = oracle_rows_tflops(w, qkv, args.cpu_rows)
+        cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 oracle on {args.cpu_rows} sampled query rows of each of the {w.B * w.H} "
+                         f"(batch, head) pairs ({n_rows} rows, {dt:.1f} s); FLOP credited per row = "
+                         f"the workload's average 4*N_k*D*block_fraction"}
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "desc": w.desc, "B": w.B, "N_q": w.n_q, "N_k": w.n_k, "H": w.H,
+                   "D": w.D, "causal": w.causal, "window_left": w.window_left, "scale": w.scale,
+                   "flop_per_step": flops,
+                   "block_fraction": W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left),
+                   "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB vs {L2_BYTES / 1e6:.0f} MB), no flush",
+                   "pct_of_nominal_dense_peak": 100.0 * per_launch_tflops / NOMINAL_TFLOPS[w.dtype],
+                   "nominal_dense_peak_tflops": NOMINAL_TFLOPS[w.dtype],
+                   "parallelism": f"replicas x{world} (independent batches per GPU)"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps, "api": "fa_fwd_host (pinned host buffers)"},
+        "roofline": {"bound": "tensor", "achieved": per_launch_tflops, "peak": peak, "unit": UNIT,
+                     "frac": per_launch_tflops / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 burst" + (" x2 for fp8" if w.dtype == "e4m3" else ""),
+                     "peak_sustained": sustained},
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+        "gpu_launches": args.steps,
+        "kernel_hash": kernel_hash(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

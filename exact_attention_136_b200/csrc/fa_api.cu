@@ -68,6 +68,7 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     ds->attr_set |= (1u << bit);
   }
   const int grid = p.num_units < ds->num_sms ? p.num_units : ds->num_sms;
+  p.rounds = (p.num_units + grid - 1) / grid;
   fa_fwd_kernel<D, DT><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -127,6 +128,20 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   const int64_t units = static_cast<int64_t>(p.pairs) * B * H;
   if (units > 0x7fffffff) return FA_ERR_ARG;
   p.num_units = static_cast<int>(units);
+  // scheduling groups: causal work runs longest-first across a group of
+  // (batch, head) pairs; the group is sized so its K and V (bytes per head:
+  // 2 * N_k * D * element size) take at most ~48 MB of the 126 MB L2 and it
+  // still spans about two waves of units
+  if (causal) {
+    const double kv_head = 2.0 * Nk * D * static_cast<double>(dtype == FA_E4M3 ? 1 : 2);
+    int g = static_cast<int>(48.0e6 / kv_head);
+    const int want = (2 * ds->num_sms + p.pairs - 1) / p.pairs;
+    g = g < want ? g : want;
+    g = g < 1 ? 1 : g;
+    p.group = g < B * H ? g : B * H;
+  } else {
+    p.group = 1;
+  }
   p.wait_limit_ns = g_wait_limit_ns;
   p.status = ds->status;
   switch (dtype * 2 + (D == 128 ? 1 : 0)) {

@@ -53,6 +53,7 @@ enum : int {
   ST_TIMEOUT_MMA = 2,
   ST_TIMEOUT_SOFTMAX = 4,
   ST_TIMEOUT_DRAIN = 8,
+  ST_SMEM_MISALIGNED = 16,
 };
 
 struct FwdParams {
@@ -64,14 +65,18 @@ struct FwdParams {
   float score_scale;   // scale * log2(e) * q_descale * k_descale
   float out_scale;     // v_descale (1 for 16-bit inputs)
   int num_units;
-  int pairs;           // ceil(N_q / 256)
+  int pairs;           // ceil(N_q / 256): work units per (batch, head)
+  int group;           // (batch, head) pairs per scheduling group (see unit_index)
+  int rounds;          // ceil(num_units / gridDim.x)
   unsigned long long wait_limit_ns;
   int* status;         // device status word
 };
 
 constexpr int BLOCK_M = 128;   // query rows per tile
 constexpr int BLOCK_N = 128;   // keys per block
-constexpr int NUM_THREADS = 384;
+constexpr int NUM_THREADS = 640;   // warpgroup 0: load + MMA; 2 warpgroups per Q tile
+constexpr int HEADER_BYTES = 1024;  // mbarriers and flags
+constexpr int XCH_BYTES = 0;        // (no shared-memory exchange)
 
 template <int D, int DT>
 struct Cfg {
@@ -80,12 +85,16 @@ struct Cfg {
   static constexpr int BOX_INNER = 128 / ES;                 // elements per 128-byte row
   static constexpr int NCHUNK = D * ES / 128;                // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = 128 * 128;              // one chunk of 128 rows
-  static constexpr int STAGES = TILE_BYTES >= 32768 ? 4 : 8; // K/V ring slots
+  // K/V ring slots: whatever shared memory is left after the header, the
+  // exchange buffer and Q0, Q1
+  static constexpr int STAGES_FIT = (232448 - HEADER_BYTES - XCH_BYTES - 2 * TILE_BYTES) / TILE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
   static constexpr int KSTEP = DT == DT_E4M3 ? 32 : 16;      // K per MMA instruction
   static constexpr int P_COLS = 128 * ES / 4;                // TMEM columns of one P row
   static constexpr int P_OFF = 64;                           // P column offset inside S_t
   static constexpr int O_COL0 = 256;
-  static constexpr int SMEM_BYTES = 1024 /*barriers*/ + (2 + STAGES) * TILE_BYTES + 1024 /*align*/;
+  // the dynamic shared memory base is 1024-byte aligned (checked at entry)
+  static constexpr int SMEM_BYTES = HEADER_BYTES + XCH_BYTES + (2 + STAGES) * TILE_BYTES;
   static constexpr uint32_t FMT = DT == DT_BF16 ? 1u : 0u;
   static constexpr uint32_t IDESC_S = make_idesc(FMT, false, 128, 128);
   static constexpr uint32_t IDESC_O = make_idesc(FMT, true, 128, D);
@@ -99,50 +108,100 @@ struct Cfg {
 
 struct SharedHeader {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[8], kv_empty[8];
+  uint64_t kv_full[12], kv_empty[12];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(SharedHeader) <= 1024, "header");
+static_assert(sizeof(SharedHeader) <= HEADER_BYTES, "header");
 
+// One 128-row query tile of a work unit and its key-block range.
+struct Tile {
+  int b, h, qs;    // batch, head, first query row
+  int lo, hi;      // inclusive key-block range
+  bool rows;       // tile has rows (qs < N_q)
+  bool valid;      // ... and at least one key block
+};
+
+// Work-unit order.  Units are numbered group by group, a group being
+// `p.group` consecutive (batch, head) pairs whose K and V fit in L2 together;
+// inside a group causal units run longest first (largest query index), and
+// consecutive units switch head so the CTAs working at the same time share
+// each head's K/V blocks through L2.  Non-causal units use groups of one head.
+__device__ __forceinline__ Tile get_tile(int u, int t, const FwdParams& p) {
+  Tile w;
+  const int bh_count = p.B * p.H;
+  const int per_group = p.group * p.pairs;
+  const int g = u / per_group;
+  const int r = u - g * per_group;
+  const int g_heads = min(p.group, bh_count - g * p.group);
+  const int m_idx = r / g_heads;
+  const int bh = g * p.group + (r - m_idx * g_heads);
+  const int m = p.causal ? (p.pairs - 1 - m_idx) : m_idx;
+  w.b = bh / p.H;
+  w.h = bh - w.b * p.H;
+  w.qs = m * (2 * BLOCK_M) + t * BLOCK_M;
+  w.rows = w.qs < p.Nq;
+  const int qe = min(w.qs + BLOCK_M - 1, p.Nq - 1);
+  w.lo = p.window_left >= 0 ? max(0, w.qs - p.window_left) / BLOCK_N : 0;
+  w.hi = p.causal ? min(qe, p.Nk - 1) / BLOCK_N : (p.Nk - 1) / BLOCK_N;
+  w.valid = w.rows && p.Nk > 0 && w.lo <= w.hi;
+  return w;
+}
+
+// Both tiles of a work unit and the union of their key-block ranges.
 struct Unit {
   int b, h, q0;
   int lo[2], hi[2];
-  bool valid[2];   // tile has rows and at least one key block
-  bool rows[2];    // tile has rows (< N_q)
-  int jlo, jhi;    // union of the valid tiles' block ranges
+  bool valid[2];
+  int jlo, jhi;    // empty (jhi < 0) when neither tile has work
 };
 
 __device__ __forceinline__ Unit get_unit(int u, const FwdParams& p) {
+  const Tile a = get_tile(u, 0, p);
+  const Tile c = get_tile(u, 1, p);
   Unit w;
-  const int bh_count = p.B * p.H;
-  const int m_idx = u / bh_count;
-  // causal: longest units (largest query index) first
-  const int m = p.causal ? (p.pairs - 1 - m_idx) : m_idx;
-  const int bh = u - m_idx * bh_count;
-  w.b = bh / p.H;
-  w.h = bh - w.b * p.H;
-  w.q0 = m * (2 * BLOCK_M);
-  w.jlo = 0x7fffffff;
-  w.jhi = -1;
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qs = w.q0 + t * BLOCK_M;
-    w.rows[t] = qs < p.Nq;
-    const int qe = min(qs + BLOCK_M - 1, p.Nq - 1);
-    const int lo = p.window_left >= 0 ? max(0, qs - p.window_left) / BLOCK_N : 0;
-    const int hi = p.causal ? min(qe, p.Nk - 1) / BLOCK_N : (p.Nk - 1) / BLOCK_N;
-    w.lo[t] = lo;
-    w.hi[t] = hi;
-    w.valid[t] = w.rows[t] && p.Nk > 0 && lo <= hi && (!p.causal || qe >= 0);
-    if (w.valid[t]) {
-      w.jlo = min(w.jlo, lo);
-      w.jhi = max(w.jhi, hi);
-    }
-  }
+  w.b = a.b;
+  w.h = a.h;
+  w.q0 = a.qs;
+  w.lo[0] = a.lo; w.hi[0] = a.hi; w.valid[0] = a.valid;
+  w.lo[1] = c.lo; w.hi[1] = c.hi; w.valid[1] = c.valid;
+  w.jlo = a.valid ? a.lo : (c.valid ? c.lo : 0);
+  if (a.valid && c.valid) w.jlo = min(a.lo, c.lo);
+  w.jhi = a.valid ? a.hi : -1;
+  if (c.valid) w.jhi = max(w.jhi, c.hi);
   return w;
+}
+
+// Optional event tracing for timeline studies (off in the library build):
+// lane 0 of one warp per role in CTA 0 stores (event, block, clock) records
+// into its own slice of g_trace with a register counter (no atomics, so the
+// tracer adds no round trip to the traced path).
+#ifdef FA_TRACE_BUILD
+__device__ unsigned long long* g_trace;
+constexpr int kTraceSlice = 16384;
+#define FA_TRACE_DECL unsigned trace_n = 0
+#define FA_TRACE(who, ev, j)                                                                          \
+  do {                                                                                                \
+    if (blockIdx.x == 0 && ((who) >= 2 || (threadIdx.x & 127) == 0) && g_trace && trace_n < kTraceSlice) \
+      g_trace[(who) * kTraceSlice + trace_n++] =                                                      \
+          (static_cast<unsigned long long>((ev) & 0xff) << 48) |                                     \
+          (static_cast<unsigned long long>((j) & 0xffff) << 32) |                                    \
+          (static_cast<unsigned long long>(clock64()) & 0xffffffffull);                              \
+  } while (0)
+#else
+#define FA_TRACE_DECL do { } while (0)
+#define FA_TRACE(who, ev, j) do { } while (0)
+#endif
+
+// The k-th unit of this CTA: rounds of gridDim.x units, assigned forward in
+// even rounds and backward in odd ones (longest-first lists then balance).
+// Returns a value >= num_units when this CTA has no unit in round k.
+__device__ __forceinline__ int unit_index(int k, const FwdParams& p) {
+  const int i = (k & 1) ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
+                        : static_cast<int>(blockIdx.x);
+  return k * static_cast<int>(gridDim.x) + i;
 }
 
 __device__ __forceinline__ void record_error(SharedHeader* sh, const FwdParams& p, int code) {
@@ -154,8 +213,17 @@ __device__ __forceinline__ bool aborted(SharedHeader* sh) {
   return *reinterpret_cast<volatile int*>(&sh->abort_flag) != 0;
 }
 
-__device__ __forceinline__ void setmaxnreg_dec80() { asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n"); }
-__device__ __forceinline__ void setmaxnreg_inc208() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n"); }
+// Register split between warpgroup 0 (one producer and one MMA thread) and
+// the four softmax warpgroups.  The launch gives every thread 96 registers
+// (640 threads, one CTA per SM: 61440 of the SM's 65536); the split must not
+// exceed that total: 128 * REGS_LOAD_MMA + 512 * REGS_SOFTMAX <= 61440.
+constexpr int REGS_LOAD_MMA = 64;
+constexpr int REGS_SOFTMAX = 104;
+static_assert(128 * REGS_LOAD_MMA + 512 * REGS_SOFTMAX <= NUM_THREADS * 96, "register split");
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N)); }
 
 // ------------------------------------------------------------------ producer
 template <int D, int DT>
@@ -170,10 +238,13 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
   uint32_t phase_mask = 0;    // bit s: parity of slot s's latest load
   bool q_outstanding = false;
   bool ok = true;
+  FA_TRACE_DECL;
   const uint64_t pol_kv = policy_evict_last();
   const uint64_t pol_q = policy_evict_first();
 
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  for (int k = 0; k < p.rounds && ok; ++k) {
+    const int u = unit_index(k, p);
+    if (u >= p.num_units) continue;
     const Unit w = get_unit(u, p);
     if (w.jhi < 0) continue;
     if (aborted(sh)) { ok = false; break; }
@@ -190,6 +261,18 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
                          c * C::BOX_INNER, w.h, w.q0 + t * BLOCK_M, w.b, pol_q);
     q_outstanding = true;
     ++q_uses;
+    // warm L2 with the Q tiles of this CTA's next unit
+    {
+      const int un = unit_index(k + 1, p);
+      if (k + 1 < p.rounds && un < p.num_units) {
+        const Unit wn = get_unit(un, p);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_prefetch_l2_4d(mq, c * C::BOX_INNER, wn.h, wn.q0 + t * BLOCK_M, wn.b);
+      }
+    }
     // K_j, V_j for the union of the tiles' block ranges
     for (int j = w.jlo; j <= w.jhi && ok; ++j) {
 #pragma unroll
@@ -199,6 +282,7 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
         if (!mbar_wait(smem_u32(&sh->kv_empty[slot]), (round & 1u) ^ 1u, p.wait_limit_ns)) {
           record_error(sh, p, ST_TIMEOUT_LOAD); ok = false; break;
         }
+        FA_TRACE(3, 1 + kv, j);
         const uint32_t bar = smem_u32(&sh->kv_full[slot]);
         mbar_arrive_expect_tx(bar, C::TILE_BYTES);
         const CUtensorMap* map = kv == 0 ? mk : mv;
@@ -225,31 +309,42 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
 }
 
 // ------------------------------------------------------------------ MMA issuer
+// Opaque copy: keeps the compiler from hoisting per-iteration address math
+// (and the descriptors built from it) out of the key-block loop, which would
+// hold dozens of 64-bit descriptors in registers.
+__device__ __forceinline__ uint32_t opaque(uint32_t x) {
+  asm volatile("mov.b32 %0, %0;" : "+r"(x));
+  return x;
+}
+
 template <int D, int DT>
 __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
   using C = Cfg<D, DT>;
+  // K-major 128B-swizzled Q and K tiles: 8-row groups 1024 B apart; the K
+  // step advances 32 B inside a 128-byte row, then jumps to the next chunk.
+  const uint64_t a0 = sdesc_sw128(q_addr, 16, 1024);
+  const uint64_t b0 = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < D / C::KSTEP; ++kk) {
     const int byte = kk * C::KSTEP * C::ES;
-    const int off = (byte / 128) * C::CHUNK_BYTES + (byte % 128);
-    const uint64_t a = sdesc_sw128(q_addr + off, 16, 1024);
-    const uint64_t b = sdesc_sw128(k_addr + off, 16, 1024);
-    if constexpr (DT == DT_E4M3) mma_f8_ss(d_tmem, a, b, C::IDESC_S, kk > 0);
-    else mma_f16_ss(d_tmem, a, b, C::IDESC_S, kk > 0);
+    const uint64_t off = static_cast<uint64_t>(((byte / 128) * C::CHUNK_BYTES + (byte % 128)) >> 4);
+    if constexpr (DT == DT_E4M3) mma_f8_ss(d_tmem, a0 + off, b0 + off, C::IDESC_S, kk > 0);
+    else mma_f16_ss(d_tmem, a0 + off, b0 + off, C::IDESC_S, kk > 0);
   }
 }
 
 template <int D, int DT>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, bool accumulate) {
   using C = Cfg<D, DT>;
+  // V tile is MN-major (head dim contiguous): 8-key groups 1024 B apart,
+  // 128-byte head-dim chunks CHUNK_BYTES apart.
+  const uint64_t b0 = sdesc_sw128(v_addr, C::CHUNK_BYTES, 1024);
 #pragma unroll
   for (int kk = 0; kk < BLOCK_N / C::KSTEP; ++kk) {
-    // V tile is MN-major (head dim contiguous): 8-key groups 1024 B apart,
-    // 128-byte head-dim chunks CHUNK_BYTES apart.
-    const uint64_t b = sdesc_sw128(v_addr + kk * C::KSTEP * 128, C::CHUNK_BYTES, 1024);
+    const uint64_t off = static_cast<uint64_t>((kk * C::KSTEP * 128) >> 4);
     const uint32_t a = p_tmem + kk * (C::KSTEP * C::ES / 4);
-    if constexpr (DT == DT_E4M3) mma_f8_ts(d_tmem, a, b, C::IDESC_O, accumulate || kk > 0);
-    else mma_f16_ts(d_tmem, a, b, C::IDESC_O, accumulate || kk > 0);
+    if constexpr (DT == DT_E4M3) mma_f8_ts(d_tmem, a, b0 + off, C::IDESC_O, accumulate || kk > 0);
+    else mma_f16_ts(d_tmem, a, b0 + off, C::IDESC_O, accumulate || kk > 0);
   }
 }
 
@@ -266,8 +361,11 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
   const uint32_t s_tmem[2] = {tbase, tbase + 128};
   const uint32_t p_tmem[2] = {tbase + C::P_OFF, tbase + 128 + C::P_OFF};
   const uint32_t o_tmem[2] = {tbase + C::O_COL0, tbase + C::O_COL0 + D};
+  FA_TRACE_DECL;
 
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  for (int k = 0; k < p.rounds && ok; ++k) {
+    const int u = unit_index(k, p);
+    if (u >= p.num_units) continue;
     const Unit w = get_unit(u, p);
     if (w.jhi < 0) continue;
     if (aborted(sh)) { ok = false; break; }
@@ -276,32 +374,39 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
     }
     ++q_uses;
     for (int j = w.jlo; j <= w.jhi + 1 && ok; ++j) {
-      uint32_t kslot = 0, vslot = 0;
-      if (j <= w.jhi) {
-        const uint32_t idx = kv_base + 2u * (j - w.jlo);
-        kslot = idx % C::STAGES;
-        if (!mbar_wait(smem_u32(&sh->kv_full[kslot]), (idx / C::STAGES) & 1u, p.wait_limit_ns)) {
-          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
-        }
-      }
-      if (j > w.jlo) {
-        const uint32_t idx = kv_base + 2u * (j - 1 - w.jlo) + 1u;
-        vslot = idx % C::STAGES;
-        if (!mbar_wait(smem_u32(&sh->kv_full[vslot]), (idx / C::STAGES) & 1u, p.wait_limit_ns)) {
-          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
-        }
-      }
-      tc_fence_after();
+      // K_j feeds S_0(j), S_1(j); V_{j-1} feeds PV_0(j-1), PV_1(j-1).  Each
+      // is waited for right before its first MMA and its ring slot released
+      // right after its last one, so a late K never holds back a PV.
+      const bool has_k = j <= w.jhi;
+      const bool has_v = j > w.jlo;
+      const uint32_t kidx = kv_base + 2u * (j - w.jlo);
+      const uint32_t vidx = kidx - 1u;
+      const uint32_t kslot = kidx % C::STAGES;
+      const uint32_t vslot = vidx % C::STAGES;
+      bool k_ready = false, v_ready = false, k_done = !has_k, v_done = !has_v;
+      const int jp = j - 1;
+      const bool pv_use[2] = {w.valid[0] && jp >= w.lo[0] && jp <= w.hi[0],
+                              w.valid[1] && jp >= w.lo[1] && jp <= w.hi[1]};
+      const bool s_use[2] = {w.valid[0] && j >= w.lo[0] && j <= w.hi[0],
+                             w.valid[1] && j >= w.lo[1] && j <= w.hi[1]};
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (!w.valid[t]) continue;
-        const int jp = j - 1;
-        if (jp >= w.lo[t] && jp <= w.hi[t]) {
+        if (pv_use[t]) {
           // O_t += P_t(j-1) V_{j-1}
+          if (!v_ready) {
+            FA_TRACE(2, 10, jp);
+            if (!mbar_wait(smem_u32(&sh->kv_full[vslot]), (vidx / C::STAGES) & 1u, p.wait_limit_ns)) {
+              record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+            }
+            v_ready = true;
+            FA_TRACE(2, 8, jp);
+          }
+          FA_TRACE(2, 11 + t, jp);
           if (!mbar_wait(smem_u32(&sh->p_full[t]), p_waits[t] & 1u, p.wait_limit_ns)) {
             record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
           }
           ++p_waits[t];
+          FA_TRACE(2, 1 + 3 * t, jp);
           if (jp == w.lo[t]) {
             // O_t must have been read out by the previous unit's epilogue
             if (!mbar_wait(smem_u32(&sh->o_empty[t]), (o_units[t] & 1u) ^ 1u, p.wait_limit_ns)) {
@@ -310,20 +415,50 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
           }
           tc_fence_after();
           issue_pv<D, DT>(o_tmem[t], p_tmem[t], ring + vslot * C::TILE_BYTES, jp > w.lo[t]);
+          FA_TRACE(2, 2 + 3 * t, jp);
           if (jp == w.hi[t]) {
             mma_commit(smem_u32(&sh->o_full[t]));
             ++o_units[t];
           }
+          if (t == 1 || !pv_use[1]) {
+            mma_commit(smem_u32(&sh->kv_empty[vslot]));   // last reader of V_{j-1}
+            v_done = true;
+          }
         }
-        if (j >= w.lo[t] && j <= w.hi[t]) {
+        if (s_use[t]) {
           // S_t(j) = Q_t K_j^T   (issued after PV_t(j-1), which read P_t from these columns)
-          issue_s<D, DT>(s_tmem[t], sq + t * C::TILE_BYTES, ring + kslot * C::TILE_BYTES);
+          if (!k_ready) {
+            FA_TRACE(2, 9, j);
+            if (!mbar_wait(smem_u32(&sh->kv_full[kslot]), (kidx / C::STAGES) & 1u, p.wait_limit_ns)) {
+              record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+            }
+            k_ready = true;
+            FA_TRACE(2, 7, j);
+            tc_fence_after();
+          }
+          issue_s<D, DT>(s_tmem[t], opaque(sq) + t * C::TILE_BYTES, ring + kslot * C::TILE_BYTES);
           mma_commit(smem_u32(&sh->s_full[t]));
+          FA_TRACE(2, 3 + 3 * t, j);
+          if (t == 1 || !s_use[1]) {
+            mma_commit(smem_u32(&sh->kv_empty[kslot]));   // last reader of K_j
+            k_done = true;
+          }
         }
       }
       if (!ok) break;
-      if (j <= w.jhi) mma_commit(smem_u32(&sh->kv_empty[kslot]));
-      if (j > w.jlo) mma_commit(smem_u32(&sh->kv_empty[vslot]));
+      // a loaded block nobody read (not expected): release it once it has landed
+      if (!k_done) {
+        if (!mbar_wait(smem_u32(&sh->kv_full[kslot]), (kidx / C::STAGES) & 1u, p.wait_limit_ns)) {
+          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+        }
+        mma_commit(smem_u32(&sh->kv_empty[kslot]));
+      }
+      if (!v_done) {
+        if (!mbar_wait(smem_u32(&sh->kv_full[vslot]), (vidx / C::STAGES) & 1u, p.wait_limit_ns)) {
+          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+        }
+        mma_commit(smem_u32(&sh->kv_empty[vslot]));
+      }
     }
     if (!ok) break;
     mma_commit(smem_u32(&sh->q_empty));
@@ -352,6 +487,12 @@ __device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float 
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
+// Two e4m3 values (low 16 bits) back to fp32.
+__device__ __forceinline__ float2 unpack2_e4m3(uint32_t bits) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(bits), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
 template <int DT>
 __device__ __forceinline__ void store_out_row16(void* dst, const float* o, float inv) {
   // 16 values -> two 16-byte stores
@@ -368,76 +509,167 @@ __device__ __forceinline__ void store_out_row16(void* dst, const float* o, float
   reinterpret_cast<uint4*>(dst)[1] = v1;
 }
 
+// 2^x on the FMA pipe for a pair of finite x (unmasked blocks only).
+// Range reduction for base 2 is exact: x = j + f with j = round(x) and
+// f in [-1/2, 1/2]; 2^j is added into the exponent field and 2^f is a cubic
+// fitted by the Remez exchange on relative error (csrc/gen_exp2_poly.py:
+// max relative error 7.5e-5, below the 16-bit P rounding).  x is clamped to
+// -125 first so 2^j stays a normal number; those terms are < 2^-124.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                        make_float2(0.2426111251115799f, 0.2426111251115799f));
+  q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  q = __ffma2_rn(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  // t's low mantissa bits hold j; shifting by 23 moves j into the exponent field
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Exponentiate this thread's 64 scores of a row, write P (16-bit or e4m3)
+// into TMEM at p_addr (16x32bx2 layout: lanes 0-15 of the access for
+// threads 0-15, the same lanes half a row of P further for threads 16-31)
+// and return their fp32 sum twice: exact, and over the values P*V uses
+// (different only for e4m3, whose 3-bit mantissa would otherwise bias O).  EMULATE: pairs 5-7 of every 8 go through
+// exp2_poly2 (37.5% of the exponentials on the FMA pipe, which balances the
+// 16/clk MUFU against the 128/clk FMA pipe).
+template <int DT, bool EMULATE>
+__device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_mref, uint32_t p_addr) {
+  const float2 cc2 = make_float2(cc, cc);
+  const float2 nm2 = make_float2(neg_mref, neg_mref);
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 accq = make_float2(0.f, 0.f);   // e4m3 only: sum of the rounded values
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t pw[8];
+    float2 prev = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int c = q * 16 + 2 * i;
+      const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), cc2, nm2);
+      float2 e;
+      if (EMULATE && i >= 5) {
+        e = exp2_poly2(x);
+      } else {
+        e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
+      acc[i & 1] = __fadd2_rn(acc[i & 1], e);
+      if constexpr (DT == DT_E4M3) {
+        if (i & 1) {
+          pw[i / 2] = pack4_e4m3(prev.x, prev.y, e.x, e.y);
+          accq = __fadd2_rn(accq, __fadd2_rn(unpack2_e4m3(pw[i / 2] & 0xffffu), unpack2_e4m3(pw[i / 2] >> 16)));
+        } else {
+          prev = e;
+        }
+      } else {
+        pw[i] = pack2<DT>(e.x, e.y);
+      }
+    }
+    if constexpr (DT == DT_E4M3) {
+      tmem_st_16x32bx2_x4<16>(p_addr + q * 4, pw);   // 16 e4m3 values = 4 columns
+    } else {
+      tmem_st_16x32bx2_x8<32>(p_addr + q * 8, pw);
+    }
+  }
+  const float2 a = __fadd2_rn(acc[0], acc[1]);
+  const float exact = a.x + a.y;
+  // (exact sum for the log-sum-exp, sum of the values P*V uses for O)
+  return make_float2(exact, DT == DT_E4M3 ? accq.x + accq.y : exact);
+}
+
+// Softmax role.  Eight warps per Q tile t; warp (quad, sub) owns the 16
+// rows 32*quad + 16*sub .. +15 (TMEM lanes), and inside the warp lanes 0-15
+// take score columns [0, 64) of those rows, lanes 16-31 columns [64, 128)
+// (the tcgen05 16x32bx2 access shape), so the two halves of a row meet with
+// one shuffle and apply identical references and rescale factors.
 template <int D, int DT>
-__device__ void softmax_role(SharedHeader* sh, uint32_t tbase, int t, const FwdParams& p) {
+__device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, const int sub, const FwdParams& p) {
   using C = Cfg<D, DT>;
-  const int warp_in_wg = (threadIdx.x / 32) & 3;
-  const int r = warp_in_wg * 32 + (int)lane_id();      // row in tile == TMEM lane
-  const uint32_t lane_off = static_cast<uint32_t>(warp_in_wg * 32) << 16;
-  const uint32_t s_col = tbase + lane_off + t * 128;
-  const uint32_t p_col = s_col + C::P_OFF;
-  const uint32_t o_col = tbase + lane_off + C::O_COL0 + t * D;
+  constexpr int HALF_N = BLOCK_N / 2;
+  constexpr int HALF_D = D / 2;
+  const int quad = (threadIdx.x / 32) & 3;
+  const int half = static_cast<int>(lane_id()) >> 4;
+  const int r = quad * 32 + sub * 16 + (static_cast<int>(lane_id()) & 15);   // row in tile
+  const uint32_t lane_off = static_cast<uint32_t>(quad * 32 + sub * 16) << 16;
+  const uint32_t s_addr = tbase + lane_off + t * 128;
+  const uint32_t p_addr = tbase + lane_off + t * 128 + C::P_OFF;
+  const uint32_t o_addr = tbase + lane_off + C::O_COL0 + t * D;
   const float cc = p.score_scale;
+  FA_TRACE_DECL;
   uint32_t s_waits = 0, units = 0;
   bool ok = true;
   constexpr int OUT_ES = 2;
 
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-    const Unit w = get_unit(u, p);
-    if (!w.rows[t]) continue;
-    const int row = w.q0 + t * BLOCK_M + r;
+  for (int k = 0; k < p.rounds && ok; ++k) {
+    const int u = unit_index(k, p);
+    if (u >= p.num_units) continue;
+    const Tile w = get_tile(u, t, p);
+    if (!w.rows) continue;
+    const int row = w.qs + r;
     const bool row_ok = row < p.Nq;
-    uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) +
-                       ((static_cast<int64_t>(w.b) * p.Nq + row) * p.H + w.h) * (int64_t)D * OUT_ES;
-    float* lse_ptr = p.lse ? p.lse + (static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row : nullptr;
-    if (!w.valid[t]) {
+    if (!w.valid) {
       // no visible key for any row of this tile
       if (row_ok) {
+        uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) +
+                           ((static_cast<int64_t>(w.b) * p.Nq + row) * p.H + w.h) * (int64_t)D * OUT_ES;
         float z[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) z[i] = 0.f;
 #pragma unroll
-        for (int c = 0; c < D; c += 16) store_out_row16<DT>(out_row + c * OUT_ES, z, 0.f);
-        if (lse_ptr) *lse_ptr = -INFINITY;
+        for (int c = 0; c < HALF_D; c += 16) store_out_row16<DT>(out_row + (half * HALF_D + c) * OUT_ES, z, 0.f);
+        if (p.lse && half == 0) p.lse[(static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row] = -INFINITY;
       }
       continue;
     }
     if (aborted(sh)) { ok = false; break; }
     float m_used = -INFINITY;   // reference max (log2 units) that P and l are taken against
-    float l = 0.f;
-    for (int j = w.lo[t]; j <= w.hi[t]; ++j) {
+    float l = 0.f;              // this thread's share of the row sum (exact)
+    float lq = 0.f;             // ... of the stored P values (differs for e4m3)
+    for (int j = w.lo; j <= w.hi; ++j) {
       bool got = mbar_wait(smem_u32(&sh->s_full[t]), s_waits & 1u, p.wait_limit_ns);
       got = __all_sync(0xffffffffu, got);
       if (!got) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
       ++s_waits;
       tc_fence_after();
-      float s[BLOCK_N];
-      tmem_ld32(s_col + 0, reinterpret_cast<uint32_t*>(s + 0));
-      tmem_ld32(s_col + 32, reinterpret_cast<uint32_t*>(s + 32));
-      tmem_ld32(s_col + 64, reinterpret_cast<uint32_t*>(s + 64));
-      tmem_ld32(s_col + 96, reinterpret_cast<uint32_t*>(s + 96));
+      FA_TRACE(t, 1, j);
+      float s[HALF_N];
+      tmem_ld_16x32bx2_x32<64>(s_addr + 0, reinterpret_cast<uint32_t*>(s + 0));
+      tmem_ld_16x32bx2_x32<64>(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
       tmem_wait_ld();
+      FA_TRACE(t, 2, j);
       // mask boundary blocks (causal diagonal, window edge, key tail)
       const int k0 = j * BLOCK_N;
-      const int qs = w.q0 + t * BLOCK_M;
-      const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > qs) ||
-                             (p.window_left >= 0 && k0 < qs + BLOCK_M - 1 - p.window_left);
+      const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
+                             (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
       if (need_mask) {
-        const int hi_c = min(p.Nk - k0, p.causal ? row - k0 + 1 : BLOCK_N);
-        const int lo_c = p.window_left >= 0 ? row - p.window_left - k0 : 0;
+        const int kh = k0 + half * HALF_N;
+        const int hi_c = min(p.Nk - kh, p.causal ? row - kh + 1 : HALF_N);
+        const int lo_c = p.window_left >= 0 ? row - p.window_left - kh : 0;
 #pragma unroll
-        for (int c = 0; c < BLOCK_N; ++c)
+        for (int c = 0; c < HALF_N; ++c)
           if (c < lo_c || c >= hi_c) s[c] = -INFINITY;
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      // half-row max (8 chains of 3-input max), then the other half's lane
+      float mx8[8];
 #pragma unroll
-      for (int c = 4; c < BLOCK_N; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(s[q], s[8 + q]);
+#pragma unroll
+      for (int c = 16; c < HALF_N; c += 16)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx8[q] = fmax3(mx8[q], s[c + q], s[c + 8 + q]);
+      const float mx_half = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+      const float mx = fmaxf(mx_half, __shfl_xor_sync(0xffffffffu, mx_half, 16));
       const float m_blk = mx * cc;   // -inf stays -inf (cc > 0)
       const float m_cand = fmaxf(m_used, m_blk);
       const bool need = m_cand > m_used + C::RESCALE_THRESHOLD;
@@ -449,82 +681,62 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, int t, const FwdP
         m_used = m_cand;
       }
       const float mref = (m_used == -INFINITY) ? 0.f : (m_used - C::PSHIFT);
-      const float neg_mref = -mref;
-      float l0 = 0.f, l1 = 0.f;
-      if constexpr (DT == DT_E4M3) {
+      FA_TRACE(t, 3, j);
+      const float2 lsum = need_mask ? exp_half<DT, false>(s, cc, -mref, p_addr)
+                                    : exp_half<DT, true>(s, cc, -mref, p_addr);
+      FA_TRACE(t, 4, j);
+      // O rescale of this thread's half row (only when some row of this warp
+      // raised its reference); PV_t(j-1) has completed: S_t(j) was issued
+      // after it and has landed.
+      if (warp_rescale && j > w.lo) {
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pw[16];
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            const int cb = half * 64 + c;
-            const float e0 = ex2_approx(fmaf(s[cb], cc, neg_mref));
-            const float e1 = ex2_approx(fmaf(s[cb + 1], cc, neg_mref));
-            const float e2 = ex2_approx(fmaf(s[cb + 2], cc, neg_mref));
-            const float e3 = ex2_approx(fmaf(s[cb + 3], cc, neg_mref));
-            l0 += e0 + e1;
-            l1 += e2 + e3;
-            pw[c / 4] = pack4_e4m3(e0, e1, e2, e3);
-          }
-          tmem_st16(p_col + half * 16, pw);
-        }
-      } else {
-#pragma unroll
-        for (int quarter = 0; quarter < 4; ++quarter) {
-          uint32_t pw[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float e0 = ex2_approx(fmaf(s[quarter * 32 + c], cc, neg_mref));
-            const float e1 = ex2_approx(fmaf(s[quarter * 32 + c + 1], cc, neg_mref));
-            l0 += e0;
-            l1 += e1;
-            pw[c / 2] = pack2<DT>(e0, e1);
-          }
-          tmem_st16(p_col + quarter * 16, pw);
-        }
-      }
-      // O rescale (only when some row of this warp raised its reference);
-      // PV_t(j-1) has completed: S_t(j) was issued after it and has landed.
-      if (warp_rescale && j > w.lo[t]) {
-#pragma unroll
-        for (int c = 0; c < D; c += 16) {
+        for (int c = 0; c < HALF_D; c += 16) {
           uint32_t o[16];
-          tmem_ld16(o_col + c, o);
+          tmem_ld_16x32bx2_x16<HALF_D>(o_addr + c, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(o_col + c, o);
+          for (int i = 0; i < 16; i += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+            o[i] = __float_as_uint(v.x);
+            o[i + 1] = __float_as_uint(v.y);
+          }
+          tmem_st_16x32bx2_x16<HALF_D>(o_addr + c, o);
         }
       }
-      l = l * alpha;
-      l += l0 + l1;
+      l = fmaf(l, alpha, lsum.x);
+      lq = fmaf(lq, alpha, lsum.y);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&sh->p_full[t]));
+      FA_TRACE(t, 5, j);
     }
     if (!ok) break;
-    // epilogue: O / l, LSE
+    // epilogue: O / l, LSE; l is the sum of both half rows
+    const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+    const float lq_row = lq + __shfl_xor_sync(0xffffffffu, lq, 16);
     bool got = mbar_wait(smem_u32(&sh->o_full[t]), units & 1u, p.wait_limit_ns);
     got = __all_sync(0xffffffffu, got);
     if (!got) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
     ++units;
     tc_fence_after();
-    const float inv = (l > 0.f ? 1.f / l : 0.f) * p.out_scale;
+    const float inv = (lq_row > 0.f ? 1.f / lq_row : 0.f) * p.out_scale;
+    uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) +
+                       ((static_cast<int64_t>(w.b) * p.Nq + row) * p.H + w.h) * (int64_t)D * OUT_ES +
+                       half * HALF_D * OUT_ES;
 #pragma unroll
-    for (int c = 0; c < D; c += 32) {
-      uint32_t o[32];
-      tmem_ld32(o_col + c, o);
+    for (int c = 0; c < HALF_D; c += 16) {
+      uint32_t o[16];
+      tmem_ld_16x32bx2_x16<HALF_D>(o_addr + c, o);
       tmem_wait_ld();
-      if (row_ok) {
-        store_out_row16<DT>(out_row + c * OUT_ES, reinterpret_cast<float*>(o), inv);
-        store_out_row16<DT>(out_row + (c + 16) * OUT_ES, reinterpret_cast<float*>(o) + 16, inv);
-      }
+      if (row_ok) store_out_row16<DT>(out_row + c * OUT_ES, reinterpret_cast<float*>(o), inv);
     }
     tc_fence_before();
     mbar_arrive(smem_u32(&sh->o_empty[t]));
-    if (row_ok && lse_ptr) {
+    if (row_ok && p.lse && half == 0) {
       // natural log of sum_j exp(scale * s_j) = (m_used + log2(l) - PSHIFT) * ln 2
-      *lse_ptr = l > 0.f ? (m_used + __log2f(l) - C::PSHIFT) * 0.69314718055994531f : -INFINITY;
+      p.lse[(static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row] =
+          l_row > 0.f ? (m_used + __log2f(l_row) - C::PSHIFT) * 0.69314718055994531f : -INFINITY;
     }
   }
 }
@@ -535,10 +747,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = Cfg<D, DT>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    // 128-byte swizzled tiles need 1024-byte alignment; never expected
+    if (threadIdx.x == 0) atomicOr(p.status, ST_SMEM_MISALIGNED);
+    return;
+  }
   SharedHeader* sh = reinterpret_cast<SharedHeader*>(smem);
-  uint8_t* tiles = smem + 1024;
+  uint8_t* tiles = smem + HEADER_BYTES + XCH_BYTES;
   const int warp = threadIdx.x / 32;
 
   if (threadIdx.x == 0) {
@@ -550,9 +766,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&sh->s_full[t]), 1);
-      mbar_init(smem_u32(&sh->p_full[t]), 128);
+      mbar_init(smem_u32(&sh->p_full[t]), 256);
       mbar_init(smem_u32(&sh->o_full[t]), 1);
-      mbar_init(smem_u32(&sh->o_empty[t]), 128);
+      mbar_init(smem_u32(&sh->o_empty[t]), 256);
     }
     mbar_init(smem_u32(&sh->mma_done), 1);
     sh->abort_flag = 0;
@@ -571,12 +787,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tbase = sh->tmem_base;
 
   if (warp < 4) {
-    setmaxnreg_dec80();
+    setmaxnreg_dec<REGS_LOAD_MMA>();
     if (warp == 0 && lane_id() == 0) producer_role<D, DT>(sh, tiles, &tm_q, &tm_k, &tm_v, p);
     else if (warp == 1 && lane_id() == 0) mma_role<D, DT>(sh, tiles, tbase, p);
   } else {
-    setmaxnreg_inc208();
-    softmax_role<D, DT>(sh, tbase, warp < 8 ? 0 : 1, p);
+    setmaxnreg_inc<REGS_SOFTMAX>();
+    // warps 4-11: tile 0, warps 12-19: tile 1; within a tile the first four
+    // warps take the upper 16 rows of each lane quadrant, the next four the lower
+    const int t = warp < 12 ? 0 : 1;
+    const int sub = ((warp - 4) >> 2) & 1;
+    softmax_role<D, DT>(sh, tbase, t, sub, p);
   }
   tc_fence_before();
   __syncthreads();

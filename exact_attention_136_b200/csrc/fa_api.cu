@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/fa.h"
 #include "fa_fwd_kernel.cuh"
@@ -17,11 +18,20 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Scheduler scratch: one {next unit, finished CTAs} pair of counters per
+// stream, from a pool allocated once per device.  Launches on one stream run
+// in order, launches on different streams use different counters, and each
+// launch leaves its counters at zero.
+constexpr int kSchedSlots = 256;
+
 struct DeviceState {
   bool init = false;
   int num_sms = 0;
   int* status = nullptr;     // device address of g_status_word
   unsigned attr_set = 0;     // bit per kernel instantiation
+  unsigned* sched_pool = nullptr;
+  std::unordered_map<cudaStream_t, int> sched_slot;
+  int next_slot = 0;
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -43,6 +53,30 @@ int device_state(DeviceState** out) {
     }
   }
   *out = &s;
+  return FA_OK;
+}
+
+int sched_counters(DeviceState* ds, cudaStream_t stream, unsigned** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!ds->sched_pool) {
+    unsigned* pool = nullptr;
+    const size_t bytes = sizeof(unsigned) * 2 * kSchedSlots;
+    if (cudaMalloc(&pool, bytes) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaMemset(pool, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaFree(pool);
+      return FA_ERR_CUDA;
+    }
+    ds->sched_pool = pool;
+  }
+  auto it = ds->sched_slot.find(stream);
+  int slot;
+  if (it != ds->sched_slot.end()) {
+    slot = it->second;
+  } else {
+    slot = ds->next_slot++ % kSchedSlots;
+    ds->sched_slot[stream] = slot;
+  }
+  *out = ds->sched_pool + 2 * slot;
   return FA_OK;
 }
 
@@ -68,7 +102,8 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     ds->attr_set |= (1u << bit);
   }
   const int grid = p.num_units < ds->num_sms ? p.num_units : ds->num_sms;
-  p.rounds = (p.num_units + grid - 1) / grid;
+  int rc = sched_counters(ds, stream, &p.sched);
+  if (rc != FA_OK) return rc;
   fa_fwd_kernel<D, DT><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -66,8 +66,9 @@ struct FwdParams {
   float out_scale;     // v_descale (1 for 16-bit inputs)
   int num_units;
   int pairs;           // ceil(N_q / 256): work units per (batch, head)
-  int group;           // (batch, head) pairs per scheduling group (see unit_index)
-  int rounds;          // ceil(num_units / gridDim.x)
+  int group;           // (batch, head) pairs per scheduling group (see get_tile)
+  unsigned* sched;     // [2] scheduler scratch: next unit to claim, CTAs finished;
+                       // zero between launches (the last CTA resets it)
   unsigned long long wait_limit_ns;
   int* status;         // device status word
 };
@@ -111,6 +112,8 @@ struct SharedHeader {
   uint64_t kv_full[12], kv_empty[12];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_done;
+  uint64_t uq_full[4], uq_empty[4];   // unit queue: producer -> MMA + softmax warps
+  int uq[4];                          // claimed unit ids, -1 = no more work
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -195,13 +198,18 @@ constexpr int kTraceSlice = 16384;
 #define FA_TRACE(who, ev, j) do { } while (0)
 #endif
 
-// The k-th unit of this CTA: rounds of gridDim.x units, assigned forward in
-// even rounds and backward in odd ones (longest-first lists then balance).
-// Returns a value >= num_units when this CTA has no unit in round k.
-__device__ __forceinline__ int unit_index(int k, const FwdParams& p) {
-  const int i = (k & 1) ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
-                        : static_cast<int>(blockIdx.x);
-  return k * static_cast<int>(gridDim.x) + i;
+// Dynamic schedule: CTAs claim units in order from a global counter, so the
+// units running at any time are a contiguous stretch of the longest-first,
+// head-grouped order (balanced and L2-friendly).  The producer thread claims
+// and passes each unit to the MMA thread and the softmax warps through a
+// 4-deep queue in shared memory.
+constexpr uint32_t UQ_CONSUMERS = 1 + 16;   // MMA thread + one arrive per softmax warp
+
+// Units [0, gridDim.x) are each CTA's first unit (no atomic on the start-up
+// path); later units come from the counter.
+__device__ __forceinline__ int claim_unit(const FwdParams& p) {
+  const int u = static_cast<int>(gridDim.x + atomicAdd(p.sched, 1u));
+  return u < p.num_units ? u : -1;
 }
 
 __device__ __forceinline__ void record_error(SharedHeader* sh, const FwdParams& p, int code) {
@@ -242,11 +250,24 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
   const uint64_t pol_kv = policy_evict_last();
   const uint64_t pol_q = policy_evict_first();
 
-  for (int k = 0; k < p.rounds && ok; ++k) {
-    const int u = unit_index(k, p);
-    if (u >= p.num_units) continue;
-    const Unit w = get_unit(u, p);
-    if (w.jhi < 0) continue;
+  int k = 0;
+  int cur = static_cast<int>(blockIdx.x);   // grid <= num_units
+  while (true) {
+    // publish the unit to the consumers (-1 ends their loops)
+    const uint32_t qs = k & 3u, qr = static_cast<uint32_t>(k) >> 2;
+    if (!mbar_wait(smem_u32(&sh->uq_empty[qs]), (qr & 1u) ^ 1u, p.wait_limit_ns)) {
+      record_error(sh, p, ST_TIMEOUT_LOAD); ok = false; break;
+    }
+    sh->uq[qs] = cur;
+    mbar_arrive(smem_u32(&sh->uq_full[qs]));
+    ++k;
+    if (cur < 0) break;
+    const Unit w = get_unit(cur, p);
+    int nxt = -2;   // claimed once this unit's first loads are on their way
+    if (w.jhi < 0) {
+      cur = claim_unit(p);
+      continue;
+    }
     if (aborted(sh)) { ok = false; break; }
     // Q tiles (wait until the previous unit's S MMAs have read them)
     if (!mbar_wait(smem_u32(&sh->q_empty), (q_uses & 1u) ^ 1u, p.wait_limit_ns)) {
@@ -261,18 +282,6 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
                          c * C::BOX_INNER, w.h, w.q0 + t * BLOCK_M, w.b, pol_q);
     q_outstanding = true;
     ++q_uses;
-    // warm L2 with the Q tiles of this CTA's next unit
-    {
-      const int un = unit_index(k + 1, p);
-      if (k + 1 < p.rounds && un < p.num_units) {
-        const Unit wn = get_unit(un, p);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int c = 0; c < C::NCHUNK; ++c)
-            tma_prefetch_l2_4d(mq, c * C::BOX_INNER, wn.h, wn.q0 + t * BLOCK_M, wn.b);
-      }
-    }
     // K_j, V_j for the union of the tiles' block ranges
     for (int j = w.jlo; j <= w.jhi && ok; ++j) {
 #pragma unroll
@@ -294,7 +303,22 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
         phase_mask = (phase_mask & ~(1u << slot)) | ((round & 1u) << slot);
         ++kv_it;
       }
+      if (nxt == -2) {
+        // claim the next unit while these loads are in flight, and warm L2
+        // with its Q tiles
+        nxt = claim_unit(p);
+        if (nxt >= 0) {
+          const Unit wn = get_unit(nxt, p);
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int c = 0; c < C::NCHUNK; ++c)
+              tma_prefetch_l2_4d(mq, c * C::BOX_INNER, wn.h, wn.q0 + t * BLOCK_M, wn.b);
+        }
+      }
     }
+    if (!ok) break;
+    cur = nxt;
   }
   // drain: every copy this thread issued must land before the CTA exits
   if (!ok) {
@@ -363,9 +387,14 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
   const uint32_t o_tmem[2] = {tbase + C::O_COL0, tbase + C::O_COL0 + D};
   FA_TRACE_DECL;
 
-  for (int k = 0; k < p.rounds && ok; ++k) {
-    const int u = unit_index(k, p);
-    if (u >= p.num_units) continue;
+  for (int k = 0; ok; ++k) {
+    const uint32_t qs = k & 3u, qr = static_cast<uint32_t>(k) >> 2;
+    if (!mbar_wait(smem_u32(&sh->uq_full[qs]), qr & 1u, p.wait_limit_ns)) {
+      record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+    }
+    const int u = *reinterpret_cast<volatile int*>(&sh->uq[qs]);
+    mbar_arrive(smem_u32(&sh->uq_empty[qs]));
+    if (u < 0) break;
     const Unit w = get_unit(u, p);
     if (w.jhi < 0) continue;
     if (aborted(sh)) { ok = false; break; }
@@ -611,9 +640,15 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
   bool ok = true;
   constexpr int OUT_ES = 2;
 
-  for (int k = 0; k < p.rounds && ok; ++k) {
-    const int u = unit_index(k, p);
-    if (u >= p.num_units) continue;
+  for (int k = 0; ok; ++k) {
+    const uint32_t qs = k & 3u, qr = static_cast<uint32_t>(k) >> 2;
+    bool have = mbar_wait(smem_u32(&sh->uq_full[qs]), qr & 1u, p.wait_limit_ns);
+    have = __all_sync(0xffffffffu, have);
+    if (!have) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
+    const int u = *reinterpret_cast<volatile int*>(&sh->uq[qs]);
+    __syncwarp();
+    if (lane_id() == 0) mbar_arrive(smem_u32(&sh->uq_empty[qs]));
+    if (u < 0) break;
     const Tile w = get_tile(u, t, p);
     if (!w.rows) continue;
     const int row = w.qs + r;
@@ -771,6 +806,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&sh->o_empty[t]), 256);
     }
     mbar_init(smem_u32(&sh->mma_done), 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&sh->uq_full[i]), 1);
+      mbar_init(smem_u32(&sh->uq_empty[i]), UQ_CONSUMERS);
+    }
     sh->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_map(&tm_q);
@@ -803,6 +842,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
+  }
+  if (threadIdx.x == 0) {
+    // this CTA claims no more units; the last CTA to get here zeroes the
+    // scheduler scratch for the next launch (every CTA gets here: all waits
+    // are bounded)
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+      __threadfence();
+    }
   }
 }
 

@@ -25,8 +25,10 @@
  * Element types: FA_FP16 -> q/k/v/out fp16; FA_BF16 -> q/k/v/out bf16;
  * FA_E4M3 -> q/k/v e4m3 (OCP FP8, 1 byte), out bf16.
  *
- * Ownership: the caller allocates and owns every buffer; the library
- * allocates no device memory and keeps no pointer after a call returns.
+ * Ownership: the caller allocates and owns every buffer.  The library keeps
+ * no pointer after a call returns; its only device memory is a 2 KB pool of
+ * work-scheduler counters allocated once per device on the first call there
+ * (one pair of counters per stream, left at zero by every launch).
  * Calls are asynchronous on `stream` (NULL = the legacy default stream);
  * outputs are ready when the stream's work completes.
  *

@@ -14,6 +14,14 @@ namespace fa {
 
 __device__ int g_status_word;
 
+// Scratch of fa_fwd_noalloc: the work scheduler's two 32-bit counters (next
+// unit, finished CTAs) live in this fixed array instead of memory from
+// cudaMalloc.  256 bytes, held by every GPU that loads the library until the
+// process exits; only the first two words are used, for any problem size.
+constexpr int kNoAllocScratchWords = 64;
+constexpr int kSchedWordsNeeded = 2;
+static __device__ __align__(256) unsigned g_noalloc_scratch[kNoAllocScratchWords];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -32,6 +40,7 @@ struct DeviceState {
   unsigned* sched_pool = nullptr;
   std::unordered_map<cudaStream_t, int> sched_slot;
   int next_slot = 0;
+  unsigned* noalloc_scratch = nullptr;   // device address of g_noalloc_scratch
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -80,11 +89,25 @@ int sched_counters(DeviceState* ds, cudaStream_t stream, unsigned** out) {
   return FA_OK;
 }
 
+// Device address of the static scratch array, looked up once per device
+// with that device current.  In host code the array's name is only a
+// host-side stand-in; kernels must be given this address.
+int noalloc_scratch(DeviceState* ds, unsigned** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!ds->noalloc_scratch) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
+    ds->noalloc_scratch = static_cast<unsigned*>(ptr);
+  }
+  *out = ds->noalloc_scratch;
+  return FA_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int D, int DT>
 int launch(const void* q, const void* k, const void* v, const FwdParams& base, cudaStream_t stream,
-           DeviceState* ds, int bit) {
+           DeviceState* ds, int bit, unsigned* sched_override) {
   using C = Cfg<D, DT>;
   FwdParams p = base;
   const CUtensorMapDataType tdt = DT == DT_FP16   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
@@ -102,8 +125,12 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     ds->attr_set |= (1u << bit);
   }
   const int grid = p.num_units < ds->num_sms ? p.num_units : ds->num_sms;
-  int rc = sched_counters(ds, stream, &p.sched);
-  if (rc != FA_OK) return rc;
+  if (sched_override) {
+    p.sched = sched_override;
+  } else {
+    int rc = sched_counters(ds, stream, &p.sched);
+    if (rc != FA_OK) return rc;
+  }
   fa_fwd_kernel<D, DT><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -129,7 +156,7 @@ int validate(const void* q, const void* k, const void* v, void* out, int B, int 
 
 int forward(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Nq, int Nk,
             int H, int D, float scale, int causal, int window_left, int dtype, float qd, float kd,
-            float vd, cudaStream_t stream) {
+            float vd, cudaStream_t stream, unsigned* sched_override = nullptr) {
   int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype);
   if (rc != FA_OK) return rc;
   if (!(qd > 0.f) || !std::isfinite(qd) || !(kd > 0.f) || !std::isfinite(kd) || !(vd > 0.f) ||
@@ -180,11 +207,11 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   p.wait_limit_ns = g_wait_limit_ns;
   p.status = ds->status;
   switch (dtype * 2 + (D == 128 ? 1 : 0)) {
-    case FA_FP16 * 2 + 0: return launch<64, DT_FP16>(q, k, v, p, stream, ds, 0);
-    case FA_FP16 * 2 + 1: return launch<128, DT_FP16>(q, k, v, p, stream, ds, 1);
-    case FA_BF16 * 2 + 0: return launch<64, DT_BF16>(q, k, v, p, stream, ds, 2);
-    case FA_BF16 * 2 + 1: return launch<128, DT_BF16>(q, k, v, p, stream, ds, 3);
-    case FA_E4M3 * 2 + 1: return launch<128, DT_E4M3>(q, k, v, p, stream, ds, 4);
+    case FA_FP16 * 2 + 0: return launch<64, DT_FP16>(q, k, v, p, stream, ds, 0, sched_override);
+    case FA_FP16 * 2 + 1: return launch<128, DT_FP16>(q, k, v, p, stream, ds, 1, sched_override);
+    case FA_BF16 * 2 + 0: return launch<64, DT_BF16>(q, k, v, p, stream, ds, 2, sched_override);
+    case FA_BF16 * 2 + 1: return launch<128, DT_BF16>(q, k, v, p, stream, ds, 3, sched_override);
+    case FA_E4M3 * 2 + 1: return launch<128, DT_E4M3>(q, k, v, p, stream, ds, 4, sched_override);
     default: return FA_ERR_UNSUPPORTED;
   }
 }
@@ -233,6 +260,30 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* l
                       s) != cudaSuccess)
     return FA_ERR_CUDA;
   return cudaStreamSynchronize(s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q,
+                   int N_k, int H, int D, float scale, int causal, int window_left, int dtype,
+                   float q_descale, float k_descale, float v_descale, fa_stream_t stream) {
+  int rc = fa::validate(q, k, v, out, B, N_q, N_k, H, D, scale, causal, window_left, dtype);
+  if (rc != FA_OK) return rc;
+  // the scheduler's counters index work units as 32-bit values: problems with
+  // more units than that (or a scratch need above the array) are rejected
+  const int64_t units = static_cast<int64_t>((N_q + 255) / 256) * B * H;
+  if (fa::kSchedWordsNeeded > fa::kNoAllocScratchWords || units > 0x7fff0000LL) return FA_ERR_ARG;
+  if (N_q == 0) return FA_OK;
+  fa::DeviceState* ds = nullptr;
+  rc = fa::device_state(&ds);
+  if (rc != FA_OK) return rc;
+  unsigned* scratch = nullptr;
+  rc = fa::noalloc_scratch(ds, &scratch);
+  if (rc != FA_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the counters must start at zero; every launch also leaves them at zero
+  if (cudaMemsetAsync(scratch, 0, sizeof(unsigned) * fa::kSchedWordsNeeded, s) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, D, scale, causal, window_left, dtype, q_descale,
+                     k_descale, v_descale, s, scratch);
 }
 
 int fa_device_status(fa_stream_t stream, int* flags) {

@@ -100,6 +100,32 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* l
                 float v_descale, fa_stream_t stream);
 
 /*
+ * fa_fwd_noalloc -- the forward of fa_fwd / fa_fwd_fp8 (dtype FA_E4M3 uses
+ * the three descales; other dtypes take 1.0) for callers that cannot
+ * allocate device memory: code whose allocations must all come from its own
+ * pre-reserved pool or arena, code that must not take the allocator's locks
+ * or risk an allocation failure on its launch path, and code running where
+ * cudaMalloc is not permitted.  The paper has no counterpart; it is an
+ * interface choice of this library.
+ *   This call allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library routine).  The work scheduler's scratch, two 32-bit counters,
+ * lives in a fixed 256-byte device array inside the library, which every GPU
+ * that loads the library holds until the process exits.  Its first call on
+ * a device looks up that array's device address (once, with the device
+ * current); make that first call before any stream capture.  Each call
+ * clears the counters on `stream` before its kernel, and the kernel leaves
+ * them at zero.  All calls share the one array, so calls that overlap on the
+ * GPU (for instance on two streams) race and give wrong results: issue them
+ * in order.  Inputs, outputs, layouts and errors are those of fa_fwd;
+ * problems with more work units than the 32-bit counters can index are
+ * rejected with FA_ERR_ARG.
+ */
+int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                   int B, int N_q, int N_k, int H, int D, float scale, int causal,
+                   int window_left, int dtype, float q_descale, float k_descale,
+                   float v_descale, fa_stream_t stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * device status word that kernels set when a wait times out.  Returns FA_OK,
  * FA_ERR_TIMEOUT (and the raw flag bits in *flags when flags != NULL) or

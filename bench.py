@@ -65,6 +65,21 @@ def dist_info():
     return world, rank, local
 
 
+def rank_seeds(w: W.Workload, rank: int):
+    """Seeds of this rank's batch: every rank draws its own inputs (weak scaling)."""
+    return tuple(s + 7919 * rank for s in w.seeds)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank float over the process group (the value itself with one process)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks(dtype: str):
     """(peak TF/s for the kernel timed alone, source string, sustained) from MEASURED_PEAKS.json."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -235,7 +250,7 @@ def main():
     if args.batch is not None:
         import dataclasses
         w = dataclasses.replace(w, B=args.batch, name=f"{w.name}@B{args.batch}")
-    seeds = tuple(s + 7919 * rank for s in w.seeds)   # each rank: its own batch
+    seeds = rank_seeds(w, rank)   # each rank: its own batch
     qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=seeds)
     hq, hk, hv = qkv.q.pin_memory(), qkv.k.pin_memory(), qkv.v.pin_memory()
     q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
@@ -276,11 +291,7 @@ def main():
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
     rc, flags = device_status(device=dev)
     if rc != 0:
         raise RuntimeError(f"device status {rc} flags {flags} in the timed region")
@@ -309,11 +320,7 @@ def main():
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ems = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ems], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ems = float(t.item())
+    ems = max_over_ranks(t0.elapsed_time(t1), dev)
     e2e_value = world * flops * args.e2e_steps / (ems / 1e3) / 1e12
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()

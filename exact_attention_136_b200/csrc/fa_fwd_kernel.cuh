@@ -570,9 +570,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // into TMEM at p_addr (16x32bx2 layout: lanes 0-15 of the access for
 // threads 0-15, the same lanes half a row of P further for threads 16-31)
 // and return their fp32 sum twice: exact, and over the values P*V uses
-// (different only for e4m3, whose 3-bit mantissa would otherwise bias O).  EMULATE: pairs 5-7 of every 8 go through
-// exp2_poly2 (37.5% of the exponentials on the FMA pipe, which balances the
-// 16/clk MUFU against the 128/clk FMA pipe).
+// (different only for e4m3, whose 3-bit mantissa would otherwise bias O).
+// Pairs i >= FA_EMU_FROM of every 8 (unmasked blocks) take exp2_poly2 on the
+// FMA pipe instead of MUFU.  Default 8 = none: in the full kernel, where the
+// two tiles' softmax warps share every scheduler, the emulation's extra
+// instructions cost more than the MUFU time they free (B200, causal D=128
+// bf16: 988 TF/s without, 939 with 3 of 8 pairs emulated; D=64 fp16 and FP8
+// the same way).  Kept as a build option for configurations where MUFU is
+// the binding limit.
+#ifndef FA_EMU_FROM
+#define FA_EMU_FROM 8
+#endif
+
 template <int DT, bool EMULATE>
 __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_mref, uint32_t p_addr) {
   const float2 cc2 = make_float2(cc, cc);
@@ -588,7 +597,7 @@ __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_m
       const int c = q * 16 + 2 * i;
       const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), cc2, nm2);
       float2 e;
-      if (EMULATE && i >= 5) {
+      if (EMULATE && i >= FA_EMU_FROM) {
         e = exp2_poly2(x);
       } else {
         e = make_float2(ex2_approx(x.x), ex2_approx(x.y));

@@ -122,6 +122,12 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FA_ERR_CUDA;
+    // The per-role register split (setmaxnreg) redistributes the registers
+    // the CTA was launched with; it is only valid for the launch count it
+    // was sized for, so a build that came out with another count is refused.
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, fa_fwd_kernel<D, DT>) != cudaSuccess) return FA_ERR_CUDA;
+    if (fa.numRegs != REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
     ds->attr_set |= (1u << bit);
   }
   const int grid = p.num_units < ds->num_sms ? p.num_units : ds->num_sms;

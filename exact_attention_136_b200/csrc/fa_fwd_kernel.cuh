@@ -20,14 +20,16 @@
 //                  PV_0(j-1), S_0(j), PV_1(j-1), S_1(j)
 //                so the tensor pipe works on one tile while the softmax
 //                warpgroup of the other tile runs (ping-pong).
-//   warps 4-7  : softmax warpgroup of tile 0, warps 8-11: tile 1.  Thread r
-//                owns query row r of its tile (TMEM lane r).  Per block it
-//                loads the 128 scores of its row, masks boundary blocks, keeps
-//                the running max / sum in registers, rescales its O row in
+//   warps 4-11 : softmax of tile 0 (two warpgroups), warps 12-19: tile 1.
+//                Two threads per query row: the tcgen05 16x32bx2 access gives
+//                lanes t and t+16 of a warp the two 64-key halves of one TMEM
+//                lane (= row), so a row max or sum is one shuffle.  Per block
+//                they load the row's 128 scores, mask boundary blocks, keep
+//                the running max / sum in registers, rescale the O row in
 //                TMEM only when the max rose by more than a threshold (the
 //                final division uses the same reference, so this is exact),
-//                writes P (16-bit, or e4m3 for the FP8 path) into TMEM over
-//                the scores, and at the end of the unit normalises O, stores
+//                write P (16-bit, or e4m3 for the FP8 path) into TMEM over
+//                the scores, and at the end of the unit normalise O and store
 //                it and the fp32 LSE.
 //   TMEM columns: S_0 [0,128) with P_0 at [64,..), S_1 [128,256) with P_1 at
 //                [192,..), O_0 [256, 256+D), O_1 [256+D, 256+2D).
@@ -42,6 +44,7 @@
 #include <cuda_fp8.h>
 
 #include "sm100.cuh"
+
 
 namespace fa {
 
@@ -103,6 +106,11 @@ struct Cfg {
   static constexpr float PSHIFT = DT == DT_E4M3 ? 7.0f : 0.0f;
   // rescale O only when the row max rose by more than this (log2 units)
   static constexpr float RESCALE_THRESHOLD = DT == DT_E4M3 ? 1.5f : 8.0f;
+  // P is handed to the MMA thread in two halves (keys k with k mod 64 below
+  // 32 first), so the first PV MMAs run while the rest is exponentiated.
+  // Measured on B200: faster for 16-bit inputs; for e4m3, whose PV is only
+  // four MMAs, the extra hand-over costs more than the overlap gains.
+  static constexpr bool PSPLIT = DT != DT_E4M3;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(D == 64 || D == 128, "head dim");
 };
@@ -111,11 +119,15 @@ struct SharedHeader {
   uint64_t q_full, q_empty;
   uint64_t kv_full[12], kv_empty[12];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t p_half[2];   // first half of P_t stored (keys k of the block with k mod 64 < 32)
   uint64_t mma_done;
   uint64_t uq_full[4], uq_empty[4];   // unit queue: producer -> MMA + softmax warps
   int uq[4];                          // claimed unit ids, -1 = no more work
   uint32_t tmem_base;
   int abort_flag;
+#ifdef FA_STATS_BUILD
+  unsigned stats[64];
+#endif
 };
 static_assert(sizeof(SharedHeader) <= HEADER_BYTES, "header");
 
@@ -193,6 +205,20 @@ constexpr int kTraceSlice = 16384;
           (static_cast<unsigned long long>((j) & 0xffff) << 32) |                                    \
           (static_cast<unsigned long long>(clock64()) & 0xffffffffull);                              \
   } while (0)
+#elif defined(FA_STATS_BUILD)
+// Tuning build: the time between consecutive events of a role is summed per
+// (role, event) in shared memory by the role's recording thread (lane 0 of
+// one warp per role and softmax warpgroup) and added to g_stats at exit.
+__device__ unsigned long long g_stats[64];
+#define FA_TRACE_DECL uint32_t stat_last = static_cast<uint32_t>(clock())
+#define FA_TRACE(who, ev, j)                                                      \
+  do {                                                                            \
+    if ((who) >= 2 || (threadIdx.x & 127) == 0) {                                 \
+      const uint32_t now_ = static_cast<uint32_t>(clock());                       \
+      atomicAdd(&sh->stats[(who) * 16 + (ev)], now_ - stat_last);                 \
+      stat_last = now_;                                                           \
+    }                                                                             \
+  } while (0)
 #else
 #define FA_TRACE_DECL do { } while (0)
 #define FA_TRACE(who, ev, j) do { } while (0)
@@ -223,11 +249,14 @@ __device__ __forceinline__ bool aborted(SharedHeader* sh) {
 
 // Register split between warpgroup 0 (one producer and one MMA thread) and
 // the four softmax warpgroups.  The launch gives every thread 96 registers
-// (640 threads, one CTA per SM: 61440 of the SM's 65536); the split must not
-// exceed that total: 128 * REGS_LOAD_MMA + 512 * REGS_SOFTMAX <= 61440.
+// (640 threads, one CTA per SM: 61440 of the SM's 65536; the kernel is
+// compiled to exactly that, checked by the host before the first launch);
+// the split must not exceed that total.
+constexpr int REGS_LAUNCH = 96;
 constexpr int REGS_LOAD_MMA = 64;
 constexpr int REGS_SOFTMAX = 104;
-static_assert(128 * REGS_LOAD_MMA + 512 * REGS_SOFTMAX <= NUM_THREADS * 96, "register split");
+static_assert(NUM_THREADS * REGS_LAUNCH <= 65536, "launch registers");
+static_assert(128 * REGS_LOAD_MMA + 512 * REGS_SOFTMAX <= NUM_THREADS * REGS_LAUNCH, "register split");
 template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N)); }
 template <int N>
@@ -330,66 +359,122 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
     if (q_outstanding && !mbar_wait(smem_u32(&sh->q_full), (q_uses - 1u) & 1u, p.wait_limit_ns))
       record_error(sh, p, ST_TIMEOUT_DRAIN);
   }
+  FA_TRACE(3, 15, 0);
 }
 
 // ------------------------------------------------------------------ MMA issuer
-// Opaque copy: keeps the compiler from hoisting per-iteration address math
-// (and the descriptors built from it) out of the key-block loop, which would
-// hold dozens of 64-bit descriptors in registers.
+// Opaque copy: keeps the compiler from hoisting per-iteration descriptor math
+// out of the key-block loop, which would hold dozens of descriptors in
+// registers.
 __device__ __forceinline__ uint32_t opaque(uint32_t x) {
   asm volatile("mov.b32 %0, %0;" : "+r"(x));
   return x;
 }
 
+// Every shared-memory descriptor here has the same high word: 8-row groups
+// 1024 B apart (stride byte offset), descriptor version 1, 128-byte swizzle.
+constexpr uint32_t DESC_HI = sdesc_sw128_hi(1024);
+
+// S = Q K^T for one 128-row tile.  a0 / b0 are the descriptor low words of
+// the K-major 128B-swizzled Q and K tiles; the K step advances 32 B inside a
+// 128-byte row, then jumps to the next 128-byte column chunk.
 template <int D, int DT>
-__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t a0, uint32_t b0, uint32_t hi) {
   using C = Cfg<D, DT>;
-  // K-major 128B-swizzled Q and K tiles: 8-row groups 1024 B apart; the K
-  // step advances 32 B inside a 128-byte row, then jumps to the next chunk.
-  const uint64_t a0 = sdesc_sw128(q_addr, 16, 1024);
-  const uint64_t b0 = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < D / C::KSTEP; ++kk) {
     const int byte = kk * C::KSTEP * C::ES;
-    const uint64_t off = static_cast<uint64_t>(((byte / 128) * C::CHUNK_BYTES + (byte % 128)) >> 4);
-    if constexpr (DT == DT_E4M3) mma_f8_ss(d_tmem, a0 + off, b0 + off, C::IDESC_S, kk > 0);
-    else mma_f16_ss(d_tmem, a0 + off, b0 + off, C::IDESC_S, kk > 0);
+    const uint32_t off = static_cast<uint32_t>(((byte / 128) * C::CHUNK_BYTES + (byte % 128)) >> 4);
+    if constexpr (DT == DT_E4M3) mma_f8_ss_lo(d_tmem, a0 + off, b0 + off, hi, C::IDESC_S, kk > 0);
+    else mma_f16_ss_lo(d_tmem, a0 + off, b0 + off, hi, C::IDESC_S, kk > 0);
   }
 }
 
-template <int D, int DT>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, bool accumulate) {
+// O += P V with P read from TMEM.  b0 is the descriptor low word of the
+// MN-major V tile (head dim contiguous): 8-key groups 1024 B apart, 128-byte
+// head-dim chunks CHUNK_BYTES apart (the leading byte offset).
+// PART 0 / 1 issue only the MMAs over keys k with k mod 64 below / at or
+// above 32 (the two halves in which the softmax hands P over: each thread
+// holds 64 keys of a row and exponentiates them in order), PART 2 all.
+template <int D, int DT, int PART = 2>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t b0, uint32_t hi,
+                                         bool accumulate) {
   using C = Cfg<D, DT>;
-  // V tile is MN-major (head dim contiguous): 8-key groups 1024 B apart,
-  // 128-byte head-dim chunks CHUNK_BYTES apart.
-  const uint64_t b0 = sdesc_sw128(v_addr, C::CHUNK_BYTES, 1024);
 #pragma unroll
   for (int kk = 0; kk < BLOCK_N / C::KSTEP; ++kk) {
-    const uint64_t off = static_cast<uint64_t>((kk * C::KSTEP * 128) >> 4);
+    const bool first_half = (kk * C::KSTEP) % 64 < 32;
+    if ((PART == 0 && !first_half) || (PART == 1 && first_half)) continue;
+    const uint32_t off = static_cast<uint32_t>((kk * C::KSTEP * 128) >> 4);
     const uint32_t a = p_tmem + kk * (C::KSTEP * C::ES / 4);
-    if constexpr (DT == DT_E4M3) mma_f8_ts(d_tmem, a, b0 + off, C::IDESC_O, accumulate || kk > 0);
-    else mma_f16_ts(d_tmem, a, b0 + off, C::IDESC_O, accumulate || kk > 0);
+    if constexpr (DT == DT_E4M3) mma_f8_ts_lo(d_tmem, a, b0 + off, hi, C::IDESC_O, accumulate || kk > 0);
+    else mma_f16_ts_lo(d_tmem, a, b0 + off, hi, C::IDESC_O, accumulate || kk > 0);
   }
 }
 
+// Ring position (slot, phase parity) of the next load.
+template <int STAGES>
+__device__ __forceinline__ void ring_next(uint32_t& slot, uint32_t& par) {
+  ++slot;
+  if (slot == static_cast<uint32_t>(STAGES)) {
+    slot = 0;
+    par ^= 1u;
+  }
+}
+
+// O_t += P_t V for one key block, issued as the softmax hands P over: with
+// the split hand-over (Cfg::PSPLIT) the MMAs over the first half of the keys
+// go as soon as that half is stored.  `before_first` runs after the first
+// wait, ahead of the first MMA.  Returns false when a wait timed out.
+template <int D, int DT, typename F>
+__device__ __forceinline__ bool issue_pv_handover(uint32_t p_half_bar, uint32_t p_full_bar, uint32_t parity,
+                                                  uint64_t lim, uint32_t o_tmem, uint32_t p_tmem,
+                                                  uint32_t v_desc, uint32_t hi, bool accumulate,
+                                                  F before_first) {
+  using C = Cfg<D, DT>;
+  if constexpr (C::PSPLIT) {
+    if (!mbar_wait(p_half_bar, parity, lim) || !before_first()) return false;
+    tc_fence_after();
+    issue_pv<D, DT, 0>(o_tmem, p_tmem, v_desc, hi, accumulate);
+    if (!mbar_wait(p_full_bar, parity, lim)) return false;
+    tc_fence_after();
+    issue_pv<D, DT, 1>(o_tmem, p_tmem, v_desc, hi, true);
+  } else {
+    if (!mbar_wait(p_full_bar, parity, lim) || !before_first()) return false;
+    tc_fence_after();
+    issue_pv<D, DT>(o_tmem, p_tmem, v_desc, hi, accumulate);
+  }
+  return true;
+}
+
+// The MMA thread runs alone on its warp and competes for issue slots with
+// the softmax warps of its sub-partition, so every instruction between two
+// MMA groups delays the tensor pipe: per key block the steady state below
+// issues its 32 MMAs with nothing but the four waits, four commits and the
+// ring advance between them; every decision is taken once per unit.
 template <int D, int DT>
 __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const FwdParams& p) {
   using C = Cfg<D, DT>;
-  const uint32_t sq = smem_u32(tiles);
+  constexpr uint32_t SLOT_DESC = C::TILE_BYTES >> 4;   // descriptor start-address step per ring slot
   const uint32_t ring = smem_u32(tiles + 2 * C::TILE_BYTES);
-  uint32_t kv_base = 0;
+  const uint32_t q_desc0 = sdesc_sw128_lo(smem_u32(tiles), 16);
+  const uint32_t k_desc0 = sdesc_sw128_lo(ring, 16);
+  const uint32_t v_desc0 = sdesc_sw128_lo(ring, C::CHUNK_BYTES);
+  const uint32_t kv_full0 = smem_u32(&sh->kv_full[0]);
+  const uint32_t kv_empty0 = smem_u32(&sh->kv_empty[0]);
+  const uint32_t s_full0 = smem_u32(&sh->s_full[0]), p_full0 = smem_u32(&sh->p_full[0]);
+  const uint32_t p_half0 = smem_u32(&sh->p_half[0]);
+  const uint64_t lim = p.wait_limit_ns;
   uint32_t q_uses = 0;
   uint32_t p_waits[2] = {0, 0};
   uint32_t o_units[2] = {0, 0};
+  uint32_t kslot = 0, kpar = 0;   // ring position of K_j (loads alternate K_j, V_j)
+  uint32_t vslot = 0, vpar = 0;   // ring position of V_{j-1}
   bool ok = true;
-  const uint32_t s_tmem[2] = {tbase, tbase + 128};
-  const uint32_t p_tmem[2] = {tbase + C::P_OFF, tbase + 128 + C::P_OFF};
-  const uint32_t o_tmem[2] = {tbase + C::O_COL0, tbase + C::O_COL0 + D};
   FA_TRACE_DECL;
 
   for (int k = 0; ok; ++k) {
     const uint32_t qs = k & 3u, qr = static_cast<uint32_t>(k) >> 2;
-    if (!mbar_wait(smem_u32(&sh->uq_full[qs]), qr & 1u, p.wait_limit_ns)) {
+    if (!mbar_wait(smem_u32(&sh->uq_full[qs]), qr & 1u, lim)) {
       record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
     }
     const int u = *reinterpret_cast<volatile int*>(&sh->uq[qs]);
@@ -398,104 +483,143 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
     const Unit w = get_unit(u, p);
     if (w.jhi < 0) continue;
     if (aborted(sh)) { ok = false; break; }
-    if (!mbar_wait(smem_u32(&sh->q_full), q_uses & 1u, p.wait_limit_ns)) {
+    if (!mbar_wait(smem_u32(&sh->q_full), q_uses & 1u, lim)) {
       record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
     }
     ++q_uses;
+    // Steady key blocks: both tiles issue PV(j-1) and S(j), and j-1 is
+    // neither tile's first block (O starts from zero there, after the
+    // previous unit's epilogue has read it) nor its last (O is handed over).
+    const bool both = w.valid[0] && w.valid[1];
+    const int js = both ? max(w.lo[0], w.lo[1]) + 2 : 0x7fffffff;
+    const int je = both ? min(w.hi[0], w.hi[1]) : -1;
     for (int j = w.jlo; j <= w.jhi + 1 && ok; ++j) {
-      // K_j feeds S_0(j), S_1(j); V_{j-1} feeds PV_0(j-1), PV_1(j-1).  Each
-      // is waited for right before its first MMA and its ring slot released
-      // right after its last one, so a late K never holds back a PV.
-      const bool has_k = j <= w.jhi;
-      const bool has_v = j > w.jlo;
-      const uint32_t kidx = kv_base + 2u * (j - w.jlo);
-      const uint32_t vidx = kidx - 1u;
-      const uint32_t kslot = kidx % C::STAGES;
-      const uint32_t vslot = vidx % C::STAGES;
-      bool k_ready = false, v_ready = false, k_done = !has_k, v_done = !has_v;
-      const int jp = j - 1;
-      const bool pv_use[2] = {w.valid[0] && jp >= w.lo[0] && jp <= w.hi[0],
-                              w.valid[1] && jp >= w.lo[1] && jp <= w.hi[1]};
-      const bool s_use[2] = {w.valid[0] && j >= w.lo[0] && j <= w.hi[0],
-                             w.valid[1] && j >= w.lo[1] && j <= w.hi[1]};
+      const uint32_t vfull = kv_full0 + 8u * vslot, kfull = kv_full0 + 8u * kslot;
+      if (j >= js && j <= je) {
+        const uint32_t v_desc = opaque(v_desc0) + vslot * SLOT_DESC;
+        const uint32_t k_desc = opaque(k_desc0) + kslot * SLOT_DESC;
+        const uint32_t hi = opaque(DESC_HI);
+        FA_TRACE(2, 0, j);
+        if (!mbar_wait(vfull, vpar, lim) ||
+            !issue_pv_handover<D, DT>(p_half0, p_full0, p_waits[0] & 1u, lim, tbase + C::O_COL0,
+                                      tbase + C::P_OFF, v_desc, hi, true, [] { return true; })) {
+          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+        }
+        ++p_waits[0];
+        FA_TRACE(2, 1, j);
+        FA_TRACE(2, 2, j);
+        if (!mbar_wait(kfull, kpar, lim)) {
+          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+        }
+        FA_TRACE(2, 7, j);
+        tc_fence_after();
+        issue_s<D, DT>(tbase, opaque(q_desc0), k_desc, hi);
+        mma_commit(s_full0);
+        FA_TRACE(2, 3, j);
+        if (!issue_pv_handover<D, DT>(p_half0 + 8u, p_full0 + 8u, p_waits[1] & 1u, lim, tbase + C::O_COL0 + D,
+                                      tbase + 128 + C::P_OFF, v_desc, hi, true, [] { return true; })) {
+          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+        }
+        ++p_waits[1];
+        FA_TRACE(2, 4, j);
+        mma_commit(kv_empty0 + 8u * vslot);   // last reader of V_{j-1}
+        FA_TRACE(2, 5, j);
+        issue_s<D, DT>(tbase + 128, opaque(q_desc0) + SLOT_DESC, k_desc, hi);
+        mma_commit(s_full0 + 8u);
+        mma_commit(kv_empty0 + 8u * kslot);   // last reader of K_j
+        FA_TRACE(2, 6, j);
+      } else {
+        // General block: either tile may skip PV(j-1) or S(j) (ragged or
+        // windowed ranges, the first and last blocks of a unit).  Each
+        // operand is waited for right before its first MMA and its ring slot
+        // released right after its last one.
+        const bool has_k = j <= w.jhi;
+        const bool has_v = j > w.jlo;
+        bool k_ready = false, v_ready = false, k_done = !has_k, v_done = !has_v;
+        const int jp = j - 1;
+        const bool pv_use[2] = {w.valid[0] && jp >= w.lo[0] && jp <= w.hi[0],
+                                w.valid[1] && jp >= w.lo[1] && jp <= w.hi[1]};
+        const bool s_use[2] = {w.valid[0] && j >= w.lo[0] && j <= w.hi[0],
+                               w.valid[1] && j >= w.lo[1] && j <= w.hi[1]};
+        const uint32_t v_desc = opaque(v_desc0) + vslot * SLOT_DESC;
+        const uint32_t k_desc = opaque(k_desc0) + kslot * SLOT_DESC;
+        const uint32_t hi = opaque(DESC_HI);
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (pv_use[t]) {
-          // O_t += P_t(j-1) V_{j-1}
-          if (!v_ready) {
-            FA_TRACE(2, 10, jp);
-            if (!mbar_wait(smem_u32(&sh->kv_full[vslot]), (vidx / C::STAGES) & 1u, p.wait_limit_ns)) {
+        for (int t = 0; t < 2; ++t) {
+          if (pv_use[t]) {
+            // O_t += P_t(j-1) V_{j-1}
+            if (!v_ready) {
+              if (!mbar_wait(vfull, vpar, lim)) {
+                record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+              }
+              v_ready = true;
+            }
+            // (the first PV of a unit also waits until the previous unit's
+            // epilogue has read O_t out)
+            const uint32_t o_empty = smem_u32(&sh->o_empty[t]), o_par = (o_units[t] & 1u) ^ 1u;
+            const bool first = jp == w.lo[t];
+            if (!issue_pv_handover<D, DT>(p_half0 + 8u * t, p_full0 + 8u * t, p_waits[t] & 1u, lim,
+                                          tbase + C::O_COL0 + D * t, tbase + 128 * t + C::P_OFF, v_desc, hi,
+                                          !first, [&] { return !first || mbar_wait(o_empty, o_par, lim); })) {
               record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
             }
-            v_ready = true;
-            FA_TRACE(2, 8, jp);
+            ++p_waits[t];
+            if (jp == w.hi[t]) {
+              mma_commit(smem_u32(&sh->o_full[t]));
+              ++o_units[t];
+            }
+            if (t == 1 || !pv_use[1]) {
+              mma_commit(kv_empty0 + 8u * vslot);   // last reader of V_{j-1}
+              v_done = true;
+            }
           }
-          FA_TRACE(2, 11 + t, jp);
-          if (!mbar_wait(smem_u32(&sh->p_full[t]), p_waits[t] & 1u, p.wait_limit_ns)) {
+          if (s_use[t]) {
+            // S_t(j) = Q_t K_j^T   (issued after PV_t(j-1), which read P_t from these columns)
+            if (!k_ready) {
+              if (!mbar_wait(kfull, kpar, lim)) {
+                record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
+              }
+              k_ready = true;
+              tc_fence_after();
+            }
+            issue_s<D, DT>(tbase + 128 * t, opaque(q_desc0) + t * SLOT_DESC, k_desc, hi);
+            mma_commit(s_full0 + 8u * t);
+            if (t == 1 || !s_use[1]) {
+              mma_commit(kv_empty0 + 8u * kslot);   // last reader of K_j
+              k_done = true;
+            }
+          }
+        }
+        if (!ok) break;
+        // a loaded block nobody read (not expected): release it once it has landed
+        if (!k_done) {
+          if (!mbar_wait(kfull, kpar, lim)) {
             record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
           }
-          ++p_waits[t];
-          FA_TRACE(2, 1 + 3 * t, jp);
-          if (jp == w.lo[t]) {
-            // O_t must have been read out by the previous unit's epilogue
-            if (!mbar_wait(smem_u32(&sh->o_empty[t]), (o_units[t] & 1u) ^ 1u, p.wait_limit_ns)) {
-              record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
-            }
-          }
-          tc_fence_after();
-          issue_pv<D, DT>(o_tmem[t], p_tmem[t], ring + vslot * C::TILE_BYTES, jp > w.lo[t]);
-          FA_TRACE(2, 2 + 3 * t, jp);
-          if (jp == w.hi[t]) {
-            mma_commit(smem_u32(&sh->o_full[t]));
-            ++o_units[t];
-          }
-          if (t == 1 || !pv_use[1]) {
-            mma_commit(smem_u32(&sh->kv_empty[vslot]));   // last reader of V_{j-1}
-            v_done = true;
-          }
+          mma_commit(kv_empty0 + 8u * kslot);
         }
-        if (s_use[t]) {
-          // S_t(j) = Q_t K_j^T   (issued after PV_t(j-1), which read P_t from these columns)
-          if (!k_ready) {
-            FA_TRACE(2, 9, j);
-            if (!mbar_wait(smem_u32(&sh->kv_full[kslot]), (kidx / C::STAGES) & 1u, p.wait_limit_ns)) {
-              record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
-            }
-            k_ready = true;
-            FA_TRACE(2, 7, j);
-            tc_fence_after();
+        if (!v_done) {
+          if (!mbar_wait(vfull, vpar, lim)) {
+            record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
           }
-          issue_s<D, DT>(s_tmem[t], opaque(sq) + t * C::TILE_BYTES, ring + kslot * C::TILE_BYTES);
-          mma_commit(smem_u32(&sh->s_full[t]));
-          FA_TRACE(2, 3 + 3 * t, j);
-          if (t == 1 || !s_use[1]) {
-            mma_commit(smem_u32(&sh->kv_empty[kslot]));   // last reader of K_j
-            k_done = true;
-          }
+          mma_commit(kv_empty0 + 8u * vslot);
         }
       }
-      if (!ok) break;
-      // a loaded block nobody read (not expected): release it once it has landed
-      if (!k_done) {
-        if (!mbar_wait(smem_u32(&sh->kv_full[kslot]), (kidx / C::STAGES) & 1u, p.wait_limit_ns)) {
-          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
-        }
-        mma_commit(smem_u32(&sh->kv_empty[kslot]));
-      }
-      if (!v_done) {
-        if (!mbar_wait(smem_u32(&sh->kv_full[vslot]), (vidx / C::STAGES) & 1u, p.wait_limit_ns)) {
-          record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
-        }
-        mma_commit(smem_u32(&sh->kv_empty[vslot]));
+      if (j <= w.jhi) {
+        // V_j follows K_j, and K_{j+1} follows V_j in the ring
+        vslot = kslot; vpar = kpar;
+        ring_next<C::STAGES>(vslot, vpar);
+        kslot = vslot; kpar = vpar;
+        ring_next<C::STAGES>(kslot, kpar);
       }
     }
     if (!ok) break;
     mma_commit(smem_u32(&sh->q_empty));
-    kv_base += 2u * (w.jhi - w.jlo + 1);
   }
+  FA_TRACE(2, 15, 0);
   // all issued MMAs complete before the CTA releases TMEM
   mma_commit(smem_u32(&sh->mma_done));
-  if (!mbar_wait(smem_u32(&sh->mma_done), 0, p.wait_limit_ns)) record_error(sh, p, ST_TIMEOUT_DRAIN);
+  if (!mbar_wait(smem_u32(&sh->mma_done), 0, lim)) record_error(sh, p, ST_TIMEOUT_DRAIN);
 }
 
 // ------------------------------------------------------------------ softmax
@@ -566,7 +690,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Exponentiate this thread's 64 scores of a row, write P (16-bit or e4m3)
+// Exponentiate chunks [Q0, Q0+NQ) of 16 of this thread's 64 scores of a
+// row, write P (16-bit or e4m3)
 // into TMEM at p_addr (16x32bx2 layout: lanes 0-15 of the access for
 // threads 0-15, the same lanes half a row of P further for threads 16-31)
 // and return their fp32 sum twice: exact, and over the values P*V uses
@@ -582,14 +707,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 #define FA_EMU_FROM 8
 #endif
 
-template <int DT, bool EMULATE>
+template <int DT, bool EMULATE, int Q0, int NQ>
 __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_mref, uint32_t p_addr) {
   const float2 cc2 = make_float2(cc, cc);
   const float2 nm2 = make_float2(neg_mref, neg_mref);
   float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   float2 accq = make_float2(0.f, 0.f);   // e4m3 only: sum of the rounded values
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = Q0; q < Q0 + NQ; ++q) {
     uint32_t pw[8];
     float2 prev = make_float2(0.f, 0.f);
 #pragma unroll
@@ -657,6 +782,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     const int u = *reinterpret_cast<volatile int*>(&sh->uq[qs]);
     __syncwarp();
     if (lane_id() == 0) mbar_arrive(smem_u32(&sh->uq_empty[qs]));
+    FA_TRACE(t, 8, 0);
     if (u < 0) break;
     const Tile w = get_tile(u, t, p);
     if (!w.rows) continue;
@@ -681,6 +807,11 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     float l = 0.f;              // this thread's share of the row sum (exact)
     float lq = 0.f;             // ... of the stored P values (differs for e4m3)
     for (int j = w.lo; j <= w.hi; ++j) {
+      // boundary blocks (causal diagonal, window edge, key tail), decided
+      // before S arrives
+      const int k0 = j * BLOCK_N;
+      const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
+                             (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
       bool got = mbar_wait(smem_u32(&sh->s_full[t]), s_waits & 1u, p.wait_limit_ns);
       got = __all_sync(0xffffffffu, got);
       if (!got) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
@@ -692,10 +823,6 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       tmem_ld_16x32bx2_x32<64>(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
       tmem_wait_ld();
       FA_TRACE(t, 2, j);
-      // mask boundary blocks (causal diagonal, window edge, key tail)
-      const int k0 = j * BLOCK_N;
-      const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
-                             (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
       if (need_mask) {
         const int kh = k0 + half * HALF_N;
         const int hi_c = min(p.Nk - kh, p.causal ? row - kh + 1 : HALF_N);
@@ -704,6 +831,19 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
         for (int c = 0; c < HALF_N; ++c)
           if (c < lo_c || c >= hi_c) s[c] = -INFINITY;
       }
+#if FA_MAXTREE
+      // half-row max: a tree of 3-input max four levels deep (64 -> 22 -> 8
+      // -> 3 -> 1), then the other half's lane
+      float m1[22];
+#pragma unroll
+      for (int i = 0; i < 21; ++i) m1[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+      m1[21] = s[63];
+      float m2[8];
+#pragma unroll
+      for (int i = 0; i < 7; ++i) m2[i] = fmax3(m1[3 * i], m1[3 * i + 1], m1[3 * i + 2]);
+      m2[7] = m1[21];
+      const float mx_half = fmax3(fmax3(m2[0], m2[1], m2[2]), fmax3(m2[3], m2[4], m2[5]), fmaxf(m2[6], m2[7]));
+#else
       // half-row max (8 chains of 3-input max), then the other half's lane
       float mx8[8];
 #pragma unroll
@@ -713,22 +853,26 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
 #pragma unroll
         for (int q = 0; q < 8; ++q) mx8[q] = fmax3(mx8[q], s[c + q], s[c + 8 + q]);
       const float mx_half = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+#endif
       const float mx = fmaxf(mx_half, __shfl_xor_sync(0xffffffffu, mx_half, 16));
       const float m_blk = mx * cc;   // -inf stays -inf (cc > 0)
       const float m_cand = fmaxf(m_used, m_blk);
       const bool need = m_cand > m_used + C::RESCALE_THRESHOLD;
       const bool warp_rescale = __any_sync(0xffffffffu, need);
-      // alpha rescales O and l from the old reference to the new one
-      float alpha = 1.f;
-      if (warp_rescale) {
-        alpha = (m_cand == -INFINITY) ? 1.f : ex2_approx(m_used - m_cand);
-        m_used = m_cand;
-      }
+      // The new reference is a select, so the exponentials start right
+      // away; alpha, which rescales O and l from the old reference to the
+      // new one (one MUFU op, rarely needed), is taken after them.
+      const float m_old = m_used;
+      m_used = warp_rescale ? m_cand : m_used;
       const float mref = (m_used == -INFINITY) ? 0.f : (m_used - C::PSHIFT);
       FA_TRACE(t, 3, j);
-      const float2 lsum = need_mask ? exp_half<DT, false>(s, cc, -mref, p_addr)
-                                    : exp_half<DT, true>(s, cc, -mref, p_addr);
-      FA_TRACE(t, 4, j);
+      // chunks of 16 scores exponentiated before the first hand-over: with
+      // the split hand-over, P over keys k with k mod 64 < 32 goes first
+      constexpr int NQ0 = C::PSPLIT ? 2 : 4;
+      float2 lsum = need_mask ? exp_half<DT, false, 0, NQ0>(s, cc, -mref, p_addr)
+                              : exp_half<DT, true, 0, NQ0>(s, cc, -mref, p_addr);
+      float alpha = 1.f;
+      if (warp_rescale) alpha = (m_cand == -INFINITY) ? 1.f : ex2_approx(m_old - m_cand);
       // O rescale of this thread's half row (only when some row of this warp
       // raised its reference); PV_t(j-1) has completed: S_t(j) was issued
       // after it and has landed.
@@ -748,6 +892,18 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
           tmem_st_16x32bx2_x16<HALF_D>(o_addr + c, o);
         }
       }
+      if constexpr (C::PSPLIT) {
+        // the first PV MMAs run while the rest of P is exponentiated; O was
+        // rescaled (above) before this first hand-over
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sh->p_half[t]));
+        FA_TRACE(t, 12, j);
+        const float2 ls2 = need_mask ? exp_half<DT, false, 2, 2>(s, cc, -mref, p_addr)
+                                     : exp_half<DT, true, 2, 2>(s, cc, -mref, p_addr);
+        lsum = make_float2(lsum.x + ls2.x, lsum.y + ls2.y);
+      }
+      FA_TRACE(t, 4, j);
       l = fmaf(l, alpha, lsum.x);
       lq = fmaf(lq, alpha, lsum.y);
       tmem_wait_st();
@@ -763,6 +919,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     got = __all_sync(0xffffffffu, got);
     if (!got) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
     ++units;
+    FA_TRACE(t, 6, 0);
     tc_fence_after();
     const float inv = (lq_row > 0.f ? 1.f / lq_row : 0.f) * p.out_scale;
     uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) +
@@ -782,7 +939,9 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       p.lse[(static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row] =
           l_row > 0.f ? (m_used + __log2f(l_row) - C::PSHIFT) * 0.69314718055994531f : -INFINITY;
     }
+    FA_TRACE(t, 7, 0);
   }
+  FA_TRACE(t, 15, 0);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -810,7 +969,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&sh->s_full[t]), 1);
-      mbar_init(smem_u32(&sh->p_full[t]), 256);
+      mbar_init(smem_u32(&sh->p_full[t]), 256);   // every thread of the tile's two softmax warpgroups
+      mbar_init(smem_u32(&sh->p_half[t]), 256);
       mbar_init(smem_u32(&sh->o_full[t]), 1);
       mbar_init(smem_u32(&sh->o_empty[t]), 256);
     }
@@ -820,6 +980,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&sh->uq_empty[i]), UQ_CONSUMERS);
     }
     sh->abort_flag = 0;
+#ifdef FA_STATS_BUILD
+    for (int i = 0; i < 64; ++i) sh->stats[i] = 0u;
+#endif
     fence_mbar_init();
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
@@ -852,6 +1015,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
+#ifdef FA_STATS_BUILD
+  if (threadIdx.x == 0)
+    for (int i = 0; i < 64; ++i) atomicAdd(&g_stats[i], static_cast<unsigned long long>(sh->stats[i]));
+#endif
   if (threadIdx.x == 0) {
     // this CTA claims no more units; the last CTA to get here zeroes the
     // scheduler scratch for the next launch (every CTA gets here: all waits

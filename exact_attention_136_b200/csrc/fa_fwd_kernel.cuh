@@ -831,19 +831,6 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
         for (int c = 0; c < HALF_N; ++c)
           if (c < lo_c || c >= hi_c) s[c] = -INFINITY;
       }
-#if FA_MAXTREE
-      // half-row max: a tree of 3-input max four levels deep (64 -> 22 -> 8
-      // -> 3 -> 1), then the other half's lane
-      float m1[22];
-#pragma unroll
-      for (int i = 0; i < 21; ++i) m1[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
-      m1[21] = s[63];
-      float m2[8];
-#pragma unroll
-      for (int i = 0; i < 7; ++i) m2[i] = fmax3(m1[3 * i], m1[3 * i + 1], m1[3 * i + 2]);
-      m2[7] = m1[21];
-      const float mx_half = fmax3(fmax3(m2[0], m2[1], m2[2]), fmax3(m2[3], m2[4], m2[5]), fmaxf(m2[6], m2[7]));
-#else
       // half-row max (8 chains of 3-input max), then the other half's lane
       float mx8[8];
 #pragma unroll
@@ -853,7 +840,6 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
 #pragma unroll
         for (int q = 0; q < 8; ++q) mx8[q] = fmax3(mx8[q], s[c + q], s[c + 8 + q]);
       const float mx_half = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
-#endif
       const float mx = fmaxf(mx_half, __shfl_xor_sync(0xffffffffu, mx_half, 16));
       const float m_blk = mx * cc;   // -inf stays -inf (cc > 0)
       const float m_cand = fmaxf(m_used, m_blk);

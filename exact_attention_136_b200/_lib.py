@@ -28,6 +28,8 @@ SIGNATURES = {
                         _c_int, _c_int, _c_int, _vp]),
     "fa_fwd_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                             _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
+    "fa_fwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                            _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
     "fa_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                              _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, _c_float,
                              _c_float, _vp]),

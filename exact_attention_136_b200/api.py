@@ -30,11 +30,14 @@ def _check_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
     if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _DT:
         raise ValueError("q, k, v must share one dtype: float16, bfloat16 or float8_e4m3fn")
     B, n_q, H, D = q.shape
-    if k.shape[0] != B or k.shape[2:] != (H, D) or v.shape != k.shape:
-        raise ValueError("k and v must be [B, N_k, H, D] with q's B, H, D")
+    h_kv = k.shape[2]
+    if k.shape[0] != B or k.shape[3] != D or v.shape != k.shape:
+        raise ValueError("k and v must be [B, N_k, H_kv, D] with q's B and D")
+    if h_kv < 1 or H % h_kv != 0:
+        raise ValueError("q's head count must be a multiple of k's and v's (grouped-query attention)")
     if not (q.device == k.device == v.device):
         raise ValueError("q, k, v must be on one device")
-    return B, n_q, k.shape[1], H, D
+    return B, n_q, k.shape[1], H, h_kv, D
 
 
 def _outputs(q, B, n_q, H, D, out, lse, want_lse):
@@ -59,19 +62,26 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
 
     scale=None means 1/sqrt(headdim), the pages' auto scale (Workflow 2,
     Step 2).  window_left=-1 means no window.  For float8_e4m3fn inputs all
-    descales are 1; use forward_fp8 to pass per-tensor scales.
+    descales are 1; use forward_fp8 to pass per-tensor scales.  k and v may
+    have fewer heads than q (multi-query / grouped-query attention, Workflow
+    2, Step 3): query head h then reads head h // (H / H_kv).
     """
-    B, n_q, n_k, H, D = _check_inputs(q, k, v)
+    B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
     if q.dtype == torch.float8_e4m3fn:
         return forward_fp8(q, k, v, 1.0, 1.0, 1.0, scale, causal, window_left, out, lse, return_lse, stream)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     out, lse = _outputs(q, B, n_q, H, D, out, lse, return_lse)
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
-        rc = _lib.lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                               lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, D, scale,
-                               int(bool(causal)), int(window_left), _DT[q.dtype], s.cuda_stream)
-    _lib.check(rc, "fa_fwd")
+        lse_p = lse.data_ptr() if lse is not None else None
+        if h_kv == H:
+            rc = _lib.lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_p, B, n_q, n_k, H,
+                                   D, scale, int(bool(causal)), int(window_left), _DT[q.dtype], s.cuda_stream)
+        else:
+            rc = _lib.lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_p, B, n_q,
+                                       n_k, H, h_kv, D, scale, int(bool(causal)), int(window_left), _DT[q.dtype],
+                                       1.0, 1.0, 1.0, s.cuda_stream)
+    _lib.check(rc, "fa_fwd" if h_kv == H else "fa_fwd_gqa")
     return out, lse
 
 
@@ -80,18 +90,23 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
                 window_left: int = -1, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                 return_lse: bool = True, stream: Optional[torch.cuda.Stream] = None):
     """FP8 e4m3 forward with per-tensor descales; out is bfloat16."""
-    B, n_q, n_k, H, D = _check_inputs(q8, k8, v8)
+    B, n_q, n_k, H, h_kv, D = _check_inputs(q8, k8, v8)
     if q8.dtype != torch.float8_e4m3fn:
         raise ValueError("forward_fp8 takes float8_e4m3fn tensors")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     out, lse = _outputs(q8, B, n_q, H, D, out, lse, return_lse)
     with torch.cuda.device(q8.device):
         s = stream if stream is not None else torch.cuda.current_stream(q8.device)
-        rc = _lib.lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
-                                   lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, D, scale,
-                                   int(bool(causal)), int(window_left), float(q_descale), float(k_descale),
-                                   float(v_descale), s.cuda_stream)
-    _lib.check(rc, "fa_fwd_fp8")
+        lse_p = lse.data_ptr() if lse is not None else None
+        if h_kv == H:
+            rc = _lib.lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(), lse_p, B, n_q,
+                                       n_k, H, D, scale, int(bool(causal)), int(window_left), float(q_descale),
+                                       float(k_descale), float(v_descale), s.cuda_stream)
+        else:
+            rc = _lib.lib().fa_fwd_gqa(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(), lse_p, B, n_q,
+                                       n_k, H, h_kv, D, scale, int(bool(causal)), int(window_left), _lib.FA_E4M3,
+                                       float(q_descale), float(k_descale), float(v_descale), s.cuda_stream)
+    _lib.check(rc, "fa_fwd_fp8" if h_kv == H else "fa_fwd_gqa")
     return out, lse
 
 

@@ -115,8 +115,8 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUtensorMap mq, mk, mv;
   if (encode_bnhd(&mq, q, tdt, C::ES, p.B, p.Nq, p.H, D, C::BOX_INNER, BLOCK_M) ||
-      encode_bnhd(&mk, k, tdt, C::ES, p.B, p.Nk, p.H, D, C::BOX_INNER, BLOCK_N) ||
-      encode_bnhd(&mv, v, tdt, C::ES, p.B, p.Nk, p.H, D, C::BOX_INNER, BLOCK_N))
+      encode_bnhd(&mk, k, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N) ||
+      encode_bnhd(&mv, v, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N))
     return FA_ERR_CUDA;
   if (!(ds->attr_set & (1u << bit))) {
     if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -142,8 +142,9 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
 }
 
 int validate(const void* q, const void* k, const void* v, void* out, int B, int Nq, int Nk, int H,
-             int D, float scale, int causal, int window_left, int dtype) {
+             int D, float scale, int causal, int window_left, int dtype, int Hkv) {
   if (B < 1 || H < 1 || Nq < 0 || Nk < 0) return FA_ERR_ARG;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_ARG;
   // q / out may be NULL only when there are no queries, k / v only when there are no keys
   if ((Nq > 0 && (!q || !out)) || (Nk > 0 && (!k || !v))) return FA_ERR_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_ARG;
@@ -154,16 +155,16 @@ int validate(const void* q, const void* k, const void* v, void* out, int B, int 
   if (dtype == FA_E4M3 && D != 128) return FA_ERR_UNSUPPORTED;
   // TMA coordinates are 32-bit; keep every index well inside int range
   const int64_t rows_q = static_cast<int64_t>(B) * Nq * H;
-  const int64_t rows_k = static_cast<int64_t>(B) * Nk * H;
+  const int64_t rows_k = static_cast<int64_t>(B) * Nk * Hkv;
   if (rows_q > (int64_t(1) << 31) || rows_k > (int64_t(1) << 31)) return FA_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FA_ERR_ALIGN;
   return FA_OK;
 }
 
 int forward(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Nq, int Nk,
-            int H, int D, float scale, int causal, int window_left, int dtype, float qd, float kd,
+            int H, int Hkv, int D, float scale, int causal, int window_left, int dtype, float qd, float kd,
             float vd, cudaStream_t stream, unsigned* sched_override = nullptr) {
-  int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype);
+  int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
   if (rc != FA_OK) return rc;
   if (!(qd > 0.f) || !std::isfinite(qd) || !(kd > 0.f) || !std::isfinite(kd) || !(vd > 0.f) ||
       !std::isfinite(vd))
@@ -187,6 +188,8 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   p.Nq = Nq;
   p.Nk = Nk;
   p.H = H;
+  p.Hkv = Hkv;
+  p.qpk = H / Hkv;
   p.causal = causal;
   p.window_left = window_left;
   p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
@@ -201,7 +204,8 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   // 2 * N_k * D * element size) take at most ~48 MB of the 126 MB L2 and it
   // still spans about two waves of units
   if (causal) {
-    const double kv_head = 2.0 * Nk * D * static_cast<double>(dtype == FA_E4M3 ? 1 : 2);
+    // (query heads of a group share one K/V head: count each head's share)
+    const double kv_head = 2.0 * Nk * D * static_cast<double>(dtype == FA_E4M3 ? 1 : 2) / p.qpk;
     int g = static_cast<int>(48.0e6 / kv_head);
     const int want = (2 * ds->num_sms + p.pairs - 1) / p.pairs;
     g = g < want ? g : want;
@@ -231,15 +235,22 @@ extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q, int N_k,
            int H, int D, float scale, int causal, int window_left, int dtype, fa_stream_t stream) {
-  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, D, scale, causal, window_left, dtype, 1.f, 1.f,
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H, D, scale, causal, window_left, dtype, 1.f, 1.f,
                      1.f, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q,
                int N_k, int H, int D, float scale, int causal, int window_left, float q_descale,
                float k_descale, float v_descale, fa_stream_t stream) {
-  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, D, scale, causal, window_left, FA_E4M3,
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H, D, scale, causal, window_left, FA_E4M3,
                      q_descale, k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q, int N_k,
+               int H, int H_kv, int D, float scale, int causal, int window_left, int dtype, float q_descale,
+               float k_descale, float v_descale, fa_stream_t stream) {
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, q_descale,
+                     k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,
@@ -247,7 +258,7 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* l
                 int causal, int window_left, int dtype, float q_descale, float k_descale,
                 float v_descale, fa_stream_t stream) {
   if (!q || !k || !v || !out) return FA_ERR_ARG;
-  int rc = fa::validate(dq, dk, dv, dout, B, N_q, N_k, H, D, scale, causal, window_left, dtype);
+  int rc = fa::validate(dq, dk, dv, dout, B, N_q, N_k, H, D, scale, causal, window_left, dtype, H);
   if (rc != FA_OK) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t es = fa::elem_bytes(dtype);
@@ -257,7 +268,7 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* l
       cudaMemcpyAsync(dk, k, nk * es, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(dv, v, nk * es, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return FA_ERR_CUDA;
-  rc = fa::forward(dq, dk, dv, dout, dlse, B, N_q, N_k, H, D, scale, causal, window_left, dtype,
+  rc = fa::forward(dq, dk, dv, dout, dlse, B, N_q, N_k, H, H, D, scale, causal, window_left, dtype,
                    q_descale, k_descale, v_descale, s);
   if (rc != FA_OK) return rc;
   if (cudaMemcpyAsync(out, dout, nq * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_CUDA;
@@ -271,7 +282,7 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* l
 int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q,
                    int N_k, int H, int D, float scale, int causal, int window_left, int dtype,
                    float q_descale, float k_descale, float v_descale, fa_stream_t stream) {
-  int rc = fa::validate(q, k, v, out, B, N_q, N_k, H, D, scale, causal, window_left, dtype);
+  int rc = fa::validate(q, k, v, out, B, N_q, N_k, H, D, scale, causal, window_left, dtype, H);
   if (rc != FA_OK) return rc;
   // the scheduler's counters index work units as 32-bit values: problems with
   // more units than that (or a scratch need above the array) are rejected
@@ -288,7 +299,7 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float
   // the counters must start at zero; every launch also leaves them at zero
   if (cudaMemsetAsync(scratch, 0, sizeof(unsigned) * fa::kSchedWordsNeeded, s) != cudaSuccess)
     return FA_ERR_CUDA;
-  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, D, scale, causal, window_left, dtype, q_descale,
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H, D, scale, causal, window_left, dtype, q_descale,
                      k_descale, v_descale, s, scratch);
 }
 

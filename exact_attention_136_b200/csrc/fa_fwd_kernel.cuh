@@ -63,6 +63,8 @@ struct FwdParams {
   void* out;           // [B, N_q, H, D] fp16 (fp16 inputs) or bf16
   float* lse;          // [B, H, N_q] fp32, may be null
   int B, Nq, Nk, H;
+  int Hkv;             // key/value heads (H a multiple of Hkv)
+  int qpk;             // H / Hkv: query head h reads K/V head h / qpk
   int causal;
   int window_left;     // -1 = unlimited
   float score_scale;   // scale * log2(e) * q_descale * k_descale
@@ -134,6 +136,7 @@ static_assert(sizeof(SharedHeader) <= HEADER_BYTES, "header");
 // One 128-row query tile of a work unit and its key-block range.
 struct Tile {
   int b, h, qs;    // batch, head, first query row
+  int hk;          // key/value head of this query head
   int lo, hi;      // inclusive key-block range
   bool rows;       // tile has rows (qs < N_q)
   bool valid;      // ... and at least one key block
@@ -156,6 +159,7 @@ __device__ __forceinline__ Tile get_tile(int u, int t, const FwdParams& p) {
   const int m = p.causal ? (p.pairs - 1 - m_idx) : m_idx;
   w.b = bh / p.H;
   w.h = bh - w.b * p.H;
+  w.hk = w.h / p.qpk;
   w.qs = m * (2 * BLOCK_M) + t * BLOCK_M;
   w.rows = w.qs < p.Nq;
   const int qe = min(w.qs + BLOCK_M - 1, p.Nq - 1);
@@ -167,7 +171,7 @@ __device__ __forceinline__ Tile get_tile(int u, int t, const FwdParams& p) {
 
 // Both tiles of a work unit and the union of their key-block ranges.
 struct Unit {
-  int b, h, q0;
+  int b, h, hk, q0;
   int lo[2], hi[2];
   bool valid[2];
   int jlo, jhi;    // empty (jhi < 0) when neither tile has work
@@ -179,6 +183,7 @@ __device__ __forceinline__ Unit get_unit(int u, const FwdParams& p) {
   Unit w;
   w.b = a.b;
   w.h = a.h;
+  w.hk = a.hk;
   w.q0 = a.qs;
   w.lo[0] = a.lo; w.hi[0] = a.hi; w.valid[0] = a.valid;
   w.lo[1] = c.lo; w.hi[1] = c.hi; w.valid[1] = c.valid;
@@ -327,7 +332,7 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d_hint(smem_u32(ring + slot * C::TILE_BYTES + c * C::CHUNK_BYTES), map, bar,
-                           c * C::BOX_INNER, w.h, j * BLOCK_N, w.b, pol_kv);
+                           c * C::BOX_INNER, w.hk, j * BLOCK_N, w.b, pol_kv);
         issued_mask |= 1u << slot;
         phase_mask = (phase_mask & ~(1u << slot)) | ((round & 1u) << slot);
         ++kv_it;

@@ -65,11 +65,13 @@ def quantize_e4m3(x: torch.Tensor):
 
 
 def make_qkv(B: int, n_q: int, n_k: int, H: int, D: int, dtype: str,
-             seeds=(1001, 1002, 1003)) -> QKV:
-    """Q [B, n_q, H, D], K and V [B, n_k, H, D] drawn N(0, 1) from the given seeds."""
+             seeds=(1001, 1002, 1003), h_kv: int = None) -> QKV:
+    """Q [B, n_q, H, D], K and V [B, n_k, h_kv, D] (h_kv defaults to H) drawn
+    N(0, 1) from the given seeds."""
+    h_kv = H if h_kv is None else h_kv
     q = randn((B, n_q, H, D), seeds[0])
-    k = randn((B, n_k, H, D), seeds[1])
-    v = randn((B, n_k, H, D), seeds[2])
+    k = randn((B, n_k, h_kv, D), seeds[1])
+    v = randn((B, n_k, h_kv, D), seeds[2])
     if dtype == "e4m3":
         q8, sq = quantize_e4m3(q)
         k8, sk = quantize_e4m3(k)

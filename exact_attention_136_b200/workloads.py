@@ -31,6 +31,11 @@ class Workload:
     scale: float
     index: int          # seed offset: seeds are 1001/1002/1003 + 100 * index
     desc: str
+    kv_heads: int = 0   # K/V heads (0 = H); fewer for multi-/grouped-query attention
+
+    @property
+    def h_kv(self):
+        return self.kv_heads if self.kv_heads > 0 else self.H
 
     @property
     def seeds(self):
@@ -59,6 +64,10 @@ WORKLOADS = {
     "b4h32n4096d64_fp16": Workload(
         "b4h32n4096d64_fp16", 4, 4096, 4096, 32, 64, "fp16", False, -1, 1.0 / 8.0, 5,
         "non-causal B4 N4096 H32 D64 fp16 (the pages' flash-attn timing shape)"),
+    "gqa_causal_b4h32kv8n8192d128_bf16": Workload(
+        "gqa_causal_b4h32kv8n8192d128_bf16", 4, 8192, 8192, 32, 128, "bf16", True, -1,
+        1.0 / math.sqrt(128.0), 6,
+        "grouped-query causal B4 H32 (8 K/V heads) N8192 D128 bf16, scale 1/sqrt(128)", 8),
 }
 
 # order used by tests; the headline bench workload is the causal bf16 D128 case

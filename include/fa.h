@@ -87,6 +87,22 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* ls
                fa_stream_t stream);
 
 /*
+ * fa_fwd_gqa -- multi-query / grouped-query attention (Flash Attention |
+ * Hermes Skill, Workflow 2, Step 3 "Enable advanced features": K and V with
+ * fewer heads than Q, shared across query heads).  k and v are
+ * [B, N_k, H_kv, D]; q and out [B, N_q, H, D]; H must be a multiple of
+ * H_kv >= 1, and query head h reads key/value head h / (H / H_kv)
+ * (contiguous groups: the pages do not fix the grouping, this is the
+ * plainest reading).  H_kv = 1 is multi-query, H_kv = H the same as
+ * fa_fwd / fa_fwd_fp8.  Every other argument, the descales (all 1 for
+ * 16-bit inputs) and the return values as for fa_fwd / fa_fwd_fp8.
+ */
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* lse,
+               int B, int N_q, int N_k, int H, int H_kv, int D, float scale, int causal,
+               int window_left, int dtype, float q_descale, float k_descale, float v_descale,
+               fa_stream_t stream);
+
+/*
  * fa_fwd_host -- the same forward on HOST buffers: copies q, k, v from host
  * to the caller's device buffers dq, dk, dv, runs fa_fwd / fa_fwd_fp8 into
  * dout / dlse, and copies out (and lse, when both lse and dlse are non-NULL)

@@ -35,6 +35,14 @@ arguments; Flash Attention | Hermes Skill, Workflow 2, Steps 2-3):
 Indices are absolute (top-left aligned) also when N_q != N_k; this is the
 plainest reading, since the pages only show N_q == N_k.
 
+Multi-query / grouped-query attention (Flash Attention | Hermes Skill,
+Workflow 2, Step 3 "Enable advanced features": K and V may have fewer heads
+than Q, "shared K/V across heads").  The pages do not say which query heads
+share a K/V head; the reading here is contiguous groups: with H query heads
+and H_kv key/value heads (H a multiple of H_kv), query head h uses key/value
+head h // (H / H_kv).  H_kv = 1 is multi-query attention, H_kv = H the
+ordinary case.
+
 Layouts follow the pages' flash_attn_func layout ``[batch, seqlen, nheads,
 headdim]`` for Q, K, V and O (Workflow 2, Step 2), and ``[batch, heads,
 N_q]`` for LSE (the pages print no LSE layout; this is our reading).
@@ -80,7 +88,9 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
                   rows=None, return_probs: bool = False):
     """Exact attention forward in float64 (definition in the module docstring).
 
-    q: [B, N_q, H, D]; k, v: [B, N_k, H, D] (any real dtype; upcast to fp64).
+    q: [B, N_q, H, D]; k, v: [B, N_k, H_kv, D] with H a multiple of H_kv
+       (query head h reads key/value head h // (H / H_kv)); any real dtype,
+       upcast to fp64.
     rows: optional 1-D array of query indices; only those rows are computed
           (used for long sequences where the full N_q x N_k matrix is large).
     Returns (O [B, R, H, D], LSE [B, H, R]) with R = len(rows) (or N_q), and
@@ -92,9 +102,12 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
     if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
         raise ValueError("q, k, v must be [batch, seqlen, heads, headdim]")
     B, n_q, H, D = q.shape
-    n_k = k.shape[1]
-    if k.shape != (B, n_k, H, D) or v.shape != (B, n_k, H, D):
-        raise ValueError("k and v must be [B, N_k, H, D] matching q")
+    n_k, h_kv = k.shape[1], k.shape[2]
+    if k.shape != (B, n_k, h_kv, D) or v.shape != (B, n_k, h_kv, D):
+        raise ValueError("k and v must be [B, N_k, H_kv, D] matching q")
+    if h_kv < 1 or H % h_kv != 0:
+        raise ValueError("the number of query heads must be a multiple of the key/value heads")
+    group = H // h_kv
     rows = np.arange(n_q, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     R = rows.shape[0]
     vis = visibility(rows, n_k, causal, window_left)
@@ -105,14 +118,15 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
     probs = np.zeros((B, H, R, n_k), dtype=np.float64) if return_probs else None
     for b in range(B):
         for h in range(H):
+            hk = h // group   # key/value head shared by this query head's group
             # scores of every selected query against every key
-            s = scale * (q[b, rows, h, :] @ k[b, :, h, :].T)
+            s = scale * (q[b, rows, h, :] @ k[b, :, hk, :].T)
             s = np.where(vis, s, -np.inf)
             m = np.where(seen, s.max(axis=1, initial=-np.inf), 0.0)
             e = np.where(vis, np.exp(s - m[:, None]), 0.0)
             l = e.sum(axis=1)
             p = e / np.where(seen, l, 1.0)[:, None]
-            out[b, :, h, :] = p @ v[b, :, h, :]
+            out[b, :, h, :] = p @ v[b, :, hk, :]
             lse[b, h, :] = np.where(seen, m + np.log(np.where(seen, l, 1.0)), -np.inf)
             if return_probs:
                 probs[b, h] = p
@@ -127,17 +141,20 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
     Written independently of ``attention_ref``: nested lists, ``math.exp``, no
     max subtraction, and the visibility rule spelled out inline.  Used only to
     pin ``attention_ref``.  Returns (O, LSE) as nested Python lists shaped like
-    ``attention_ref``'s outputs.
+    ``attention_ref``'s outputs.  K and V may have fewer heads than Q (query
+    head h then reads head h * H_kv // H, the same contiguous groups).
     """
     B = len(q)
     n_q = len(q[0])
     H = len(q[0][0])
     D = len(q[0][0][0])
     n_k = len(k[0])
+    h_kv = len(k[0][0])
     O = [[[[0.0] * D for _ in range(H)] for _ in range(n_q)] for _ in range(B)]
     L = [[[float("-inf")] * n_q for _ in range(H)] for _ in range(B)]
     for b in range(B):
         for h in range(H):
+            g = h * h_kv // H
             for i in range(n_q):
                 weights = []
                 for j in range(n_k):
@@ -147,7 +164,7 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
                         continue
                     dot = 0.0
                     for d in range(D):
-                        dot += float(q[b][i][h][d]) * float(k[b][j][h][d])
+                        dot += float(q[b][i][h][d]) * float(k[b][j][g][d])
                     weights.append((j, math.exp(scale * dot)))
                 total = sum(w for _, w in weights)
                 if not weights:
@@ -156,6 +173,6 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
                 for d in range(D):
                     acc = 0.0
                     for j, w in weights:
-                        acc += w * float(v[b][j][h][d])
+                        acc += w * float(v[b][j][g][d])
                     O[b][i][h][d] = acc / total
     return O, L

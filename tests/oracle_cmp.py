@@ -21,6 +21,16 @@ def oracle(qkv, scale, causal, window_left, rows=None):
     """(O [B, R, H, D], LSE [B, H, R]) in float64 for the given QKV bundle."""
     B, n_q, H, D = qkv.q.shape
     R = n_q if rows is None else len(rows)
+    if qkv.k.shape[2] != H:
+        # grouped K/V heads: the oracle maps query heads to K/V heads itself
+        # (one batch at a time, all heads)
+        O = np.zeros((B, R, H, D))
+        L = np.zeros((B, H, R))
+        for b in range(B):
+            o, l = attention_ref(_f64(qkv.q[b:b + 1], qkv.q_descale), _f64(qkv.k[b:b + 1], qkv.k_descale),
+                                 _f64(qkv.v[b:b + 1], qkv.v_descale), scale, causal, window_left, rows=rows)
+            O[b], L[b] = o[0], l[0]
+        return O, L
     O = np.zeros((B, R, H, D))
     L = np.zeros((B, H, R))
     for b in range(B):

@@ -100,3 +100,17 @@ def test_python_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 4, 1, 64, dtype=torch.float16)
     with pytest.raises(ValueError):
         forward(x, x, x)
+
+
+@pytest.mark.parametrize("H, h_kv", [(8, 0), (8, 3), (6, 4), (4, 8), (8, -1)])
+def test_gqa_head_counts_validated(H, h_kv):
+    """H must be a positive multiple of H_kv; rejected on the host, before any GPU work."""
+    f = _lib.lib().fa_fwd_gqa
+    assert f(A, A, A, A, None, 1, 128, 128, H, h_kv, 128, 0.1, 0, -1, _lib.FA_BF16, 1.0, 1.0, 1.0,
+             None) == _lib.FA_ERR_ARG
+
+
+def test_gqa_descales_validated():
+    f = _lib.lib().fa_fwd_gqa
+    assert f(A, A, A, A, None, 1, 128, 128, 8, 2, 128, 0.1, 0, -1, _lib.FA_E4M3, 1.0, 0.0, 1.0,
+             None) == _lib.FA_ERR_ARG

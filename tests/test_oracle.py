@@ -300,3 +300,89 @@ def test_planted_mask_mistake_is_caught(monkeypatch, bad):
 
     monkeypatch.setattr(oa, "visibility", mutated)
     assert _caught(oa.attention_ref)
+
+
+# --------------------------------------------------------------------------
+# grouped / multi-query K/V heads (H_kv < H): query head h reads K/V head
+# h // (H / H_kv), the reading of "shared K/V across heads" stated in the
+# oracle's docstring
+# --------------------------------------------------------------------------
+
+def gqa_pin_bruteforce(fn):
+    """Against the brute force, whose head map is written as h * H_kv // H."""
+    for (H, h_kv) in [(4, 1), (4, 2), (6, 3), (6, 2)]:
+        for causal, wl in MODES[:5]:
+            q = _rand((1, 7, H, 4), 60 + H)
+            k = _rand((1, 9, h_kv, 4), 61 + h_kv)
+            v = _rand((1, 9, h_kv, 4), 62 + h_kv)
+            o, l = fn(q, k, v, 0.7, causal, wl)
+            ob, lb = attention_bruteforce(q.tolist(), k.tolist(), v.tolist(), 0.7, causal, wl)
+            np.testing.assert_allclose(o, np.array(ob), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(l, np.array(lb), rtol=0, atol=1e-12)
+
+
+def gqa_pin_constant_v_per_group(fn):
+    """V constant over keys and dims within each K/V head, different across heads:
+    every visible row of query head h returns K/V head h // (H / H_kv)'s constant."""
+    H, h_kv = 8, 4
+    q, k = _rand((2, 11, H, 8), 63), _rand((2, 11, h_kv, 8), 64)
+    consts = np.array([1.5, -2.0, 0.25, 7.0])
+    v = np.broadcast_to(consts[None, None, :, None], (2, 11, h_kv, 8)).copy()
+    for causal, wl in [(False, -1), (True, -1), (True, 2)]:
+        o, _ = fn(q, k, v, 0.9, causal, wl)
+        for h in range(H):
+            np.testing.assert_allclose(o[:, :, h, :], consts[h // 2], rtol=0, atol=1e-12)
+
+
+def gqa_pin_repeated_heads(fn):
+    """Sharing a K/V head equals giving each query head its own copy of it (numpy repeat)."""
+    H, h_kv = 6, 2
+    q, k, v = _rand((2, 13, H, 4), 65), _rand((2, 13, h_kv, 4), 66), _rand((2, 13, h_kv, 4), 67)
+    for causal, wl in MODES[:4]:
+        o, l = fn(q, k, v, 0.8, causal, wl)
+        o2, l2 = fn(q, np.repeat(k, H // h_kv, axis=2), np.repeat(v, H // h_kv, axis=2), 0.8, causal, wl)
+        np.testing.assert_allclose(o, o2, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l, l2, rtol=0, atol=1e-13)
+
+
+def gqa_pin_mqa_zero_query(fn):
+    """Multi-query (H_kv = 1) with Q = 0: every head returns the mean of the single V head's
+    visible rows and LSE = ln(#visible keys)."""
+    q = np.zeros((1, 9, 4, 4))
+    k, v = _rand((1, 9, 1, 4), 68), _rand((1, 9, 1, 4), 69)
+    o, l = fn(q, k, v, 1.3, True, 3)
+    for i in range(9):
+        lo = max(0, i - 3)
+        for h in range(4):
+            np.testing.assert_allclose(o[0, i, h], v[0, lo:i + 1, 0].mean(axis=0), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(l[0, h, i], math.log(i - lo + 1), rtol=0, atol=1e-12)
+
+
+GQA_PINS = [gqa_pin_bruteforce, gqa_pin_constant_v_per_group, gqa_pin_repeated_heads, gqa_pin_mqa_zero_query]
+
+
+@pytest.mark.parametrize("pin", GQA_PINS, ids=[p.__name__ for p in GQA_PINS])
+def test_oracle_gqa_pin(pin):
+    pin(attention_ref)
+
+
+def test_oracle_rejects_uneven_head_groups():
+    q, k = _rand((1, 4, 6, 4), 70), _rand((1, 4, 4, 4), 71)
+    with pytest.raises(ValueError):
+        attention_ref(q, k, k, 1.0)
+
+
+def test_planted_head_map_mistake_is_caught():
+    """An oracle that maps query head h to K/V head h mod H_kv (interleaved groups) fails a pin."""
+    def mutated(q, k, v, scale, causal=False, wl=-1, **kw):
+        H, h_kv = q.shape[2], k.shape[2]
+        idx = np.arange(H) % h_kv
+        return attention_ref(q, k[:, :, idx], v[:, :, idx], scale, causal, wl, **kw)
+
+    caught = False
+    for pin in GQA_PINS:
+        try:
+            pin(mutated)
+        except AssertionError:
+            caught = True
+    assert caught

@@ -96,6 +96,41 @@ def test_small_exact_parity(case):
     check(qkv, dt, 1.0 / math.sqrt(D), causal, wl)
 
 
+# grouped / multi-query K/V heads: (B, N_q, N_k, H, H_kv, D, dtype, causal, window_left)
+GQA = [
+    (1, 256, 256, 8, 1, 128, "bf16", True, -1),     # multi-query
+    (2, 300, 300, 8, 2, 64, "fp16", False, -1),
+    (1, 700, 700, 6, 3, 128, "bf16", True, 200),
+    (1, 513, 1025, 4, 2, 128, "fp16", True, -1),
+    (1, 1000, 1000, 8, 4, 128, "e4m3", True, -1),
+    (1, 129, 129, 4, 1, 64, "bf16", False, 50),
+]
+
+
+@pytest.mark.parametrize("case", GQA, ids=[
+    f"B{c[0]}_q{c[1]}_k{c[2]}_H{c[3]}_Hkv{c[4]}_D{c[5]}_{c[6]}_{'c' if c[7] else 'nc'}_w{c[8]}" for c in GQA])
+def test_gqa_parity(case):
+    B, nq, nk, H, h_kv, D, dt, causal, wl = case
+    qkv = inputs.make_qkv(B, nq, nk, H, D, dt, seeds=(41 + nq, 42 + nk, 43 + H), h_kv=h_kv)
+    check(qkv, dt, 1.0 / math.sqrt(D), causal, wl)
+
+
+def test_gqa_with_all_heads_equals_mha_entry():
+    """fa_fwd_gqa with H_kv = H is the ordinary forward, bit for bit."""
+    qkv = inputs.make_qkv(1, 384, 384, 4, 128, "bf16", seeds=(51, 52, 53))
+    dev = torch.device("cuda", 0)
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    o1, l1 = forward(q, k, v, 0.09, True, -1)
+    o2 = torch.empty_like(o1)
+    l2 = torch.empty_like(l1)
+    s = torch.cuda.current_stream()
+    rc = _lib.lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o2.data_ptr(), l2.data_ptr(), 1, 384, 384,
+                               4, 4, 128, 0.09, 1, -1, _lib.FA_BF16, 1.0, 1.0, 1.0, s.cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 @pytest.mark.parametrize("dt,D", [("fp16", 64), ("bf16", 128), ("e4m3", 128)])
 @pytest.mark.parametrize("mult", [4.0, 12.0])
 def test_large_scores_exercise_rescaling(dt, D, mult):
@@ -135,7 +170,7 @@ def test_pages_accuracy_check_bound():
 def test_full_workload_sampled_rows(name):
     """Every workload at full size; all rows finite, sampled rows of every head vs the oracle."""
     w = W.WORKLOADS[name]
-    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=w.seeds)
+    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=w.seeds, h_kv=w.h_kv)
     rows = W.sample_rows(w, count=64 if w.n_q > 4096 else 256)
     out, lse = run(qkv, w.scale, w.causal, w.window_left)
     assert bool(torch.isfinite(out).all()) and bool(torch.isfinite(lse).all())

@@ -224,6 +224,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=W.HEADLINE, choices=W.ORDER)
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--splits", type=int, default=None, help="override the workload's key-range slices")
     ap.add_argument("--cpu-rows", type=int, default=128, help="oracle rows per (batch, head) for cpu_baseline")
     ap.add_argument("--reference-rows", type=int, default=256, help="oracle rows per step in --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -260,12 +261,14 @@ def main():
     lse = torch.empty((w.B, w.H, w.n_q), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    splits = w.splits if args.splits is None else args.splits
+
     def step():
         if w.dtype == "e4m3":
             forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, w.scale, w.causal, w.window_left,
-                        out=out, lse=lse, stream=stream)
+                        out=out, lse=lse, stream=stream, num_splits=splits)
         else:
-            forward(q, k, v, w.scale, w.causal, w.window_left, out=out, lse=lse, stream=stream)
+            forward(q, k, v, w.scale, w.causal, w.window_left, out=out, lse=lse, stream=stream, num_splits=splits)
 
     def barrier():
         if world > 1:
@@ -311,7 +314,7 @@ def main():
     desc = (qkv.q_descale, qkv.k_descale, qkv.v_descale)
 
     def e2e_step():
-        if w.h_kv == w.H:
+        if w.h_kv == w.H and splits == 1:
             forward_host(hq, hk, hv, staging, w.scale, w.causal, w.window_left, desc, ho, hl, stream)
         else:
             # fa_fwd_host takes H K/V heads; grouped heads go through pinned
@@ -362,7 +365,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "desc": w.desc, "B": w.B, "N_q": w.n_q, "N_k": w.n_k, "H": w.H,
-                   "H_kv": w.h_kv, "D": w.D, "causal": w.causal, "window_left": w.window_left, "scale": w.scale,
+                   "H_kv": w.h_kv, "splits": splits, "D": w.D, "causal": w.causal, "window_left": w.window_left, "scale": w.scale,
                    "flop_per_step": flops,
                    "block_fraction": W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left),
                    "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB vs {L2_BYTES / 1e6:.0f} MB), no flush",
@@ -371,8 +374,8 @@ def main():
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps,
-                "api": "fa_fwd_host (pinned host buffers)" if w.h_kv == w.H
-                       else "pinned host copies + forward (fa_fwd_gqa)"},
+                "api": "fa_fwd_host (pinned host buffers)" if (w.h_kv == w.H and splits == 1)
+                       else "pinned host copies + forward"},
         "roofline": {"bound": "tensor", "achieved": per_launch_tflops, "peak": peak, "unit": UNIT,
                      "frac": per_launch_tflops / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 burst" + (" x2 for fp8" if w.dtype == "e4m3" else ""),

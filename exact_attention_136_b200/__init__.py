@@ -7,6 +7,6 @@ The computation runs in libfa_b200.so (hand-written sm_100a CUDA, C ABI in
 include/fa.h); this package only marshals arguments.
 """
 
-from .api import device_status, forward, forward_fp8, forward_host, set_wait_limit_ns, wait_probe
+from .api import auto_splits, device_status, forward, forward_fp8, forward_host, set_wait_limit_ns, wait_probe
 
-__all__ = ["forward", "forward_fp8", "forward_host", "device_status", "set_wait_limit_ns", "wait_probe"]
+__all__ = ["forward", "forward_fp8", "forward_host", "auto_splits", "device_status", "set_wait_limit_ns", "wait_probe"]

@@ -30,6 +30,10 @@ SIGNATURES = {
                             _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
     "fa_fwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                             _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
+    "fa_fwd_splitkv_workspace_bytes": (ctypes.c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "fa_fwd_splitkv": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _c_int, _vp, ctypes.c_size_t,
+                                _vp]),
     "fa_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                              _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, _c_float,
                              _c_float, _vp]),

@@ -54,26 +54,61 @@ def _outputs(q, B, n_q, H, D, out, lse, want_lse):
     return out, lse
 
 
+def auto_splits(B: int, n_q: int, n_k: int, H: int, device=None) -> int:
+    """Key-range slices that fill the GPU: one per SM for every work unit
+    (256 query rows of one (batch, head)) short of the SM count, at most one
+    per 128-key block; 1 when the units already cover the SMs."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    units = B * H * max(1, -(-n_q // 256))
+    if units >= sms:
+        return 1
+    return max(1, min(-(-n_k // 128), -(-sms // units)))
+
+
+def _splitkv(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, dt, descales,
+             num_splits, s):
+    """fa_fwd_splitkv with a workspace from PyTorch's allocator."""
+    nbytes = _lib.lib().fa_fwd_splitkv_workspace_bytes(B, n_q, n_k, H, D, num_splits)
+    ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=q.device)
+    rc = _lib.lib().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, h_kv, D, scale,
+                                   int(bool(causal)), int(window_left), dt, float(descales[0]),
+                                   float(descales[1]), float(descales[2]), int(num_splits),
+                                   ws.data_ptr() if nbytes else None, int(nbytes), s.cuda_stream)
+    _lib.check(rc, "fa_fwd_splitkv")
+
+
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
             causal: bool = False, window_left: int = -1, out: Optional[torch.Tensor] = None,
             lse: Optional[torch.Tensor] = None, return_lse: bool = True,
-            stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            stream: Optional[torch.cuda.Stream] = None,
+            num_splits: int = 1) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Exact attention forward; returns (out, lse).
 
     scale=None means 1/sqrt(headdim), the pages' auto scale (Workflow 2,
     Step 2).  window_left=-1 means no window.  For float8_e4m3fn inputs all
     descales are 1; use forward_fp8 to pass per-tensor scales.  k and v may
     have fewer heads than q (multi-query / grouped-query attention, Workflow
-    2, Step 3): query head h then reads head h // (H / H_kv).
+    2, Step 3): query head h then reads head h // (H / H_kv).  num_splits > 1
+    splits the key range into that many slices run in parallel and merged
+    (for few query rows against many keys); 0 picks it with auto_splits.
     """
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
+    if num_splits == 0:
+        num_splits = auto_splits(B, n_q, n_k, H, q.device)
     if q.dtype == torch.float8_e4m3fn:
-        return forward_fp8(q, k, v, 1.0, 1.0, 1.0, scale, causal, window_left, out, lse, return_lse, stream)
+        return forward_fp8(q, k, v, 1.0, 1.0, 1.0, scale, causal, window_left, out, lse, return_lse, stream,
+                           num_splits)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     out, lse = _outputs(q, B, n_q, H, D, out, lse, return_lse)
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
         lse_p = lse.data_ptr() if lse is not None else None
+        if num_splits > 1:
+            _splitkv(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _DT[q.dtype],
+                     (1.0, 1.0, 1.0), num_splits, s)
+            return out, lse
         if h_kv == H:
             rc = _lib.lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_p, B, n_q, n_k, H,
                                    D, scale, int(bool(causal)), int(window_left), _DT[q.dtype], s.cuda_stream)
@@ -88,9 +123,11 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
 def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale: float, k_descale: float,
                 v_descale: float, scale: Optional[float] = None, causal: bool = False,
                 window_left: int = -1, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                return_lse: bool = True, stream: Optional[torch.cuda.Stream] = None):
+                return_lse: bool = True, stream: Optional[torch.cuda.Stream] = None, num_splits: int = 1):
     """FP8 e4m3 forward with per-tensor descales; out is bfloat16."""
     B, n_q, n_k, H, h_kv, D = _check_inputs(q8, k8, v8)
+    if num_splits == 0:
+        num_splits = auto_splits(B, n_q, n_k, H, q8.device)
     if q8.dtype != torch.float8_e4m3fn:
         raise ValueError("forward_fp8 takes float8_e4m3fn tensors")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -98,6 +135,10 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
     with torch.cuda.device(q8.device):
         s = stream if stream is not None else torch.cuda.current_stream(q8.device)
         lse_p = lse.data_ptr() if lse is not None else None
+        if num_splits > 1:
+            _splitkv(q8, k8, v8, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _lib.FA_E4M3,
+                     (q_descale, k_descale, v_descale), num_splits, s)
+            return out, lse
         if h_kv == H:
             rc = _lib.lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(), lse_p, B, n_q,
                                        n_k, H, D, scale, int(bool(causal)), int(window_left), float(q_descale),

@@ -105,7 +105,7 @@ int noalloc_scratch(DeviceState* ds, unsigned** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int D, int DT>
+template <int D, int DT, bool SPLIT>
 int launch(const void* q, const void* k, const void* v, const FwdParams& base, cudaStream_t stream,
            DeviceState* ds, int bit, unsigned* sched_override) {
   using C = Cfg<D, DT>;
@@ -119,14 +119,14 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
       encode_bnhd(&mv, v, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N))
     return FA_ERR_CUDA;
   if (!(ds->attr_set & (1u << bit))) {
-    if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FA_ERR_CUDA;
     // The per-role register split (setmaxnreg) redistributes the registers
     // the CTA was launched with; it is only valid for the launch count it
     // was sized for, so a build that came out with another count is refused.
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, fa_fwd_kernel<D, DT>) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaFuncGetAttributes(&fa, fa_fwd_kernel<D, DT, SPLIT>) != cudaSuccess) return FA_ERR_CUDA;
     if (fa.numRegs != REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
     ds->attr_set |= (1u << bit);
   }
@@ -137,7 +137,7 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     int rc = sched_counters(ds, stream, &p.sched);
     if (rc != FA_OK) return rc;
   }
-  fa_fwd_kernel<D, DT><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  fa_fwd_kernel<D, DT, SPLIT><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -161,13 +161,29 @@ int validate(const void* q, const void* k, const void* v, void* out, int B, int 
   return FA_OK;
 }
 
+// Workspace of a split forward: fp32 O of every slice [splits, B, N_q, H, D]
+// followed by its LSE [splits, B, H, N_q].
+size_t splitkv_workspace_bytes(int B, int Nq, int H, int D, int splits) {
+  return static_cast<size_t>(splits) * B * Nq * H * (static_cast<size_t>(D) + 1) * sizeof(float);
+}
+
 int forward(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Nq, int Nk,
             int H, int Hkv, int D, float scale, int causal, int window_left, int dtype, float qd, float kd,
-            float vd, cudaStream_t stream, unsigned* sched_override = nullptr) {
+            float vd, cudaStream_t stream, unsigned* sched_override = nullptr, int splits = 1,
+            void* workspace = nullptr, size_t workspace_bytes = 0) {
   int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
   if (rc != FA_OK) return rc;
+  if (splits < 1) return FA_ERR_ARG;
   if (!(qd > 0.f) || !std::isfinite(qd) || !(kd > 0.f) || !std::isfinite(kd) || !(vd > 0.f) ||
       !std::isfinite(vd))
+    return FA_ERR_ARG;
+  // key-range slices: at most one per key block, none left empty
+  const int nkb = (Nk + BLOCK_N - 1) / BLOCK_N;
+  const int split_blocks = nkb > 0 ? (nkb + splits - 1) / splits : 1;
+  const int used_splits = nkb > 0 ? (nkb + split_blocks - 1) / split_blocks : 1;
+  if (used_splits > 1 && Nq > 0 &&
+      (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+       workspace_bytes < splitkv_workspace_bytes(B, Nq, H, D, used_splits)))
     return FA_ERR_ARG;
   if (Nq == 0) return FA_OK;
   DeviceState* ds = nullptr;
@@ -196,7 +212,13 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
                                      static_cast<double>(qd) * static_cast<double>(kd));
   p.out_scale = vd;
   p.pairs = (Nq + 2 * BLOCK_M - 1) / (2 * BLOCK_M);
-  const int64_t units = static_cast<int64_t>(p.pairs) * B * H;
+  p.split_blocks = split_blocks;
+  p.splits = used_splits;
+  if (p.splits > 1) {
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = p.o_part + static_cast<size_t>(p.splits) * B * Nq * H * D;
+  }
+  const int64_t units = static_cast<int64_t>(p.pairs) * B * H * p.splits;
   if (units > 0x7fffffff) return FA_ERR_ARG;
   p.num_units = static_cast<int>(units);
   // scheduling groups: causal work runs longest-first across a group of
@@ -216,14 +238,37 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   }
   p.wait_limit_ns = g_wait_limit_ns;
   p.status = ds->status;
-  switch (dtype * 2 + (D == 128 ? 1 : 0)) {
-    case FA_FP16 * 2 + 0: return launch<64, DT_FP16>(q, k, v, p, stream, ds, 0, sched_override);
-    case FA_FP16 * 2 + 1: return launch<128, DT_FP16>(q, k, v, p, stream, ds, 1, sched_override);
-    case FA_BF16 * 2 + 0: return launch<64, DT_BF16>(q, k, v, p, stream, ds, 2, sched_override);
-    case FA_BF16 * 2 + 1: return launch<128, DT_BF16>(q, k, v, p, stream, ds, 3, sched_override);
-    case FA_E4M3 * 2 + 1: return launch<128, DT_E4M3>(q, k, v, p, stream, ds, 4, sched_override);
+  // the split forward is its own instantiation, so the plain one carries no
+  // slice bookkeeping
+  const bool split = p.splits > 1;
+  switch ((dtype * 2 + (D == 128 ? 1 : 0)) * 2 + (split ? 1 : 0)) {
+    case (FA_FP16 * 2 + 0) * 2 + 0: rc = launch<64, DT_FP16, false>(q, k, v, p, stream, ds, 0, sched_override); break;
+    case (FA_FP16 * 2 + 1) * 2 + 0: rc = launch<128, DT_FP16, false>(q, k, v, p, stream, ds, 1, sched_override); break;
+    case (FA_BF16 * 2 + 0) * 2 + 0: rc = launch<64, DT_BF16, false>(q, k, v, p, stream, ds, 2, sched_override); break;
+    case (FA_BF16 * 2 + 1) * 2 + 0: rc = launch<128, DT_BF16, false>(q, k, v, p, stream, ds, 3, sched_override); break;
+    case (FA_E4M3 * 2 + 1) * 2 + 0: rc = launch<128, DT_E4M3, false>(q, k, v, p, stream, ds, 4, sched_override); break;
+    case (FA_FP16 * 2 + 0) * 2 + 1: rc = launch<64, DT_FP16, true>(q, k, v, p, stream, ds, 5, sched_override); break;
+    case (FA_FP16 * 2 + 1) * 2 + 1: rc = launch<128, DT_FP16, true>(q, k, v, p, stream, ds, 6, sched_override); break;
+    case (FA_BF16 * 2 + 0) * 2 + 1: rc = launch<64, DT_BF16, true>(q, k, v, p, stream, ds, 7, sched_override); break;
+    case (FA_BF16 * 2 + 1) * 2 + 1: rc = launch<128, DT_BF16, true>(q, k, v, p, stream, ds, 8, sched_override); break;
+    case (FA_E4M3 * 2 + 1) * 2 + 1: rc = launch<128, DT_E4M3, true>(q, k, v, p, stream, ds, 9, sched_override); break;
     default: return FA_ERR_UNSUPPORTED;
   }
+  if (rc != FA_OK || p.splits == 1) return rc;
+  // combine the slices (same stream, so it runs after the forward)
+  const int64_t rows = static_cast<int64_t>(B) * Nq * H;
+  const int warps_per_block = 8;
+  const int64_t want = (rows + warps_per_block - 1) / warps_per_block;
+  const int blocks = static_cast<int>(want < 8 * 148 ? want : 8 * 148);
+  const bool fp16_out = dtype == FA_FP16;
+  if (D == 64) {
+    if (fp16_out) fa_merge_kernel<64, DT_FP16><<<blocks, 32 * warps_per_block, 0, stream>>>(p.o_part, p.lse_part, out, lse, p.splits, B, Nq, H);
+    else fa_merge_kernel<64, DT_BF16><<<blocks, 32 * warps_per_block, 0, stream>>>(p.o_part, p.lse_part, out, lse, p.splits, B, Nq, H);
+  } else {
+    if (fp16_out) fa_merge_kernel<128, DT_FP16><<<blocks, 32 * warps_per_block, 0, stream>>>(p.o_part, p.lse_part, out, lse, p.splits, B, Nq, H);
+    else fa_merge_kernel<128, DT_BF16><<<blocks, 32 * warps_per_block, 0, stream>>>(p.o_part, p.lse_part, out, lse, p.splits, B, Nq, H);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 size_t elem_bytes(int dtype) { return dtype == FA_E4M3 ? 1 : 2; }
@@ -251,6 +296,25 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* ls
                float k_descale, float v_descale, fa_stream_t stream) {
   return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, q_descale,
                      k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int N_q, int N_k, int H, int D, int num_splits) {
+  if (B < 1 || N_q < 0 || N_k < 0 || H < 1 || D < 1 || num_splits < 1) return 0;
+  // the slices the forward will actually use
+  const int nkb = (N_k + fa::BLOCK_N - 1) / fa::BLOCK_N;
+  if (nkb == 0) return 0;
+  const int per = (nkb + num_splits - 1) / num_splits;
+  const int splits = (nkb + per - 1) / per;
+  return splits > 1 ? fa::splitkv_workspace_bytes(B, N_q, H, D, splits) : 0;
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q, int N_k,
+                   int H, int H_kv, int D, float scale, int causal, int window_left, int dtype, float q_descale,
+                   float k_descale, float v_descale, int num_splits, void* workspace, size_t workspace_bytes,
+                   fa_stream_t stream) {
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, q_descale,
+                     k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream), nullptr, num_splits, workspace,
+                     workspace_bytes);
 }
 
 int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,

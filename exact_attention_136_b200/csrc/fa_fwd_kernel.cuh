@@ -76,6 +76,15 @@ struct FwdParams {
                        // zero between launches (the last CTA resets it)
   unsigned long long wait_limit_ns;
   int* status;         // device status word
+  // split key range (decode-like shapes): every work unit covers key blocks
+  // [s * split_blocks, (s + 1) * split_blocks) of one slice s and writes its
+  // O (normalised by the slice's own row sum) and LSE in fp32 to the
+  // partial buffers; a merge kernel combines the slices.  splits = 1: O and
+  // LSE go straight to out / lse.
+  int splits;
+  int split_blocks;
+  float* o_part;       // [splits, B, N_q, H, D]
+  float* lse_part;     // [splits, B, H, N_q]
 };
 
 constexpr int BLOCK_M = 128;   // query rows per tile
@@ -125,6 +134,7 @@ struct SharedHeader {
   uint64_t mma_done;
   uint64_t uq_full[4], uq_empty[4];   // unit queue: producer -> MMA + softmax warps
   int uq[4];                          // claimed unit ids, -1 = no more work
+  int uq_split[4];                    // ... and their key-range slices
   uint32_t tmem_base;
   int abort_flag;
 #ifdef FA_STATS_BUILD
@@ -138,6 +148,7 @@ struct Tile {
   int b, h, qs;    // batch, head, first query row
   int hk;          // key/value head of this query head
   int lo, hi;      // inclusive key-block range
+  int split;       // key-range slice (0 when not split)
   bool rows;       // tile has rows (qs < N_q)
   bool valid;      // ... and at least one key block
 };
@@ -147,8 +158,10 @@ struct Tile {
 // inside a group causal units run longest first (largest query index), and
 // consecutive units switch head so the CTAs working at the same time share
 // each head's K/V blocks through L2.  Non-causal units use groups of one head.
-__device__ __forceinline__ Tile get_tile(int u, int t, const FwdParams& p) {
+template <bool SPLIT>
+__device__ __forceinline__ Tile get_tile(int u, int split, int t, const FwdParams& p) {
   Tile w;
+  w.split = split;
   const int bh_count = p.B * p.H;
   const int per_group = p.group * p.pairs;
   const int g = u / per_group;
@@ -165,6 +178,10 @@ __device__ __forceinline__ Tile get_tile(int u, int t, const FwdParams& p) {
   const int qe = min(w.qs + BLOCK_M - 1, p.Nq - 1);
   w.lo = p.window_left >= 0 ? max(0, w.qs - p.window_left) / BLOCK_N : 0;
   w.hi = p.causal ? min(qe, p.Nk - 1) / BLOCK_N : (p.Nk - 1) / BLOCK_N;
+  if (SPLIT) {
+    w.lo = max(w.lo, w.split * p.split_blocks);
+    w.hi = min(w.hi, (w.split + 1) * p.split_blocks - 1);
+  }
   w.valid = w.rows && p.Nk > 0 && w.lo <= w.hi;
   return w;
 }
@@ -177,9 +194,10 @@ struct Unit {
   int jlo, jhi;    // empty (jhi < 0) when neither tile has work
 };
 
-__device__ __forceinline__ Unit get_unit(int u, const FwdParams& p) {
-  const Tile a = get_tile(u, 0, p);
-  const Tile c = get_tile(u, 1, p);
+template <bool SPLIT>
+__device__ __forceinline__ Unit get_unit(int u, int split, const FwdParams& p) {
+  const Tile a = get_tile<SPLIT>(u, split, 0, p);
+  const Tile c = get_tile<SPLIT>(u, split, 1, p);
   Unit w;
   w.b = a.b;
   w.h = a.h;
@@ -268,7 +286,7 @@ template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N)); }
 
 // ------------------------------------------------------------------ producer
-template <int D, int DT>
+template <int D, int DT, bool SPLIT>
 __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMap* mq,
                               const CUtensorMap* mk, const CUtensorMap* mv, const FwdParams& p) {
   using C = Cfg<D, DT>;
@@ -292,11 +310,16 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
     if (!mbar_wait(smem_u32(&sh->uq_empty[qs]), (qr & 1u) ^ 1u, p.wait_limit_ns)) {
       record_error(sh, p, ST_TIMEOUT_LOAD); ok = false; break;
     }
-    sh->uq[qs] = cur;
+    // a claimed index enumerates (unit, slice) with the slices of a unit
+    // consecutive; decoded once here for every role
+    const int cu = (cur < 0 || !SPLIT) ? cur : cur / p.splits;
+    const int cs = (cur < 0 || !SPLIT) ? 0 : cur - cu * p.splits;
+    sh->uq[qs] = cu;
+    sh->uq_split[qs] = cs;
     mbar_arrive(smem_u32(&sh->uq_full[qs]));
     ++k;
     if (cur < 0) break;
-    const Unit w = get_unit(cur, p);
+    const Unit w = get_unit<SPLIT>(cu, cs, p);
     int nxt = -2;   // claimed once this unit's first loads are on their way
     if (w.jhi < 0) {
       cur = claim_unit(p);
@@ -342,7 +365,8 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
         // with its Q tiles
         nxt = claim_unit(p);
         if (nxt >= 0) {
-          const Unit wn = get_unit(nxt, p);
+          const int nu = SPLIT ? nxt / p.splits : nxt;
+          const Unit wn = get_unit<SPLIT>(nu, SPLIT ? nxt - nu * p.splits : 0, p);
 #pragma unroll
           for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -456,7 +480,7 @@ __device__ __forceinline__ bool issue_pv_handover(uint32_t p_half_bar, uint32_t 
 // MMA groups delays the tensor pipe: per key block the steady state below
 // issues its 32 MMAs with nothing but the four waits, four commits and the
 // ring advance between them; every decision is taken once per unit.
-template <int D, int DT>
+template <int D, int DT, bool SPLIT>
 __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const FwdParams& p) {
   using C = Cfg<D, DT>;
   constexpr uint32_t SLOT_DESC = C::TILE_BYTES >> 4;   // descriptor start-address step per ring slot
@@ -483,9 +507,10 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
       record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
     }
     const int u = *reinterpret_cast<volatile int*>(&sh->uq[qs]);
+    const int us = SPLIT ? *reinterpret_cast<volatile int*>(&sh->uq_split[qs]) : 0;
     mbar_arrive(smem_u32(&sh->uq_empty[qs]));
     if (u < 0) break;
-    const Unit w = get_unit(u, p);
+    const Unit w = get_unit<SPLIT>(u, us, p);
     if (w.jhi < 0) continue;
     if (aborted(sh)) { ok = false; break; }
     if (!mbar_wait(smem_u32(&sh->q_full), q_uses & 1u, lim)) {
@@ -667,6 +692,14 @@ __device__ __forceinline__ void store_out_row16(void* dst, const float* o, float
   reinterpret_cast<uint4*>(dst)[1] = v1;
 }
 
+// 16 fp32 values times inv -> four 16-byte stores (slice partials)
+__device__ __forceinline__ void store_part_row16(float* dst, const float* o, float inv) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    reinterpret_cast<float4*>(dst)[i] =
+        make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+}
+
 // 2^x on the FMA pipe for a pair of finite x (unmasked blocks only).
 // Range reduction for base 2 is exact: x = j + f with j = round(x) and
 // f in [-1/2, 1/2]; 2^j is added into the exponent field and 2^f is a cubic
@@ -761,7 +794,7 @@ __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_m
 // take score columns [0, 64) of those rows, lanes 16-31 columns [64, 128)
 // (the tcgen05 16x32bx2 access shape), so the two halves of a row meet with
 // one shuffle and apply identical references and rescale factors.
-template <int D, int DT>
+template <int D, int DT, bool SPLIT>
 __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, const int sub, const FwdParams& p) {
   using C = Cfg<D, DT>;
   constexpr int HALF_N = BLOCK_N / 2;
@@ -785,25 +818,39 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     have = __all_sync(0xffffffffu, have);
     if (!have) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
     const int u = *reinterpret_cast<volatile int*>(&sh->uq[qs]);
+    const int us = SPLIT ? *reinterpret_cast<volatile int*>(&sh->uq_split[qs]) : 0;
     __syncwarp();
     if (lane_id() == 0) mbar_arrive(smem_u32(&sh->uq_empty[qs]));
     FA_TRACE(t, 8, 0);
     if (u < 0) break;
-    const Tile w = get_tile(u, t, p);
+    const Tile w = get_tile<SPLIT>(u, us, t, p);
     if (!w.rows) continue;
     const int row = w.qs + r;
     const bool row_ok = row < p.Nq;
+    // this row's O and LSE elements (in the output, or in this key slice's
+    // partials, which hold part_rows() more rows per slice); taken where
+    // they are used, so nothing extra stays live through the block loop
+    auto o_elem = [&]() {
+      return ((static_cast<int64_t>(w.b) * p.Nq + row) * p.H + w.h) * (int64_t)D + half * HALF_D;
+    };
+    auto l_elem = [&]() { return (static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row; };
+    auto part_rows = [&]() { return static_cast<int64_t>(w.split) * p.B * p.Nq * p.H; };
     if (!w.valid) {
-      // no visible key for any row of this tile
+      // no visible key for any row of this tile (in this slice)
       if (row_ok) {
-        uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) +
-                           ((static_cast<int64_t>(w.b) * p.Nq + row) * p.H + w.h) * (int64_t)D * OUT_ES;
         float z[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) z[i] = 0.f;
+        if constexpr (SPLIT) {
 #pragma unroll
-        for (int c = 0; c < HALF_D; c += 16) store_out_row16<DT>(out_row + (half * HALF_D + c) * OUT_ES, z, 0.f);
-        if (p.lse && half == 0) p.lse[(static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row] = -INFINITY;
+          for (int c = 0; c < HALF_D; c += 16) store_part_row16(p.o_part + part_rows() * D + o_elem() + c, z, 0.f);
+          if (half == 0) p.lse_part[part_rows() + l_elem()] = -INFINITY;
+        } else {
+          uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem() * OUT_ES;
+#pragma unroll
+          for (int c = 0; c < HALF_D; c += 16) store_out_row16<DT>(out_row + c * OUT_ES, z, 0.f);
+          if (p.lse && half == 0) p.lse[l_elem()] = -INFINITY;
+        }
       }
       continue;
     }
@@ -913,22 +960,32 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     FA_TRACE(t, 6, 0);
     tc_fence_after();
     const float inv = (lq_row > 0.f ? 1.f / lq_row : 0.f) * p.out_scale;
-    uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) +
-                       ((static_cast<int64_t>(w.b) * p.Nq + row) * p.H + w.h) * (int64_t)D * OUT_ES +
-                       half * HALF_D * OUT_ES;
+    if constexpr (SPLIT) {
+      float* part_row = p.o_part + part_rows() * D + o_elem();
 #pragma unroll
-    for (int c = 0; c < HALF_D; c += 16) {
-      uint32_t o[16];
-      tmem_ld_16x32bx2_x16<HALF_D>(o_addr + c, o);
-      tmem_wait_ld();
-      if (row_ok) store_out_row16<DT>(out_row + c * OUT_ES, reinterpret_cast<float*>(o), inv);
+      for (int c = 0; c < HALF_D; c += 16) {
+        uint32_t o[16];
+        tmem_ld_16x32bx2_x16<HALF_D>(o_addr + c, o);
+        tmem_wait_ld();
+        if (row_ok) store_part_row16(part_row + c, reinterpret_cast<float*>(o), inv);
+      }
+    } else {
+      uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem() * OUT_ES;
+#pragma unroll
+      for (int c = 0; c < HALF_D; c += 16) {
+        uint32_t o[16];
+        tmem_ld_16x32bx2_x16<HALF_D>(o_addr + c, o);
+        tmem_wait_ld();
+        if (row_ok) store_out_row16<DT>(out_row + c * OUT_ES, reinterpret_cast<float*>(o), inv);
+      }
     }
     tc_fence_before();
     mbar_arrive(smem_u32(&sh->o_empty[t]));
-    if (row_ok && p.lse && half == 0) {
+    if (row_ok && half == 0) {
       // natural log of sum_j exp(scale * s_j) = (m_used + log2(l) - PSHIFT) * ln 2
-      p.lse[(static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row] =
-          l_row > 0.f ? (m_used + __log2f(l_row) - C::PSHIFT) * 0.69314718055994531f : -INFINITY;
+      const float lse_v = l_row > 0.f ? (m_used + __log2f(l_row) - C::PSHIFT) * 0.69314718055994531f : -INFINITY;
+      if constexpr (SPLIT) p.lse_part[part_rows() + l_elem()] = lse_v;
+      else if (p.lse) p.lse[l_elem()] = lse_v;
     }
     FA_TRACE(t, 7, 0);
   }
@@ -936,7 +993,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, int DT>
+template <int D, int DT, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -990,15 +1047,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp < 4) {
     setmaxnreg_dec<REGS_LOAD_MMA>();
-    if (warp == 0 && lane_id() == 0) producer_role<D, DT>(sh, tiles, &tm_q, &tm_k, &tm_v, p);
-    else if (warp == 1 && lane_id() == 0) mma_role<D, DT>(sh, tiles, tbase, p);
+    if (warp == 0 && lane_id() == 0) producer_role<D, DT, SPLIT>(sh, tiles, &tm_q, &tm_k, &tm_v, p);
+    else if (warp == 1 && lane_id() == 0) mma_role<D, DT, SPLIT>(sh, tiles, tbase, p);
   } else {
     setmaxnreg_inc<REGS_SOFTMAX>();
     // warps 4-11: tile 0, warps 12-19: tile 1; within a tile the first four
     // warps take the upper 16 rows of each lane quadrant, the next four the lower
     const int t = warp < 12 ? 0 : 1;
     const int sub = ((warp - 4) >> 2) & 1;
-    softmax_role<D, DT>(sh, tbase, t, sub, p);
+    softmax_role<D, DT, SPLIT>(sh, tbase, t, sub, p);
   }
   tc_fence_before();
   __syncthreads();
@@ -1020,6 +1077,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       atomicExch(p.sched + 1, 0u);
       __threadfence();
     }
+  }
+}
+
+// Combines the key-range slices of a split forward.  One warp per output
+// row (b, n, h): with slice LSEs L_s and slice outputs O_s (each normalised
+// by its own row sum), LSE = log sum_s exp(L_s) and O = sum_s exp(L_s - LSE)
+// O_s; a row no slice sees gets O = 0, LSE = -inf.
+template <int D, int OUT_DT>
+__global__ void fa_merge_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, void* out,
+                                float* lse, int splits, int B, int Nq, int H) {
+  constexpr int PER_LANE = D / 32;
+  const int64_t rows = static_cast<int64_t>(B) * Nq * H;
+  const int lane = static_cast<int>(threadIdx.x & 31u);
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x / 32) + threadIdx.x / 32; i < rows; i += warps) {
+    // i enumerates (b, n, h) like O; the LSE layout is [B, H, N_q]
+    const int64_t h = i % H;
+    const int64_t bn = i / H;
+    const int64_t n = bn % Nq;
+    const int64_t b = bn / Nq;
+    const int64_t l_idx = (b * H + h) * Nq + n;
+    float m = -INFINITY;
+    for (int s = 0; s < splits; ++s) m = fmaxf(m, lse_part[static_cast<int64_t>(s) * rows + l_idx]);
+    float acc[PER_LANE];
+#pragma unroll
+    for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
+    float wsum = 0.f;
+    if (m != -INFINITY) {
+      for (int s = 0; s < splits; ++s) {
+        const float ls = lse_part[static_cast<int64_t>(s) * rows + l_idx];
+        if (ls == -INFINITY) continue;
+        const float wgt = expf(ls - m);
+        wsum += wgt;
+        const float* src = o_part + (static_cast<int64_t>(s) * rows + i) * D + lane * PER_LANE;
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) acc[e] = fmaf(wgt, src[e], acc[e]);
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    float o[PER_LANE];
+#pragma unroll
+    for (int e = 0; e < PER_LANE; ++e) o[e] = acc[e] * inv;
+    uint32_t packed[PER_LANE / 2];
+#pragma unroll
+    for (int e = 0; e < PER_LANE / 2; ++e) packed[e] = pack2<OUT_DT>(o[2 * e], o[2 * e + 1]);
+    uint8_t* dst = reinterpret_cast<uint8_t*>(out) + (i * D + lane * PER_LANE) * 2;
+    if constexpr (PER_LANE == 4) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = packed[0];
+    }
+    if (lse && lane == 0) lse[l_idx] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
   }
 }
 

@@ -32,6 +32,7 @@ class Workload:
     index: int          # seed offset: seeds are 1001/1002/1003 + 100 * index
     desc: str
     kv_heads: int = 0   # K/V heads (0 = H); fewer for multi-/grouped-query attention
+    splits: int = 1     # key-range slices (fa_fwd_splitkv) for few query rows against many keys
 
     @property
     def h_kv(self):
@@ -68,6 +69,11 @@ WORKLOADS = {
         "gqa_causal_b4h32kv8n8192d128_bf16", 4, 8192, 8192, 32, 128, "bf16", True, -1,
         1.0 / math.sqrt(128.0), 6,
         "grouped-query causal B4 H32 (8 K/V heads) N8192 D128 bf16, scale 1/sqrt(128)", 8),
+    "splitkv_b1h32kv8q128k65536d128_bf16": Workload(
+        "splitkv_b1h32kv8q128k65536d128_bf16", 1, 128, 65536, 32, 128, "bf16", False, -1,
+        1.0 / math.sqrt(128.0), 7,
+        "128 query rows against 65536 keys (decode-like: 32 work units for 148 SMs unsplit), "
+        "B1 H32 (8 K/V heads) D128 bf16, key range in 4 slices", 8, 4),
 }
 
 # order used by tests; the headline bench workload is the causal bf16 D128 case

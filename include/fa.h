@@ -40,6 +40,8 @@
 #ifndef FA_B200_H
 #define FA_B200_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -101,6 +103,33 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* ls
                int B, int N_q, int N_k, int H, int H_kv, int D, float scale, int causal,
                int window_left, int dtype, float q_descale, float k_descale, float v_descale,
                fa_stream_t stream);
+
+/*
+ * fa_fwd_splitkv -- the forward of fa_fwd_gqa with the key range split into
+ * up to num_splits slices that run as separate work units, for shapes with
+ * few query tiles and many keys (decode-like N_q << N_k), which would
+ * otherwise occupy only B * H * ceil(N_q / 256) of the GPU's SMs.  Every
+ * slice computes the same online softmax over its keys and writes its O
+ * (normalised by the slice's own row sum) and LSE in fp32 to `workspace`;
+ * a second kernel on the same stream combines them:
+ *   LSE = log sum_s exp(LSE_s),  O = sum_s exp(LSE_s - LSE) * O_s
+ * which is the same softmax over all keys (the explainer page's online
+ * softmax rescaling, FlashAttention, aiunderstanding.org, "Technical
+ * insight", applied across slices instead of across blocks).
+ *   num_splits >= 1; the slices used are min(num_splits, key blocks of 128)
+ *   rounded so none is empty; 1 is the plain forward (workspace unused).
+ *   workspace: caller-owned device memory of at least
+ *   fa_fwd_splitkv_workspace_bytes(...) bytes, 256-byte aligned (NULL
+ *   allowed when that size is 0).  The library allocates nothing.
+ * Other arguments and return values as fa_fwd_gqa; FA_ERR_ARG also for
+ * num_splits < 1 or a missing / short / misaligned workspace.
+ */
+size_t fa_fwd_splitkv_workspace_bytes(int B, int N_q, int N_k, int H, int D, int num_splits);
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* out, float* lse,
+                   int B, int N_q, int N_k, int H, int H_kv, int D, float scale, int causal,
+                   int window_left, int dtype, float q_descale, float k_descale,
+                   float v_descale, int num_splits, void* workspace, size_t workspace_bytes,
+                   fa_stream_t stream);
 
 /*
  * fa_fwd_host -- the same forward on HOST buffers: copies q, k, v from host

@@ -114,3 +114,26 @@ def test_gqa_descales_validated():
     f = _lib.lib().fa_fwd_gqa
     assert f(A, A, A, A, None, 1, 128, 128, 8, 2, 128, 0.1, 0, -1, _lib.FA_E4M3, 1.0, 0.0, 1.0,
              None) == _lib.FA_ERR_ARG
+
+
+def test_splitkv_workspace_size():
+    f = _lib.lib().fa_fwd_splitkv_workspace_bytes
+    # one slice (or one key block): no workspace
+    assert f(1, 16, 1024, 4, 128, 1) == 0
+    assert f(1, 16, 100, 4, 128, 8) == 0
+    # 8 key blocks in 4 slices of 2: 4 * B * N_q * H * (D + 1) floats
+    assert f(2, 16, 1024, 4, 128, 4) == 4 * 2 * 16 * 4 * 129 * 4
+    # more slices than key blocks: one slice per block
+    assert f(1, 3, 1024, 2, 64, 100) == 8 * 1 * 3 * 2 * 65 * 4
+    # 10 blocks in "4" slices of 3 -> 4 slices; in "6" slices of 2 -> 5 slices
+    assert f(1, 1, 1280, 1, 64, 4) == 4 * 65 * 4
+    assert f(1, 1, 1280, 1, 64, 6) == 5 * 65 * 4
+    assert f(0, 1, 1280, 1, 64, 6) == 0 and f(1, 1, 1280, 1, 64, 0) == 0
+
+
+@pytest.mark.parametrize("splits, ws, nbytes", [(0, A, 1 << 30), (4, None, 1 << 30), (4, A, 16), (4, A + 16, 1 << 30)])
+def test_splitkv_arguments_validated(splits, ws, nbytes):
+    """Slice count and workspace are checked on the host, before any GPU work."""
+    f = _lib.lib().fa_fwd_splitkv
+    assert f(A, A, A, A, None, 1, 16, 1024, 4, 4, 128, 0.1, 0, -1, _lib.FA_BF16, 1.0, 1.0, 1.0, splits, ws, nbytes,
+             None) == _lib.FA_ERR_ARG

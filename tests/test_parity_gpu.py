@@ -30,14 +30,14 @@ def _need_gpu():
     _lib.lib()  # fails loudly when the library is missing
 
 
-def run(qkv, scale, causal, wl, want_lse=True, stream=None):
+def run(qkv, scale, causal, wl, want_lse=True, stream=None, num_splits=1):
     dev = torch.device("cuda", 0)
     q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
     if q.dtype == torch.float8_e4m3fn:
         out, lse = forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, scale, causal, wl,
-                               return_lse=want_lse, stream=stream)
+                               return_lse=want_lse, stream=stream, num_splits=num_splits)
     else:
-        out, lse = forward(q, k, v, scale, causal, wl, return_lse=want_lse, stream=stream)
+        out, lse = forward(q, k, v, scale, causal, wl, return_lse=want_lse, stream=stream, num_splits=num_splits)
     torch.cuda.synchronize()
     rc, flags = device_status()
     assert rc == 0, f"device status {rc} flags {flags}"
@@ -131,6 +131,67 @@ def test_gqa_with_all_heads_equals_mha_entry():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+# split key range: (B, N_q, N_k, H, H_kv, D, dtype, causal, window_left, num_splits)
+SPLIT = [
+    (2, 1, 4096, 8, 2, 128, "bf16", False, -1, 8),      # decode-like: one query row
+    (1, 16, 3000, 4, 4, 64, "fp16", False, -1, 5),      # ragged last key block
+    (1, 1000, 1000, 2, 2, 128, "bf16", True, -1, 3),    # causal: later slices empty for early rows
+    (1, 2000, 2000, 2, 1, 128, "fp16", True, 300, 4),   # window: most slices empty for each row
+    (1, 64, 5000, 4, 2, 128, "e4m3", False, -1, 6),
+    (1, 200, 700, 2, 2, 64, "bf16", False, -1, 100),    # more slices than key blocks
+    (1, 300, 40, 2, 2, 64, "fp16", True, 10, 4),        # one key block: no split, rows with no key
+]
+
+
+@pytest.mark.parametrize("case", SPLIT, ids=[
+    f"B{c[0]}_q{c[1]}_k{c[2]}_H{c[3]}_Hkv{c[4]}_D{c[5]}_{c[6]}_{'c' if c[7] else 'nc'}_w{c[8]}_s{c[9]}"
+    for c in SPLIT])
+def test_splitkv_parity(case):
+    B, nq, nk, H, h_kv, D, dt, causal, wl, ns = case
+    qkv = inputs.make_qkv(B, nq, nk, H, D, dt, seeds=(61 + nq, 62 + nk, 63 + ns), h_kv=h_kv)
+    dev = torch.device("cuda", 0)
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    scale = 1.0 / math.sqrt(D)
+    if dt == "e4m3":
+        out, lse = forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, scale, causal, wl,
+                               num_splits=ns)
+    else:
+        out, lse = forward(q, k, v, scale, causal, wl, num_splits=ns)
+    torch.cuda.synchronize()
+    rc, flags = device_status()
+    assert rc == 0, f"device status {rc} flags {flags}"
+    ref_o, ref_l = oracle(qkv, scale, causal, wl)
+    d_o, d_l = compare(out, lse, ref_o, ref_l)
+    assert d_o <= TOL_O[dt], f"max|dO| {d_o:.3e} > {TOL_O[dt]}"
+    assert d_l <= TOL_LSE, f"max|dLSE| {d_l:.3e} > {TOL_LSE}"
+
+
+def test_splitkv_auto_slices():
+    """num_splits = 0 picks the slices from the SM count; the result still matches the oracle."""
+    from exact_attention_136_b200 import auto_splits
+    assert auto_splits(1, 100, 4096, 2) > 1                 # 2 units, 148 SMs
+    assert auto_splits(4, 8192, 8192, 32) == 1              # thousands of units
+    assert auto_splits(1, 100, 256, 2) == 2                 # capped at the key blocks
+    qkv = inputs.make_qkv(1, 100, 4096, 2, 128, "bf16", seeds=(81, 82, 83))
+    dev = torch.device("cuda", 0)
+    out, lse = forward(qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev), 0.1, False, -1, num_splits=0)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle(qkv, 0.1, False, -1)
+    d_o, d_l = compare(out, lse, ref_o, ref_l)
+    assert d_o <= TOL_O["bf16"] and d_l <= TOL_LSE, (d_o, d_l)
+
+
+def test_splitkv_one_slice_is_the_plain_forward():
+    """num_splits = 1 takes the plain path: bit-identical to forward()."""
+    qkv = inputs.make_qkv(1, 300, 900, 4, 128, "bf16", seeds=(71, 72, 73))
+    dev = torch.device("cuda", 0)
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    o1, l1 = forward(q, k, v, 0.1, False, -1)
+    o2, l2 = forward(q, k, v, 0.1, False, -1, num_splits=1)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 @pytest.mark.parametrize("dt,D", [("fp16", 64), ("bf16", 128), ("e4m3", 128)])
 @pytest.mark.parametrize("mult", [4.0, 12.0])
 def test_large_scores_exercise_rescaling(dt, D, mult):
@@ -172,7 +233,7 @@ def test_full_workload_sampled_rows(name):
     w = W.WORKLOADS[name]
     qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=w.seeds, h_kv=w.h_kv)
     rows = W.sample_rows(w, count=64 if w.n_q > 4096 else 256)
-    out, lse = run(qkv, w.scale, w.causal, w.window_left)
+    out, lse = run(qkv, w.scale, w.causal, w.window_left, num_splits=w.splits)
     assert bool(torch.isfinite(out).all()) and bool(torch.isfinite(lse).all())
     ref_o, ref_l = oracle(qkv, w.scale, w.causal, w.window_left, rows=rows)
     d_o, d_l = compare(out, lse, ref_o, ref_l, rows=rows)

@@ -262,13 +262,16 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     splits = w.splits if args.splits is None else args.splits
+    mask_cpu = W.make_mask(w)
+    mask = mask_cpu.to(dev) if mask_cpu is not None else None
 
     def step():
         if w.dtype == "e4m3":
             forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, w.scale, w.causal, w.window_left,
-                        out=out, lse=lse, stream=stream, num_splits=splits)
+                        out=out, lse=lse, stream=stream, num_splits=splits, attn_mask=mask)
         else:
-            forward(q, k, v, w.scale, w.causal, w.window_left, out=out, lse=lse, stream=stream, num_splits=splits)
+            forward(q, k, v, w.scale, w.causal, w.window_left, out=out, lse=lse, stream=stream, num_splits=splits,
+                    attn_mask=mask)
 
     def barrier():
         if world > 1:
@@ -314,7 +317,7 @@ def main():
     desc = (qkv.q_descale, qkv.k_descale, qkv.v_descale)
 
     def e2e_step():
-        if w.h_kv == w.H and splits == 1:
+        if w.h_kv == w.H and splits == 1 and mask is None:
             forward_host(hq, hk, hv, staging, w.scale, w.causal, w.window_left, desc, ho, hl, stream)
         else:
             # fa_fwd_host takes H K/V heads; grouped heads go through pinned
@@ -365,7 +368,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "desc": w.desc, "B": w.B, "N_q": w.n_q, "N_k": w.n_k, "H": w.H,
-                   "H_kv": w.h_kv, "splits": splits, "D": w.D, "causal": w.causal, "window_left": w.window_left, "scale": w.scale,
+                   "H_kv": w.h_kv, "splits": splits, "mask": w.mask or None, "D": w.D, "causal": w.causal, "window_left": w.window_left, "scale": w.scale,
                    "flop_per_step": flops,
                    "block_fraction": W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left),
                    "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB vs {L2_BYTES / 1e6:.0f} MB), no flush",
@@ -374,7 +377,7 @@ def main():
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps,
-                "api": "fa_fwd_host (pinned host buffers)" if (w.h_kv == w.H and splits == 1)
+                "api": "fa_fwd_host (pinned host buffers)" if (w.h_kv == w.H and splits == 1 and mask is None)
                        else "pinned host copies + forward"},
         "roofline": {"bound": "tensor", "achieved": per_launch_tflops, "peak": peak, "unit": UNIT,
                      "frac": per_launch_tflops / peak, "traffic": traffic,

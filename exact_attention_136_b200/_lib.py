@@ -19,6 +19,7 @@ FA_ERR_CUDA = -4
 FA_ERR_TIMEOUT = -5
 
 FA_FP16, FA_BF16, FA_E4M3 = 0, 1, 2
+FA_MASK_BOOL, FA_MASK_ADD = 1, 2
 
 _c_int, _c_float, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
 _fp = ctypes.POINTER(ctypes.c_float)
@@ -34,6 +35,9 @@ SIGNATURES = {
     "fa_fwd_splitkv": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                                 _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _c_int, _vp, ctypes.c_size_t,
                                 _vp]),
+    "fa_fwd_mask": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                             _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp, _c_int,
+                             ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, _vp]),
     "fa_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                              _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, _c_float,
                              _c_float, _vp]),

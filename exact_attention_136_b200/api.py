@@ -54,6 +54,38 @@ def _outputs(q, B, n_q, H, D, out, lse, want_lse):
     return out, lse
 
 
+def _mask_args(attn_mask: torch.Tensor, q: torch.Tensor, B: int, H: int, n_q: int, n_k: int):
+    """attn_mask ([N_q, N_k] or [B or 1, H or 1, N_q, N_k]; bool = attend where True, float = added to
+    the scaled scores) as the library takes it: bytes or the output's 16-bit type, rows padded to
+    16 bytes, broadcast dimensions with stride 0.  Returns (buffer, kind, stride_b, stride_h, stride_q)."""
+    m = attn_mask
+    if m.dim() == 2:
+        m = m[None, None]
+    if (m.dim() != 4 or m.shape[2] != n_q or m.shape[3] != n_k or m.shape[0] not in (1, B)
+            or m.shape[1] not in (1, H)):
+        raise ValueError("attn_mask must be [N_q, N_k] or [B or 1, H or 1, N_q, N_k]")
+    if m.dtype == torch.bool:
+        kind, dt = _lib.FA_MASK_BOOL, torch.uint8
+    else:
+        kind, dt = _lib.FA_MASK_ADD, (torch.float16 if q.dtype == torch.float16 else torch.bfloat16)
+    per = 16 // torch.empty((), dtype=dt).element_size()
+    n_pad = -(-n_k // per) * per
+    buf = torch.zeros((m.shape[0], m.shape[1], n_q, n_pad), dtype=dt, device=q.device)
+    buf[..., :n_k] = m.to(device=q.device, dtype=dt)
+    sb = buf.stride(0) if m.shape[0] > 1 else 0
+    sh = buf.stride(1) if m.shape[1] > 1 else 0
+    return buf, kind, sb, sh, buf.stride(2)
+
+
+def _masked(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, dt, descales, attn_mask, s):
+    buf, kind, sb, sh, sq = _mask_args(attn_mask, q, B, H, n_q, n_k)
+    rc = _lib.lib().fa_fwd_mask(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, h_kv, D, scale,
+                                int(bool(causal)), int(window_left), dt, float(descales[0]), float(descales[1]),
+                                float(descales[2]), buf.data_ptr(), kind, sb, sh, sq, s.cuda_stream)
+    _lib.check(rc, "fa_fwd_mask")
+
+
 def auto_splits(B: int, n_q: int, n_k: int, H: int, device=None) -> int:
     """Key-range slices that fill the GPU: one per SM for every work unit
     (256 query rows of one (batch, head)) short of the SM count, at most one
@@ -82,8 +114,8 @@ def _splitkv(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_l
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
             causal: bool = False, window_left: int = -1, out: Optional[torch.Tensor] = None,
             lse: Optional[torch.Tensor] = None, return_lse: bool = True,
-            stream: Optional[torch.cuda.Stream] = None,
-            num_splits: int = 1) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            stream: Optional[torch.cuda.Stream] = None, num_splits: int = 1,
+            attn_mask: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Exact attention forward; returns (out, lse).
 
     scale=None means 1/sqrt(headdim), the pages' auto scale (Workflow 2,
@@ -93,18 +125,27 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
     2, Step 3): query head h then reads head h // (H / H_kv).  num_splits > 1
     splits the key range into that many slices run in parallel and merged
     (for few query rows against many keys); 0 picks it with auto_splits.
+    attn_mask: the pages' SDPA mask (Workflow 1, Step 2) -- bool (attend where
+    True) or float (added to the scaled scores), [N_q, N_k] or
+    [B or 1, H or 1, N_q, N_k]; not combined with num_splits.
     """
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
     if num_splits == 0:
         num_splits = auto_splits(B, n_q, n_k, H, q.device)
     if q.dtype == torch.float8_e4m3fn:
         return forward_fp8(q, k, v, 1.0, 1.0, 1.0, scale, causal, window_left, out, lse, return_lse, stream,
-                           num_splits)
+                           num_splits, attn_mask)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     out, lse = _outputs(q, B, n_q, H, D, out, lse, return_lse)
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
         lse_p = lse.data_ptr() if lse is not None else None
+        if attn_mask is not None:
+            if num_splits > 1:
+                raise ValueError("attn_mask is not combined with num_splits")
+            _masked(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _DT[q.dtype],
+                    (1.0, 1.0, 1.0), attn_mask, s)
+            return out, lse
         if num_splits > 1:
             _splitkv(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _DT[q.dtype],
                      (1.0, 1.0, 1.0), num_splits, s)
@@ -123,7 +164,8 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
 def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale: float, k_descale: float,
                 v_descale: float, scale: Optional[float] = None, causal: bool = False,
                 window_left: int = -1, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                return_lse: bool = True, stream: Optional[torch.cuda.Stream] = None, num_splits: int = 1):
+                return_lse: bool = True, stream: Optional[torch.cuda.Stream] = None, num_splits: int = 1,
+                attn_mask: Optional[torch.Tensor] = None):
     """FP8 e4m3 forward with per-tensor descales; out is bfloat16."""
     B, n_q, n_k, H, h_kv, D = _check_inputs(q8, k8, v8)
     if num_splits == 0:
@@ -135,6 +177,12 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
     with torch.cuda.device(q8.device):
         s = stream if stream is not None else torch.cuda.current_stream(q8.device)
         lse_p = lse.data_ptr() if lse is not None else None
+        if attn_mask is not None:
+            if num_splits > 1:
+                raise ValueError("attn_mask is not combined with num_splits")
+            _masked(q8, k8, v8, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _lib.FA_E4M3,
+                    (q_descale, k_descale, v_descale), attn_mask, s)
+            return out, lse
         if num_splits > 1:
             _splitkv(q8, k8, v8, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _lib.FA_E4M3,
                      (q_descale, k_descale, v_descale), num_splits, s)

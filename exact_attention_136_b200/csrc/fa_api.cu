@@ -105,7 +105,7 @@ int noalloc_scratch(DeviceState* ds, unsigned** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int D, int DT, bool SPLIT>
+template <int D, int DT, bool SPLIT, int MASK = MASK_NONE>
 int launch(const void* q, const void* k, const void* v, const FwdParams& base, cudaStream_t stream,
            DeviceState* ds, int bit, unsigned* sched_override) {
   using C = Cfg<D, DT>;
@@ -119,14 +119,14 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
       encode_bnhd(&mv, v, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N))
     return FA_ERR_CUDA;
   if (!(ds->attr_set & (1u << bit))) {
-    if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT, SPLIT, MASK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FA_ERR_CUDA;
     // The per-role register split (setmaxnreg) redistributes the registers
     // the CTA was launched with; it is only valid for the launch count it
     // was sized for, so a build that came out with another count is refused.
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, fa_fwd_kernel<D, DT, SPLIT>) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaFuncGetAttributes(&fa, fa_fwd_kernel<D, DT, SPLIT, MASK>) != cudaSuccess) return FA_ERR_CUDA;
     if (fa.numRegs != REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
     ds->attr_set |= (1u << bit);
   }
@@ -137,7 +137,7 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     int rc = sched_counters(ds, stream, &p.sched);
     if (rc != FA_OK) return rc;
   }
-  fa_fwd_kernel<D, DT, SPLIT><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  fa_fwd_kernel<D, DT, SPLIT, MASK><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -170,10 +170,20 @@ size_t splitkv_workspace_bytes(int B, int Nq, int H, int D, int splits) {
 int forward(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Nq, int Nk,
             int H, int Hkv, int D, float scale, int causal, int window_left, int dtype, float qd, float kd,
             float vd, cudaStream_t stream, unsigned* sched_override = nullptr, int splits = 1,
-            void* workspace = nullptr, size_t workspace_bytes = 0) {
+            void* workspace = nullptr, size_t workspace_bytes = 0, const void* mask = nullptr,
+            int mask_type = 0, long long mask_sb = 0, long long mask_sh = 0, long long mask_sq = 0) {
   int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
   if (rc != FA_OK) return rc;
   if (splits < 1) return FA_ERR_ARG;
+  if (mask_type != 0) {
+    // byte (boolean) or 16-bit (additive) elements; every row of the mask
+    // starts on a 16-byte boundary and holds N_k elements
+    const long long mes = mask_type == FA_MASK_BOOL ? 1 : 2;
+    if ((mask_type != FA_MASK_BOOL && mask_type != FA_MASK_ADD) || !mask || splits != 1 ||
+        !aligned16(mask) || mask_sb < 0 || mask_sh < 0 || mask_sq < Nk || (mask_sb * mes) % 16 != 0 ||
+        (mask_sh * mes) % 16 != 0 || (mask_sq * mes) % 16 != 0)
+      return FA_ERR_ARG;
+  }
   if (!(qd > 0.f) || !std::isfinite(qd) || !(kd > 0.f) || !std::isfinite(kd) || !(vd > 0.f) ||
       !std::isfinite(vd))
     return FA_ERR_ARG;
@@ -238,6 +248,28 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   }
   p.wait_limit_ns = g_wait_limit_ns;
   p.status = ds->status;
+  p.mask = mask;
+  p.mask_sb = mask_sb;
+  p.mask_sh = mask_sh;
+  p.mask_sq = mask_sq;
+  p.mask_scale = static_cast<float>(1.0 / (static_cast<double>(scale) * qd * kd));
+  if (mask_type != 0) {
+    // masked forwards: every key block in the causal / window range is
+    // computed (the mask decides inside the blocks)
+    switch ((dtype * 2 + (D == 128 ? 1 : 0)) * 2 + (mask_type == FA_MASK_ADD ? 1 : 0)) {
+      case (FA_FP16 * 2 + 0) * 2 + 0: return launch<64, DT_FP16, false, MASK_BOOL>(q, k, v, p, stream, ds, 10, sched_override);
+      case (FA_FP16 * 2 + 1) * 2 + 0: return launch<128, DT_FP16, false, MASK_BOOL>(q, k, v, p, stream, ds, 11, sched_override);
+      case (FA_BF16 * 2 + 0) * 2 + 0: return launch<64, DT_BF16, false, MASK_BOOL>(q, k, v, p, stream, ds, 12, sched_override);
+      case (FA_BF16 * 2 + 1) * 2 + 0: return launch<128, DT_BF16, false, MASK_BOOL>(q, k, v, p, stream, ds, 13, sched_override);
+      case (FA_E4M3 * 2 + 1) * 2 + 0: return launch<128, DT_E4M3, false, MASK_BOOL>(q, k, v, p, stream, ds, 14, sched_override);
+      case (FA_FP16 * 2 + 0) * 2 + 1: return launch<64, DT_FP16, false, MASK_ADD>(q, k, v, p, stream, ds, 15, sched_override);
+      case (FA_FP16 * 2 + 1) * 2 + 1: return launch<128, DT_FP16, false, MASK_ADD>(q, k, v, p, stream, ds, 16, sched_override);
+      case (FA_BF16 * 2 + 0) * 2 + 1: return launch<64, DT_BF16, false, MASK_ADD>(q, k, v, p, stream, ds, 17, sched_override);
+      case (FA_BF16 * 2 + 1) * 2 + 1: return launch<128, DT_BF16, false, MASK_ADD>(q, k, v, p, stream, ds, 18, sched_override);
+      case (FA_E4M3 * 2 + 1) * 2 + 1: return launch<128, DT_E4M3, false, MASK_ADD>(q, k, v, p, stream, ds, 19, sched_override);
+      default: return FA_ERR_UNSUPPORTED;
+    }
+  }
   // the split forward is its own instantiation, so the plain one carries no
   // slice bookkeeping
   const bool split = p.splits > 1;
@@ -315,6 +347,16 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* out, float
   return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, q_descale,
                      k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream), nullptr, num_splits, workspace,
                      workspace_bytes);
+}
+
+int fa_fwd_mask(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q, int N_k,
+                int H, int H_kv, int D, float scale, int causal, int window_left, int dtype, float q_descale,
+                float k_descale, float v_descale, const void* mask, int mask_type, long long mask_stride_b,
+                long long mask_stride_h, long long mask_stride_q, fa_stream_t stream) {
+  if (mask_type != FA_MASK_BOOL && mask_type != FA_MASK_ADD) return FA_ERR_ARG;
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, q_descale,
+                     k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream), nullptr, 1, nullptr, 0, mask,
+                     mask_type, mask_stride_b, mask_stride_h, mask_stride_q);
 }
 
 int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,

@@ -50,6 +50,9 @@ namespace fa {
 
 enum : int { DT_FP16 = 0, DT_BF16 = 1, DT_E4M3 = 2 };
 
+// attention-mask kinds of the masked kernel instantiations
+enum : int { MASK_NONE = 0, MASK_BOOL = 1, MASK_ADD = 2 };
+
 // device status word: bit flags of the role whose wait timed out
 enum : int {
   ST_TIMEOUT_LOAD = 1,
@@ -85,6 +88,13 @@ struct FwdParams {
   int split_blocks;
   float* o_part;       // [splits, B, N_q, H, D]
   float* lse_part;     // [splits, B, H, N_q]
+  // attention mask (masked kernels): element (b, h, i, j) at
+  // mask + b * mask_sb + h * mask_sh + i * mask_sq + j; boolean masks are
+  // bytes (0 = masked out), additive ones 16-bit floats added to the scaled
+  // score, applied to the raw score as mask * mask_scale
+  const void* mask;
+  long long mask_sb, mask_sh, mask_sq;
+  float mask_scale;    // 1 / (scale * q_descale * k_descale)
 };
 
 constexpr int BLOCK_M = 128;   // query rows per tile
@@ -794,7 +804,7 @@ __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_m
 // take score columns [0, 64) of those rows, lanes 16-31 columns [64, 128)
 // (the tcgen05 16x32bx2 access shape), so the two halves of a row meet with
 // one shuffle and apply identical references and rescale factors.
-template <int D, int DT, bool SPLIT>
+template <int D, int DT, bool SPLIT, int MASK>
 __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, const int sub, const FwdParams& p) {
   using C = Cfg<D, DT>;
   constexpr int HALF_N = BLOCK_N / 2;
@@ -858,12 +868,35 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     float m_used = -INFINITY;   // reference max (log2 units) that P and l are taken against
     float l = 0.f;              // this thread's share of the row sum (exact)
     float lq = 0.f;             // ... of the stored P values (differs for e4m3)
+    // this thread's mask row (its 64 keys of each block start at key
+    // k0 + 64 * half); rows past N_q read nothing
+    constexpr int MES = MASK == MASK_BOOL ? 1 : 2;   // mask element bytes
+    const uint8_t* mask_row = nullptr;
+    if constexpr (MASK != MASK_NONE) {
+      if (row_ok)
+        mask_row = static_cast<const uint8_t*>(p.mask) +
+                   (static_cast<int64_t>(w.b) * p.mask_sb + static_cast<int64_t>(w.h) * p.mask_sh +
+                    static_cast<int64_t>(row) * p.mask_sq + half * HALF_N) * MES;
+    }
     for (int j = w.lo; j <= w.hi; ++j) {
       // boundary blocks (causal diagonal, window edge, key tail), decided
       // before S arrives
       const int k0 = j * BLOCK_N;
       const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
                              (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
+      // the mask values of this block, loaded while S is computed (16-byte
+      // chunks that start at or past N_k are not read)
+      constexpr int MCHUNKS = MASK == MASK_NONE ? 1 : HALF_N * MES / 16;
+      uint4 mk[MCHUNKS];
+      if constexpr (MASK != MASK_NONE) {
+#pragma unroll
+        for (int c = 0; c < MCHUNKS; ++c) {
+          const int key = k0 + half * HALF_N + c * (16 / MES);
+          mk[c] = (mask_row && key < p.Nk)
+                      ? __ldg(reinterpret_cast<const uint4*>(mask_row + static_cast<int64_t>(k0) * MES) + c)
+                      : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       bool got = mbar_wait(smem_u32(&sh->s_full[t]), s_waits & 1u, p.wait_limit_ns);
       got = __all_sync(0xffffffffu, got);
       if (!got) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
@@ -875,6 +908,28 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       tmem_ld_16x32bx2_x32<64>(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
       tmem_wait_ld();
       FA_TRACE(t, 2, j);
+      if constexpr (MASK == MASK_BOOL) {
+        // byte c of the thread's 64: key k0 + 64 * half + c; 0 = masked out
+#pragma unroll
+        for (int c = 0; c < HALF_N; ++c) {
+          const uint32_t word = reinterpret_cast<const uint32_t*>(mk)[c / 4];
+          if (((word >> (8 * (c % 4))) & 0xffu) == 0u) s[c] = -INFINITY;
+        }
+      } else if constexpr (MASK == MASK_ADD) {
+        // the additive mask goes into the raw score: s + m / (scale * descales)
+#pragma unroll
+        for (int c = 0; c < HALF_N; c += 2) {
+          const uint32_t word = reinterpret_cast<const uint32_t*>(mk)[c / 2];
+          float2 m2;
+          if constexpr (DT == DT_FP16) {
+            m2 = __half22float2(*reinterpret_cast<const __half2*>(&word));
+          } else {
+            m2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&word));
+          }
+          s[c] = fmaf(m2.x, p.mask_scale, s[c]);
+          s[c + 1] = fmaf(m2.y, p.mask_scale, s[c + 1]);
+        }
+      }
       if (need_mask) {
         const int kh = k0 + half * HALF_N;
         const int hi_c = min(p.Nk - kh, p.causal ? row - kh + 1 : HALF_N);
@@ -993,7 +1048,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, int DT, bool SPLIT>
+template <int D, int DT, bool SPLIT, int MASK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -1055,7 +1110,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // warps take the upper 16 rows of each lane quadrant, the next four the lower
     const int t = warp < 12 ? 0 : 1;
     const int sub = ((warp - 4) >> 2) & 1;
-    softmax_role<D, DT, SPLIT>(sh, tbase, t, sub, p);
+    softmax_role<D, DT, SPLIT, MASK>(sh, tbase, t, sub, p);
   }
   tc_fence_before();
   __syncthreads();

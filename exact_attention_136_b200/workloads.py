@@ -33,6 +33,7 @@ class Workload:
     desc: str
     kv_heads: int = 0   # K/V heads (0 = H); fewer for multi-/grouped-query attention
     splits: int = 1     # key-range slices (fa_fwd_splitkv) for few query rows against many keys
+    mask: str = ""      # "" none; "bool30": boolean [1, 1, N_q, N_k] mask, 30 % of pairs masked out
 
     @property
     def h_kv(self):
@@ -74,6 +75,11 @@ WORKLOADS = {
         1.0 / math.sqrt(128.0), 7,
         "128 query rows against 65536 keys (decode-like: 32 work units for 148 SMs unsplit), "
         "B1 H32 (8 K/V heads) D128 bf16, key range in 4 slices", 8, 4),
+    "mask_b2h16n4096d128_bf16": Workload(
+        "mask_b2h16n4096d128_bf16", 2, 4096, 4096, 16, 128, "bf16", False, -1,
+        1.0 / math.sqrt(128.0), 8,
+        "non-causal B2 H16 N4096 D128 bf16 with a boolean attn_mask [1, 1, N, N] (30 % masked out)",
+        0, 1, "bool30"),
 }
 
 # order used by tests; the headline bench workload is the causal bf16 D128 case
@@ -110,6 +116,18 @@ def element_fraction(n_q, n_k, causal, window_left):
         lo, hi = _visible_range(i, n_k, causal, window_left)
         total += max(0, hi - lo + 1)
     return total / float(n_q * n_k)
+
+
+def make_mask(w: Workload):
+    """The workload's attention mask as a CPU torch tensor (None when it has none); seeded like
+    the inputs (seed 1004 + 100 * index)."""
+    if not w.mask:
+        return None
+    import torch
+    g = torch.Generator().manual_seed(1004 + 100 * w.index)
+    if w.mask == "bool30":
+        return torch.rand((1, 1, w.n_q, w.n_k), generator=g) >= 0.3
+    raise ValueError(f"unknown mask {w.mask!r}")
 
 
 def flops(w: Workload) -> float:

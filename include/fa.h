@@ -132,6 +132,32 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* out, float
                    fa_stream_t stream);
 
 /*
+ * fa_fwd_mask -- the forward of fa_fwd_gqa with an attention mask, the
+ * `attn_mask` of the pages' scaled_dot_product_attention call (Flash
+ * Attention | Hermes Skill, Workflow 1, Step 2), read with that call's
+ * convention:
+ *   FA_MASK_BOOL: bytes, key j takes part for query i where the byte is
+ *                 nonzero;
+ *   FA_MASK_ADD:  16-bit floats (fp16 for fp16 inputs, else bf16) added to
+ *                 the scaled score scale * q_i.k_j before the softmax
+ *                 (-inf removes the key).
+ * Element (b, h, i, j) is at mask + b * mask_stride_b + h * mask_stride_h
+ * + i * mask_stride_q + j (strides in elements; 0 broadcasts over batch or
+ * heads).  mask must be 16-byte aligned, mask_stride_q >= N_k, and every
+ * stride times the element size a multiple of 16 bytes.  Causal and window
+ * visibility apply as well; every key block in their range is computed.
+ * A row whose keys are all masked gets O = 0, LSE = -inf.  Other arguments
+ * and return values as fa_fwd_gqa; FA_ERR_ARG also for a bad mask type,
+ * pointer or stride.
+ */
+typedef enum { FA_MASK_BOOL = 1, FA_MASK_ADD = 2 } fa_mask_type;
+int fa_fwd_mask(const void* q, const void* k, const void* v, void* out, float* lse,
+                int B, int N_q, int N_k, int H, int H_kv, int D, float scale, int causal,
+                int window_left, int dtype, float q_descale, float k_descale, float v_descale,
+                const void* mask, int mask_type, long long mask_stride_b, long long mask_stride_h,
+                long long mask_stride_q, fa_stream_t stream);
+
+/*
  * fa_fwd_host -- the same forward on HOST buffers: copies q, k, v from host
  * to the caller's device buffers dq, dk, dv, runs fa_fwd / fa_fwd_fp8 into
  * dout / dlse, and copies out (and lse, when both lse and dlse are non-NULL)

@@ -35,6 +35,15 @@ arguments; Flash Attention | Hermes Skill, Workflow 2, Steps 2-3):
 Indices are absolute (top-left aligned) also when N_q != N_k; this is the
 plainest reading, since the pages only show N_q == N_k.
 
+Attention mask (the ``attn_mask`` argument of the pages' SDPA call, Flash
+Attention | Hermes Skill, Workflow 1, Step 2).  The pages pass ``mask`` to
+``scaled_dot_product_attention`` without defining it; the reading here is
+that call's convention: a boolean mask keeps key j for query i where it is
+True, a floating-point mask is added to the scaled scores, S_ij =
+scale * q_i.k_j + mask_ij, before the softmax.  It broadcasts over batch and
+heads like ``[B or 1, H or 1, N_q, N_k]`` and applies together with causal
+and window visibility.
+
 Multi-query / grouped-query attention (Flash Attention | Hermes Skill,
 Workflow 2, Step 3 "Enable advanced features": K and V may have fewer heads
 than Q, "shared K/V across heads").  The pages do not say which query heads
@@ -85,7 +94,7 @@ def visibility(rows: Iterable[int], n_k: int, causal: bool, window_left: int) ->
 
 
 def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
-                  rows=None, return_probs: bool = False):
+                  rows=None, return_probs: bool = False, mask=None):
     """Exact attention forward in float64 (definition in the module docstring).
 
     q: [B, N_q, H, D]; k, v: [B, N_k, H_kv, D] with H a multiple of H_kv
@@ -93,6 +102,8 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
        upcast to fp64.
     rows: optional 1-D array of query indices; only those rows are computed
           (used for long sequences where the full N_q x N_k matrix is large).
+    mask: optional boolean (True = attend) or real array broadcastable to
+          [B, H, N_q, N_k]; a real mask is added to the scaled scores.
     Returns (O [B, R, H, D], LSE [B, H, R]) with R = len(rows) (or N_q), and
     with ``return_probs`` also P [B, H, R, N_k].
     """
@@ -110,8 +121,13 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
     group = H // h_kv
     rows = np.arange(n_q, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     R = rows.shape[0]
-    vis = visibility(rows, n_k, causal, window_left)
-    seen = vis.any(axis=1)
+    vis0 = visibility(rows, n_k, causal, window_left)
+    if mask is not None:
+        mask = np.asarray(mask)
+        if mask.ndim != 4 or mask.shape[2] != n_q or mask.shape[3] != n_k or mask.shape[0] not in (1, B) \
+                or mask.shape[1] not in (1, H):
+            raise ValueError("mask must be [B or 1, H or 1, N_q, N_k]")
+        is_bool = mask.dtype == np.bool_
 
     out = np.zeros((B, R, H, D), dtype=np.float64)
     lse = np.full((B, H, R), -np.inf, dtype=np.float64)
@@ -119,8 +135,20 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
     for b in range(B):
         for h in range(H):
             hk = h // group   # key/value head shared by this query head's group
+            vis = vis0
+            add = None
+            if mask is not None:
+                m_bh = mask[b if mask.shape[0] > 1 else 0, h if mask.shape[1] > 1 else 0][rows]
+                if is_bool:
+                    vis = vis0 & m_bh
+                else:
+                    add = m_bh.astype(np.float64)
+                    vis = vis0 & (add > -np.inf)
+            seen = vis.any(axis=1)
             # scores of every selected query against every key
             s = scale * (q[b, rows, h, :] @ k[b, :, hk, :].T)
+            if add is not None:
+                s = s + np.where(vis, add, 0.0)
             s = np.where(vis, s, -np.inf)
             m = np.where(seen, s.max(axis=1, initial=-np.inf), 0.0)
             e = np.where(vis, np.exp(s - m[:, None]), 0.0)
@@ -135,14 +163,16 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
     return out, lse
 
 
-def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_left: int = -1):
+def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_left: int = -1, mask=None):
     """Pure-Python triple loop over (query, key, dim), for tiny shapes only.
 
     Written independently of ``attention_ref``: nested lists, ``math.exp``, no
     max subtraction, and the visibility rule spelled out inline.  Used only to
     pin ``attention_ref``.  Returns (O, LSE) as nested Python lists shaped like
     ``attention_ref``'s outputs.  K and V may have fewer heads than Q (query
-    head h then reads head h * H_kv // H, the same contiguous groups).
+    head h then reads head h * H_kv // H, the same contiguous groups).  mask:
+    optional nested [B or 1][H or 1][N_q][N_k] of booleans (keep where True)
+    or numbers (added to the scaled score).
     """
     B = len(q)
     n_q = len(q[0])
@@ -162,10 +192,20 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
                         continue
                     if window_left != -1 and i - j > window_left:
                         continue
+                    bias = 0.0
+                    if mask is not None:
+                        mval = mask[b if len(mask) > 1 else 0][h if len(mask[0]) > 1 else 0][i][j]
+                        if isinstance(mval, bool):
+                            if not mval:
+                                continue
+                        else:
+                            if mval == float("-inf"):
+                                continue
+                            bias = float(mval)
                     dot = 0.0
                     for d in range(D):
                         dot += float(q[b][i][h][d]) * float(k[b][j][g][d])
-                    weights.append((j, math.exp(scale * dot)))
+                    weights.append((j, math.exp(scale * dot + bias)))
                 total = sum(w for _, w in weights)
                 if not weights:
                     continue

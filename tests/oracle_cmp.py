@@ -17,18 +17,21 @@ def _f64(t: torch.Tensor, descale: float) -> np.ndarray:
     return (t.to(torch.float64) * descale).numpy()
 
 
-def oracle(qkv, scale, causal, window_left, rows=None):
-    """(O [B, R, H, D], LSE [B, H, R]) in float64 for the given QKV bundle."""
+def oracle(qkv, scale, causal, window_left, rows=None, mask=None):
+    """(O [B, R, H, D], LSE [B, H, R]) in float64 for the given QKV bundle (mask: numpy,
+    [B or 1, H or 1, N_q, N_k], bool or real)."""
     B, n_q, H, D = qkv.q.shape
     R = n_q if rows is None else len(rows)
-    if qkv.k.shape[2] != H:
+    if qkv.k.shape[2] != H or mask is not None:
         # grouped K/V heads: the oracle maps query heads to K/V heads itself
         # (one batch at a time, all heads)
         O = np.zeros((B, R, H, D))
         L = np.zeros((B, H, R))
         for b in range(B):
+            mb = None if mask is None else mask[b:b + 1] if mask.shape[0] > 1 else mask
             o, l = attention_ref(_f64(qkv.q[b:b + 1], qkv.q_descale), _f64(qkv.k[b:b + 1], qkv.k_descale),
-                                 _f64(qkv.v[b:b + 1], qkv.v_descale), scale, causal, window_left, rows=rows)
+                                 _f64(qkv.v[b:b + 1], qkv.v_descale), scale, causal, window_left, rows=rows,
+                                 mask=mb)
             O[b], L[b] = o[0], l[0]
         return O, L
     O = np.zeros((B, R, H, D))

@@ -137,3 +137,15 @@ def test_splitkv_arguments_validated(splits, ws, nbytes):
     f = _lib.lib().fa_fwd_splitkv
     assert f(A, A, A, A, None, 1, 16, 1024, 4, 4, 128, 0.1, 0, -1, _lib.FA_BF16, 1.0, 1.0, 1.0, splits, ws, nbytes,
              None) == _lib.FA_ERR_ARG
+
+
+@pytest.mark.parametrize("kind, mask, sb, sh, sq", [
+    (0, A, 0, 0, 128), (3, A, 0, 0, 128), (_lib.FA_MASK_BOOL, None, 0, 0, 128),
+    (_lib.FA_MASK_BOOL, A + 8, 0, 0, 128), (_lib.FA_MASK_BOOL, A, 0, 0, 100),     # misaligned, short row
+    (_lib.FA_MASK_BOOL, A, 0, 0, 136), (_lib.FA_MASK_ADD, A, 0, 4, 128),           # strides not 16 B
+    (_lib.FA_MASK_ADD, A, -128, 0, 128)])
+def test_mask_arguments_validated(kind, mask, sb, sh, sq):
+    """Mask kind, pointer and strides are checked on the host, before any GPU work."""
+    f = _lib.lib().fa_fwd_mask
+    assert f(A, A, A, A, None, 1, 16, 128, 4, 4, 128, 0.1, 0, -1, _lib.FA_BF16, 1.0, 1.0, 1.0, mask, kind, sb, sh,
+             sq, None) == _lib.FA_ERR_ARG

@@ -386,3 +386,101 @@ def test_planted_head_map_mistake_is_caught():
         except AssertionError:
             caught = True
     assert caught
+
+
+# --------------------------------------------------------------------------
+# attention mask (boolean: attend where True; real: added to scale * q.k),
+# broadcast over batch / heads
+# --------------------------------------------------------------------------
+
+def _bool_mask(shape, seed):
+    m = np.random.default_rng(seed).random(shape) > 0.35
+    return m
+
+
+def mask_pin_bruteforce(fn):
+    """Against the brute force for boolean and additive masks, broadcast and not."""
+    q, k, v = _rand((2, 7, 2, 4), 90), _rand((2, 9, 2, 4), 91), _rand((2, 9, 2, 4), 92)
+    masks = [_bool_mask((2, 2, 7, 9), 93), _bool_mask((1, 2, 7, 9), 94), _rand((2, 1, 7, 9), 95),
+             np.where(_bool_mask((1, 1, 7, 9), 96), _rand((1, 1, 7, 9), 97), -np.inf)]
+    for m in masks:
+        for causal, wl in [(False, -1), (True, -1), (True, 2)]:
+            o, l = fn(q, k, v, 0.6, causal, wl, mask=m)
+            ob, lb = attention_bruteforce(q.tolist(), k.tolist(), v.tolist(), 0.6, causal, wl, mask=m.tolist())
+            np.testing.assert_allclose(o, np.array(ob), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(l, np.array(lb), rtol=0, atol=1e-12)
+
+
+def mask_pin_zero_query(fn):
+    """Q = 0: the scores are the additive mask alone, so O = softmax(mask) V and
+    LSE = logsumexp(mask) (scipy) -- also fixes that the mask is added after scaling."""
+    q = np.zeros((1, 6, 1, 4))
+    k, v = _rand((1, 11, 1, 4), 98), _rand((1, 11, 1, 4), 99)
+    m = 3.0 * _rand((1, 1, 6, 11), 100)
+    o, l = fn(q, k, v, 0.37, False, -1, mask=m)
+    p = scipy.special.softmax(m[0, 0], axis=-1)
+    np.testing.assert_allclose(o[0, :, 0], p @ v[0, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l[0, 0], scipy.special.logsumexp(m[0, 0], axis=-1), rtol=0, atol=1e-12)
+
+
+def mask_pin_causal_pattern(fn):
+    """A boolean mask holding the causal pattern (and an additive one holding -inf above the
+    diagonal) is causal attention."""
+    q, k, v = _rand((1, 13, 2, 4), 101), _rand((1, 13, 2, 4), 102), _rand((1, 13, 2, 4), 103)
+    tri = np.tril(np.ones((13, 13), dtype=bool))[None, None]
+    o_c, l_c = fn(q, k, v, 0.5, True, -1)
+    o_b, l_b = fn(q, k, v, 0.5, False, -1, mask=tri)
+    o_a, l_a = fn(q, k, v, 0.5, False, -1, mask=np.where(tri, 0.0, -np.inf))
+    for o, l in [(o_b, l_b), (o_a, l_a)]:
+        np.testing.assert_allclose(o, o_c, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l, l_c, rtol=0, atol=1e-13)
+
+
+def mask_pin_row_constant(fn):
+    """Adding a per-row constant c_i to every score of row i leaves O and moves LSE by c_i."""
+    q, k, v = _rand((1, 8, 1, 4), 104), _rand((1, 8, 1, 4), 105), _rand((1, 8, 1, 4), 106)
+    c = np.linspace(-2.0, 5.0, 8)
+    m = np.broadcast_to(c[None, None, :, None], (1, 1, 8, 8))
+    o0, l0 = fn(q, k, v, 0.8, True, -1)
+    o1, l1 = fn(q, k, v, 0.8, True, -1, mask=m)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1[0, 0], l0[0, 0] + c, rtol=0, atol=1e-12)
+
+
+MASK_PINS = [mask_pin_bruteforce, mask_pin_zero_query, mask_pin_causal_pattern, mask_pin_row_constant]
+
+
+@pytest.mark.parametrize("pin", MASK_PINS, ids=[p.__name__ for p in MASK_PINS])
+def test_oracle_mask_pin(pin):
+    pin(attention_ref)
+
+
+def test_fully_masked_rows_are_empty():
+    q, k, v = _rand((1, 4, 1, 4), 107), _rand((1, 5, 1, 4), 108), _rand((1, 5, 1, 4), 109)
+    m = np.ones((1, 1, 4, 5), dtype=bool)
+    m[0, 0, 2] = False
+    o, l = attention_ref(q, k, v, 1.0, mask=m)
+    assert np.all(o[0, 2] == 0.0) and l[0, 0, 2] == -np.inf and np.all(np.isfinite(l[0, 0, [0, 1, 3]]))
+
+
+@pytest.mark.parametrize("bad", ["before_scale", "inverted", "transposed"])
+def test_planted_mask_application_mistake_is_caught(bad):
+    def mutated(q, k, v, scale, causal=False, wl=-1, mask=None, **kw):
+        if mask is None:
+            return attention_ref(q, k, v, scale, causal, wl, mask=mask, **kw)
+        m = np.asarray(mask)
+        if bad == "before_scale" and m.dtype != np.bool_:
+            m = m / scale            # the mask scaled along with the scores
+        elif bad == "inverted" and m.dtype == np.bool_:
+            m = ~m
+        elif bad == "transposed" and m.shape[2] == m.shape[3]:
+            m = np.swapaxes(m, 2, 3)
+        return attention_ref(q, k, v, scale, causal, wl, mask=m, **kw)
+
+    caught = False
+    for pin in MASK_PINS:
+        try:
+            pin(mutated)
+        except AssertionError:
+            caught = True
+    assert caught

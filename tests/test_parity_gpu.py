@@ -192,6 +192,68 @@ def test_splitkv_one_slice_is_the_plain_forward():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+# attention mask: (B, N_q, N_k, H, D, dtype, causal, window_left, kind, mask batch, mask heads)
+MASKED = [
+    (2, 256, 256, 2, 128, "bf16", False, -1, "bool", 2, 2),
+    (1, 300, 517, 2, 64, "fp16", True, -1, "bool", 1, 1),      # N_k not a multiple of 16: padded rows
+    (2, 384, 384, 2, 128, "bf16", False, -1, "add", 2, 1),
+    (1, 200, 333, 2, 128, "fp16", False, 100, "add", 1, 2),
+    (1, 500, 500, 2, 128, "e4m3", True, -1, "add", 1, 1),
+    (1, 257, 257, 1, 64, "bf16", False, -1, "bool_rows", 1, 1),  # some rows fully masked
+]
+
+
+def _make_mask(case, seed):
+    B, nq, nk, H, D, dt, causal, wl, kind, mb, mh = case
+    g = torch.Generator().manual_seed(seed)
+    if kind.startswith("bool"):
+        m = torch.rand((mb, mh, nq, nk), generator=g) > 0.3
+        if kind == "bool_rows":
+            m[:, :, ::7] = False
+        return m, m.numpy()
+    t = torch.float16 if dt == "fp16" else torch.bfloat16
+    m = (2.0 * torch.randn((mb, mh, nq, nk), generator=g)).to(t)
+    m[torch.rand((mb, mh, nq, nk), generator=g) < 0.1] = float("-inf")
+    return m, m.to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("case", MASKED, ids=[
+    f"B{c[0]}_q{c[1]}_k{c[2]}_H{c[3]}_D{c[4]}_{c[5]}_{'c' if c[6] else 'nc'}_w{c[7]}_{c[8]}_mb{c[9]}mh{c[10]}"
+    for c in MASKED])
+def test_attn_mask_parity(case):
+    B, nq, nk, H, D, dt, causal, wl, kind, mb, mh = case
+    qkv = inputs.make_qkv(B, nq, nk, H, D, dt, seeds=(91 + nq, 92 + nk, 93 + H))
+    mask_t, mask_np = _make_mask(case, 94 + nq)
+    dev = torch.device("cuda", 0)
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    scale = 1.0 / math.sqrt(D)
+    if dt == "e4m3":
+        out, lse = forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, scale, causal, wl,
+                               attn_mask=mask_t.to(dev))
+    else:
+        out, lse = forward(q, k, v, scale, causal, wl, attn_mask=mask_t.to(dev))
+    torch.cuda.synchronize()
+    rc, flags = device_status()
+    assert rc == 0, f"device status {rc} flags {flags}"
+    ref_o, ref_l = oracle(qkv, scale, causal, wl, mask=mask_np)
+    d_o, d_l = compare(out, lse, ref_o, ref_l)
+    assert d_o <= TOL_O[dt], f"max|dO| {d_o:.3e} > {TOL_O[dt]}"
+    assert d_l <= TOL_LSE, f"max|dLSE| {d_l:.3e} > {TOL_LSE}"
+
+
+def test_causal_pattern_mask_equals_causal():
+    """A boolean mask holding the causal pattern gives the causal forward (to rounding)."""
+    qkv = inputs.make_qkv(1, 640, 640, 2, 128, "bf16", seeds=(95, 96, 97))
+    dev = torch.device("cuda", 0)
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    tri = torch.tril(torch.ones((640, 640), dtype=torch.bool, device=dev))
+    o1, l1 = forward(q, k, v, 0.09, True, -1)
+    o2, l2 = forward(q, k, v, 0.09, False, -1, attn_mask=tri)
+    torch.cuda.synchronize()
+    assert float((o1.float() - o2.float()).abs().max()) <= 8e-3
+    assert float((l1 - l2).abs().max()) <= 1e-4
+
+
 @pytest.mark.parametrize("dt,D", [("fp16", 64), ("bf16", 128), ("e4m3", 128)])
 @pytest.mark.parametrize("mult", [4.0, 12.0])
 def test_large_scores_exercise_rescaling(dt, D, mult):
@@ -233,9 +295,17 @@ def test_full_workload_sampled_rows(name):
     w = W.WORKLOADS[name]
     qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=w.seeds, h_kv=w.h_kv)
     rows = W.sample_rows(w, count=64 if w.n_q > 4096 else 256)
-    out, lse = run(qkv, w.scale, w.causal, w.window_left, num_splits=w.splits)
+    mask = W.make_mask(w)
+    if mask is None:
+        out, lse = run(qkv, w.scale, w.causal, w.window_left, num_splits=w.splits)
+    else:
+        dev = torch.device("cuda", 0)
+        out, lse = forward(qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev), w.scale, w.causal, w.window_left,
+                           attn_mask=mask.to(dev))
+        torch.cuda.synchronize()
     assert bool(torch.isfinite(out).all()) and bool(torch.isfinite(lse).all())
-    ref_o, ref_l = oracle(qkv, w.scale, w.causal, w.window_left, rows=rows)
+    ref_o, ref_l = oracle(qkv, w.scale, w.causal, w.window_left, rows=rows,
+                          mask=None if mask is None else mask.numpy())
     d_o, d_l = compare(out, lse, ref_o, ref_l, rows=rows)
     assert d_o <= TOL_O[w.dtype] and d_l <= TOL_LSE, (d_o, d_l)
 

@@ -72,6 +72,7 @@ __all__ = [
     "visibility",
     "attention_ref",
     "attention_bruteforce",
+    "attention_backward_ref",
 ]
 
 
@@ -216,3 +217,55 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
                         acc += w * float(v[b][j][g][d])
                     O[b][i][h][d] = acc / total
     return O, L
+
+
+def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, window_left: int = -1):
+    """Gradients of the exact attention forward, in float64.
+
+    The pages name the backward pass only by its method: the speed and memory
+    savings come from tiling and recomputation, i.e. the attention matrix is
+    recomputed from the inputs instead of stored (Flash Attention | Hermes
+    Skill, "Quick start"; the same on the Russian mirror "Flash Attention -
+    Fast Memory-Efficient Attention"), and FlashAttention-3 runs FP16/BF16
+    forward and backward (same pages, "Workflow 3: H100 FP8 optimization
+    (FlashAttention-3)").  What it computes is fixed by the forward:
+    for an upstream gradient dO of O, the vector-Jacobian products
+
+        dV = P^T dO
+        dP = dO V^T
+        dS_ij = P_ij (dP_ij - sum_j' P_ij' dP_ij')      (softmax Jacobian)
+        dQ = scale * dS K
+        dK = scale * dS^T Q
+
+    with P, S, visibility and the K/V head of each query head exactly as in
+    ``attention_ref``; a K/V head shared by a group of query heads gets the sum
+    of their dK and dV.  Invisible (i, j) pairs have P_ij = 0 and contribute
+    nothing, and a row with no visible key contributes nothing at all.
+
+    q, do: [B, N_q, H, D]; k, v: [B, N_k, H_kv, D].  Returns (dQ, dK, dV)
+    shaped like q, k, v.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    B, n_q, H, D = q.shape
+    n_k, h_kv = k.shape[1], k.shape[2]
+    if do.shape != q.shape:
+        raise ValueError("do must be shaped like q")
+    _, _, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True)
+    group = H // h_kv
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            hk = h // group
+            p = probs[b, h]                       # [N_q, N_k], zero where invisible
+            g = do[b, :, h, :]                    # [N_q, D]
+            dv[b, :, hk, :] += p.T @ g
+            dp = g @ v[b, :, hk, :].T             # [N_q, N_k]
+            ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+            dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])
+            dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])
+    return dq, dk, dv

@@ -484,3 +484,143 @@ def test_planted_mask_application_mistake_is_caught(bad):
         except AssertionError:
             caught = True
     assert caught
+
+
+# --------------------------------------------------------------------------
+# backward: pins for attention_backward_ref.  Each pin takes a function with
+# its signature; the finite-difference pin uses only the forward oracle.
+# --------------------------------------------------------------------------
+
+BWD_MODES = [(False, -1), (True, -1), (True, 1), (False, 2)]
+
+
+def _fd_grads(q, k, v, do, scale, causal, wl, eps=1e-6):
+    """Central differences of L = sum(dO * O(q, k, v)) through attention_ref."""
+    def loss(q_, k_, v_):
+        o, _ = attention_ref(q_, k_, v_, scale, causal, wl)
+        return float(np.sum(do * o))
+    grads = []
+    for which in range(3):
+        args = [q.copy(), k.copy(), v.copy()]
+        g = np.zeros_like(args[which])
+        it = np.nditer(g, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            g[idx] = (loss(*plus) - loss(*minus)) / (2 * eps)
+        grads.append(g)
+    return grads
+
+
+def pin_backward_finite_differences(fn):
+    for (n_q, n_k, H, h_kv, D) in [(5, 5, 2, 2, 3), (7, 4, 2, 1, 4), (3, 8, 4, 2, 2)]:
+        for causal, wl in BWD_MODES:
+            q = _rand((1, n_q, H, D), 300 + n_q)
+            k = _rand((1, n_k, h_kv, D), 310 + n_k)
+            v = _rand((1, n_k, h_kv, D), 320 + D)
+            do = _rand((1, n_q, H, D), 330 + H)
+            got = fn(q, k, v, do, 0.6, causal, wl)
+            want = _fd_grads(q, k, v, do, 0.6, causal, wl)
+            for g, w in zip(got, want):
+                assert np.allclose(g, w, rtol=1e-6, atol=1e-7), float(np.max(np.abs(g - w)))
+
+
+def pin_backward_key_shift_invariance(fn):
+    # adding one vector to every key moves each query's scores by a constant:
+    # O does not change, so the key gradients of each head sum to zero
+    for causal, wl in BWD_MODES:
+        q = _rand((2, 9, 2, 4), 340)
+        k = _rand((2, 9, 2, 4), 341)
+        v = _rand((2, 9, 2, 4), 342)
+        do = _rand((2, 9, 2, 4), 343)
+        _, dk, _ = fn(q, k, v, do, 0.8, causal, wl)
+        assert np.allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+
+
+def pin_backward_uniform_attention(fn):
+    # Q = 0: every visible key of row i has weight 1 / n_i, so
+    # dV_j = sum over the rows that see key j of dO_i / n_i
+    for causal, wl in BWD_MODES:
+        n, D = 8, 3
+        q = np.zeros((1, n, 1, D))
+        k = _rand((1, n, 1, D), 350)
+        v = _rand((1, n, 1, D), 351)
+        do = _rand((1, n, 1, D), 352)
+        _, _, dv = fn(q, k, v, do, 1.3, causal, wl)
+        want = np.zeros((n, D))
+        for i in range(n):
+            seen = [j for j in range(n) if (not causal or j <= i) and (wl < 0 or j >= i - wl)]
+            for j in seen:
+                want[j] += do[0, i, 0] / len(seen)
+        assert np.allclose(dv[0, :, 0], want, atol=1e-13)
+
+
+def pin_backward_value_linearity(fn):
+    # O is linear in V with weights P: for dO = 1 in one column, dV's column
+    # is the column sums of P
+    for causal, wl in BWD_MODES:
+        q = _rand((1, 6, 1, 2), 360)
+        k = _rand((1, 6, 1, 2), 361)
+        v = _rand((1, 6, 1, 2), 362)
+        do = np.zeros((1, 6, 1, 2))
+        do[..., 1] = 1.0
+        _, _, p = attention_ref(q, k, v, 0.9, causal, wl, return_probs=True)
+        _, _, dv = fn(q, k, v, do, 0.9, causal, wl)
+        assert np.allclose(dv[0, :, 0, 1], p[0, 0].sum(axis=0), atol=1e-13)
+        assert np.allclose(dv[0, :, 0, 0], 0.0, atol=1e-15)
+
+
+BWD_PINS = [pin_backward_finite_differences, pin_backward_key_shift_invariance, pin_backward_uniform_attention,
+            pin_backward_value_linearity]
+
+
+@pytest.mark.parametrize("pin", BWD_PINS)
+def test_oracle_backward_pin(pin):
+    pin(oa.attention_backward_ref)
+
+
+def _bwd_mutant(kind):
+    """attention_backward_ref with one plausible mistake planted."""
+    def fn(q, k, v, do, scale, causal, wl):
+        B, n_q, H, D = q.shape
+        h_kv = k.shape[2]
+        _, _, probs = attention_ref(q, k, v, scale, causal, wl, return_probs=True)
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        for b in range(B):
+            for h in range(H):
+                hk = h // (H // h_kv)
+                p, g = probs[b, h], do[b, :, h, :]
+                dv[b, :, hk, :] += (p if kind == "dv_untransposed" and n_q == p.shape[1] else p.T) @ g
+                dp = g @ v[b, :, hk, :].T
+                row = (p * dp).sum(axis=1, keepdims=True)
+                ds = p * dp if kind == "no_row_term" else p * (dp - row)
+                if kind == "sign":
+                    ds = -ds
+                s = 1.0 if kind == "no_scale" else scale
+                dq[b, :, h, :] = s * (ds @ k[b, :, hk, :])
+                dk_h = s * (ds.T @ q[b, :, h, :])
+                if kind == "last_group_head_only":
+                    dk[b, :, hk, :] = dk_h
+                else:
+                    dk[b, :, hk, :] += dk_h
+        return dq, dk, dv
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["no_row_term", "sign", "no_scale", "last_group_head_only", "dv_untransposed"])
+def test_planted_backward_mistake_is_caught(kind):
+    caught = False
+    for pin in BWD_PINS:
+        try:
+            pin(_bwd_mutant(kind))
+        except AssertionError:
+            caught = True
+    assert caught, kind
+
+
+def test_backward_mutant_harness_without_mistake_passes():
+    for pin in BWD_PINS:
+        pin(_bwd_mutant("none"))

@@ -14,6 +14,10 @@ data path).
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (rank 0 only).
+
+--backward times the backward instead (fa_bwd: dQ, dK, dV from a fixed
+forward's O and LSE and a random dO), credited 2.5x the forward's FLOP (five
+matrix products per block against two).
 """
 
 from __future__ import annotations
@@ -41,12 +45,15 @@ from exact_attention_136_b200 import workloads as W  # noqa: E402
 from exact_attention_136_b200 import inputs  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s and % of dense tensor peak (1×B200) vs CPU oracle"
+METRIC_BWD = "attention bwd TFLOP/s and % of dense tensor peak (1×B200) vs CPU oracle"
+BWD_FLOP_RATIO = 2.5
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_TFLOPS = {"fp16": 2250.0, "bf16": 2250.0, "e4m3": 4500.0}
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["exact_attention_136_b200/csrc/fa_fwd_kernel.cuh", "exact_attention_136_b200/csrc/sm100.cuh",
+                  "exact_attention_136_b200/csrc/fa_bwd_kernel.cuh",
                   "exact_attention_136_b200/csrc/fa_api.cu", "exact_attention_136_b200/csrc/tmap.h"]
 
 
@@ -229,6 +236,7 @@ def main():
     ap.add_argument("--reference-rows", type=int, default=256, help="oracle rows per step in --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling cases)")
+    ap.add_argument("--backward", action="store_true", help="time the backward (fa_bwd) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -252,6 +260,9 @@ def main():
     if args.batch is not None:
         import dataclasses
         w = dataclasses.replace(w, B=args.batch, name=f"{w.name}@B{args.batch}")
+    if args.backward:
+        run_backward(args, w, world, rank, local, dev)
+        return
     seeds = rank_seeds(w, rank)   # each rank: its own batch
     qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=seeds, h_kv=w.h_kv)
     hq, hk, hv = qkv.q.pin_memory(), qkv.k.pin_memory(), qkv.v.pin_memory()
@@ -386,6 +397,135 @@ def main():
         "cpu_baseline": cpu,
         "clocks": clocks,
         "gpu_launches": args.steps,
+        "kernel_hash": kernel_hash(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def oracle_backward_tflops(w: W.Workload, qkv, dout):
+    """The fp64 oracle's backward on one full (batch, head) of the workload
+    (bounded sample: about 10-30 s for N = 8192); FLOP credited like the GPU's."""
+    sys.path.insert(0, ROOT)
+    from oracle import attention_backward_ref
+    f = lambda t: t[:1, :, :1].double().numpy()
+    t0 = time.perf_counter()
+    attention_backward_ref(f(qkv.q), f(qkv.k), f(qkv.v), f(dout), w.scale, w.causal, w.window_left)
+    dt = time.perf_counter() - t0
+    flop = BWD_FLOP_RATIO * W.flops(w) / (w.B * w.H)
+    return flop / dt / 1e12, dt, blas_threads()
+
+
+def run_backward(args, w, world, rank, local, dev):
+    from exact_attention_136_b200 import backward, device_status, forward
+
+    if w.dtype == "e4m3" or w.h_kv != w.H or w.mask or w.splits != 1:
+        raise SystemExit("--backward takes fp16 / bf16 workloads with K/V heads = query heads, no mask or split")
+    seeds = rank_seeds(w, rank)
+    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=seeds)
+    g = inputs.make_qkv(w.B, w.n_q, w.n_q, w.H, w.D, w.dtype, seeds=tuple(x + 17 for x in seeds)).q
+    host = {n: t.pin_memory() for n, t in (("q", qkv.q), ("k", qkv.k), ("v", qkv.v), ("dout", g))}
+    q, k, v, dout = (host[n].to(dev) for n in ("q", "k", "v", "dout"))
+    stream = torch.cuda.current_stream(dev)
+    out, lse = forward(q, k, v, w.scale, w.causal, w.window_left, stream=stream)
+    host["out"], host["lse"] = out.cpu().pin_memory(), lse.cpu().pin_memory()
+
+    def step():
+        return backward(q, k, v, out, lse, dout, w.scale, w.causal, w.window_left, stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        grads = step()
+    torch.cuda.synchronize(dev)
+    rc, flags = device_status(device=dev)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} flags {flags} after warm-up")
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        grads = step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    rc, flags = device_status(device=dev)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} flags {flags} in the timed region")
+    if not all(bool(torch.isfinite(t).all()) for t in grads):
+        raise RuntimeError("non-finite gradient")
+    flops = BWD_FLOP_RATIO * W.flops(w)
+    ms_per_step = ms / args.steps
+    value = world * flops * args.steps / (ms / 1e3) / 1e12
+    per_step_tflops = flops / (ms_per_step / 1e3) / 1e12
+
+    # end to end: inputs (q, k, v, out, lse, dout) from pinned host memory,
+    # the backward, and dq, dk, dv back to pinned host memory
+    hg = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (q, k, v)]
+
+    def e2e_step():
+        for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout)):
+            t.copy_(host[name], non_blocking=True)
+        for hdst, dsrc in zip(hg, step()):
+            hdst.copy_(dsrc, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ems = max_over_ranks(t0.elapsed_time(t1), dev)
+    e2e_value = world * flops * args.e2e_steps / (ems / 1e3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in hg)
+
+    peak, peak_src, sustained = measured_peaks(w.dtype)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, dt, threads = oracle_backward_tflops(w, qkv, g)
+        cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 oracle backward on one full (batch, head) of the {w.B * w.H} ({dt:.1f} s); "
+                         f"FLOP credited as 2.5x the forward's per head"}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, out, dout))
+    line = {
+        "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": "bwd_" + w.name, "desc": "backward of " + w.desc, "B": w.B, "N_q": w.n_q,
+                   "N_k": w.n_k, "H": w.H, "D": w.D, "causal": w.causal, "window_left": w.window_left,
+                   "scale": w.scale, "flop_per_step": flops,
+                   "block_fraction": W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left),
+                   "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB vs {L2_BYTES / 1e6:.0f} MB), no flush",
+                   "pct_of_nominal_dense_peak": 100.0 * per_step_tflops / NOMINAL_TFLOPS[w.dtype],
+                   "nominal_dense_peak_tflops": NOMINAL_TFLOPS[w.dtype],
+                   "parallelism": f"replicas x{world} (independent batches per GPU)"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps, "api": "pinned host copies + backward"},
+        "roofline": {"bound": "tensor", "achieved": per_step_tflops, "peak": peak, "unit": UNIT,
+                     "frac": per_step_tflops / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst", "peak_sustained": sustained,
+                     "note": "achieved over the whole step (four kernels; the main kernel is ~all of it)"},
+        "cpu_baseline": cpu,
+        "clocks": clocks,
+        "gpu_launches": 4 * args.steps,
         "kernel_hash": kernel_hash(),
     }
     print(json.dumps(line), flush=True)

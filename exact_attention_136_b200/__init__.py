@@ -1,12 +1,15 @@
-"""Exact attention forward for NVIDIA B200 (sm_100a).
+"""Exact attention forward and backward for NVIDIA B200 (sm_100a).
 
-    from exact_attention_136_b200 import forward
+    from exact_attention_136_b200 import forward, backward
     out, lse = forward(q, k, v, causal=True)      # [batch, seqlen, heads, headdim]
+    dq, dk, dv = backward(q, k, v, out, lse, dout, causal=True)
 
 The computation runs in libfa_b200.so (hand-written sm_100a CUDA, C ABI in
 include/fa.h); this package only marshals arguments.
 """
 
-from .api import auto_splits, device_status, forward, forward_fp8, forward_host, set_wait_limit_ns, wait_probe
+from .api import (auto_splits, backward, device_status, forward, forward_fp8, forward_host, set_wait_limit_ns,
+                  wait_probe)
 
-__all__ = ["forward", "forward_fp8", "forward_host", "auto_splits", "device_status", "set_wait_limit_ns", "wait_probe"]
+__all__ = ["forward", "forward_fp8", "forward_host", "backward", "auto_splits", "device_status",
+           "set_wait_limit_ns", "wait_probe"]

@@ -199,6 +199,39 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
     return out, lse
 
 
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+             dout: torch.Tensor, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,
+             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients (dq, dk, dv) of forward(q, k, v, scale, causal, window_left)
+    for the upstream gradient dout, from the forward's out and lse (fp16 /
+    bf16, K/V heads equal to query heads).  The fp32 workspace the library
+    needs is taken from torch's allocator for the call."""
+    B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
+    if h_kv != H:
+        raise ValueError("backward needs as many K/V heads as query heads")
+    if q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("backward takes fp16 or bf16 inputs")
+    for name, t in (("out", out), ("dout", dout)):
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous tensor like q")
+    if lse.shape != (B, H, n_q) or lse.dtype != torch.float32 or lse.device != q.device or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, N_q] tensor on q's device")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        nbytes = int(_lib.lib().fa_bwd_workspace_bytes(B, n_q, H, D))
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+        rc = _lib.lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                               lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H, D, scale,
+                               int(bool(causal)), int(window_left), _DT[q.dtype], ws.data_ptr(), nbytes,
+                               s.cuda_stream)
+        # keep the workspace alive until the kernels that use it have run
+        ws.record_stream(s)
+    _lib.check(rc, "fa_bwd")
+    return dq, dk, dv
+
+
 def forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, staging, scale: float, causal: bool = False,
                  window_left: int = -1, descales=(1.0, 1.0, 1.0), out: Optional[torch.Tensor] = None,
                  lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):

@@ -8,6 +8,7 @@
 
 #include "../../include/fa.h"
 #include "fa_fwd_kernel.cuh"
+#include "fa_bwd_kernel.cuh"
 #include "tmap.h"
 
 namespace fa {
@@ -305,6 +306,103 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
 
 size_t elem_bytes(int dtype) { return dtype == FA_E4M3 ? 1 : 2; }
 
+// Workspace of the backward: fp32 dQ accumulator [B, N_q, H, D] followed by
+// D_i = rowsum(dO * O) [B, H, N_q].
+size_t bwd_workspace_bytes(int B, int Nq, int H, int D) {
+  return static_cast<size_t>(B) * Nq * H * (static_cast<size_t>(D) + 1) * sizeof(float);
+}
+
+template <int D, int DT>
+int launch_bwd(const void* q, const void* k, const void* v, const void* dout, const BwdParams& p,
+               cudaStream_t stream, DeviceState* ds, int bit) {
+  using C = BwdCfg<D>;
+  const CUtensorMapDataType tdt = DT == DT_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap mq, mk, mv, mdo;
+  if (encode_bnhd(&mq, q, tdt, 2, p.B, p.Nq, p.H, D, 64, 128) ||
+      encode_bnhd(&mk, k, tdt, 2, p.B, p.Nk, p.H, D, 64, 128) ||
+      encode_bnhd(&mv, v, tdt, 2, p.B, p.Nk, p.H, D, 64, 128) ||
+      encode_bnhd(&mdo, dout, tdt, 2, p.B, p.Nq, p.H, D, 64, 128))
+    return FA_ERR_CUDA;
+  if (!(ds->attr_set & (1u << bit))) {
+    if (cudaFuncSetAttribute(fa_bwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    ds->attr_set |= (1u << bit);
+  }
+  const int64_t grid = static_cast<int64_t>(p.nkb) * p.B * p.H;
+  if (grid > 0x7fffffff) return FA_ERR_ARG;
+  fa_bwd_kernel<D, DT><<<static_cast<int>(grid), BWD_THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int backward(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+             void* dq, void* dk, void* dv, int B, int Nq, int Nk, int H, int D, float scale, int causal,
+             int window_left, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int rc = validate(q, k, v, const_cast<void*>(out), B, Nq, Nk, H, D, scale, causal, window_left, dtype, H);
+  if (rc != FA_OK) return rc;
+  if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
+  if ((Nq > 0 && (!dout || !lse || !dq)) || (Nk > 0 && (!dk || !dv))) return FA_ERR_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return FA_ERR_ALIGN;
+  const size_t ws = bwd_workspace_bytes(B, Nq, H, D);
+  if (ws > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws))
+    return FA_ERR_ARG;
+  if (Nq == 0 && Nk == 0) return FA_OK;
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if (Nq == 0) {
+    // no query sees any key: dK = dV = 0
+    const size_t kv_bytes = static_cast<size_t>(B) * Nk * H * D * 2;
+    if (cudaMemsetAsync(dk, 0, kv_bytes, stream) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  float* dq_acc = static_cast<float*>(workspace);
+  float* delta = dq_acc + static_cast<size_t>(B) * Nq * H * D;
+  const int64_t rows = static_cast<int64_t>(B) * Nq * H;
+  {
+    const int64_t want = (rows + 7) / 8;
+    const int blocks = static_cast<int>(want < 8 * 148 ? want : 8 * 148);
+    if (D == 64) fa_bwd_prologue_kernel<64><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, dq_acc, B, Nq, H);
+    else fa_bwd_prologue_kernel<128><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, dq_acc, B, Nq, H);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (Nk > 0) {
+    BwdParams p{};
+    p.dk = dk;
+    p.dv = dv;
+    p.dq_acc = dq_acc;
+    p.lse = lse;
+    p.delta = delta;
+    p.B = B;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.H = H;
+    p.causal = causal;
+    p.window_left = window_left;
+    p.scale = scale;
+    p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.nkb = (Nk + 127) / 128;
+    p.wait_limit_ns = g_wait_limit_ns;
+    p.status = ds->status;
+    switch (dtype * 2 + (D == 128 ? 1 : 0)) {
+      case FA_FP16 * 2 + 0: rc = launch_bwd<64, DT_FP16>(q, k, v, dout, p, stream, ds, 20); break;
+      case FA_FP16 * 2 + 1: rc = launch_bwd<128, DT_FP16>(q, k, v, dout, p, stream, ds, 21); break;
+      case FA_BF16 * 2 + 0: rc = launch_bwd<64, DT_BF16>(q, k, v, dout, p, stream, ds, 22); break;
+      case FA_BF16 * 2 + 1: rc = launch_bwd<128, DT_BF16>(q, k, v, dout, p, stream, ds, 23); break;
+      default: return FA_ERR_UNSUPPORTED;
+    }
+    if (rc != FA_OK) return rc;
+  }
+  const long long n = static_cast<long long>(rows) * D;
+  const long long want = (n / 4 + 255) / 256;
+  const int blocks = static_cast<int>(want < 16 * 148 ? want : 16 * 148);
+  fa_bwd_epilogue_kernel<<<blocks, 256, 0, stream>>>(dq_acc, dq, dtype, n);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -407,6 +505,18 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float
     return FA_ERR_CUDA;
   return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H, D, scale, causal, window_left, dtype, q_descale,
                      k_descale, v_descale, s, scratch);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int N_q, int H, int D) {
+  if (B < 1 || N_q < 0 || H < 1 || (D != 64 && D != 128)) return 0;
+  return fa::bwd_workspace_bytes(B, N_q, H, D);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int D, float scale, int causal,
+           int window_left, int dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, D, scale, causal, window_left, dtype,
+                      workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_device_status(fa_stream_t stream, int* flags) {

@@ -197,6 +197,35 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float
                    float v_descale, fa_stream_t stream);
 
 /*
+ * fa_bwd -- gradients of the forward for FA_FP16 / FA_BF16 inputs (K/V heads
+ * equal to query heads): given dout = dL/dO, writes dq = dL/dQ, dk, dv.  The
+ * pages give the backward only by its method, recomputation of the attention
+ * matrix from the inputs and the forward's softmax statistics (Flash
+ * Attention | Hermes Skill, "Quick start"; FlashAttention-3 FP16/BF16
+ * forward and backward, "Workflow 3: H100 FP8 optimization
+ * (FlashAttention-3)"); the result is the exact vector-Jacobian product of
+ * the forward defined above:
+ *     P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,
+ *     dS = P * (dP - rowsum(dO * O)),  dQ = scale dS K,  dK = scale dS^T Q.
+ *   q, k, v, out, lse: the forward's inputs and outputs (same B, N_q, N_k,
+ *     H, D, scale, causal, window_left, dtype); lse is required here.
+ *   dout, dq: [B, N_q, H, D]; dk, dv: [B, N_k, H, D]; 16-bit like q.
+ *   workspace: caller-owned device memory of at least
+ *     fa_bwd_workspace_bytes(B, N_q, H, D) bytes, 256-byte aligned: an fp32
+ *     dQ accumulator and rowsum(dO * O).  The library allocates nothing.
+ * Four kernels run in order on `stream`.  Returns FA_ERR_ARG /
+ * FA_ERR_UNSUPPORTED (FA_E4M3, other head dims) / FA_ERR_ALIGN (16-byte
+ * aligned tensors, 4-byte aligned lse) before any GPU work, FA_ERR_CUDA on a
+ * launch failure, else FA_OK; waits that time out are reported by
+ * fa_device_status().  fa_bwd_workspace_bytes returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int N_q, int H, int D);
+int fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int D,
+           float scale, int causal, int window_left, int dtype, void* workspace,
+           size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * device status word that kernels set when a wait times out.  Returns FA_OK,
  * FA_ERR_TIMEOUT (and the raw flag bits in *flags when flags != NULL) or

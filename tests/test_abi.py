@@ -149,3 +149,41 @@ def test_mask_arguments_validated(kind, mask, sb, sh, sq):
     f = _lib.lib().fa_fwd_mask
     assert f(A, A, A, A, None, 1, 16, 128, 4, 4, 128, 0.1, 0, -1, _lib.FA_BF16, 1.0, 1.0, 1.0, mask, kind, sb, sh,
              sq, None) == _lib.FA_ERR_ARG
+
+
+def test_backward_workspace_size():
+    f = _lib.lib().fa_bwd_workspace_bytes
+    # fp32 dQ accumulator [B, N_q, H, D] plus the row term [B, H, N_q]
+    assert f(2, 300, 4, 128) == 2 * 300 * 4 * 129 * 4
+    assert f(1, 0, 1, 64) == 0
+    assert f(0, 10, 1, 64) == 0 and f(1, 10, 1, 96) == 0
+
+
+def _bwd(**kw):
+    args = dict(q=A, k=A, v=A, out=A, dout=A, lse=A, dq=A, dk=A, dv=A, B=1, N_q=16, N_k=16, H=2, D=64,
+                scale=0.125, causal=0, window_left=-1, dtype=_lib.FA_FP16, ws=A, nbytes=1 << 20)
+    args.update(kw)
+    return _lib.lib().fa_bwd(args["q"], args["k"], args["v"], args["out"], args["dout"], args["lse"], args["dq"],
+                             args["dk"], args["dv"], args["B"], args["N_q"], args["N_k"], args["H"], args["D"],
+                             args["scale"], args["causal"], args["window_left"], args["dtype"], args["ws"],
+                             args["nbytes"], None)
+
+
+@pytest.mark.parametrize("kw, expect", [
+    (dict(dtype=_lib.FA_E4M3, D=128), _lib.FA_ERR_UNSUPPORTED),
+    (dict(D=96), _lib.FA_ERR_UNSUPPORTED),
+    (dict(dout=None), _lib.FA_ERR_ARG),
+    (dict(lse=None), _lib.FA_ERR_ARG),
+    (dict(dq=None), _lib.FA_ERR_ARG),
+    (dict(dk=None), _lib.FA_ERR_ARG),
+    (dict(ws=None), _lib.FA_ERR_ARG),
+    (dict(nbytes=100), _lib.FA_ERR_ARG),
+    (dict(ws=A + 16), _lib.FA_ERR_ARG),
+    (dict(dq=A + 8), _lib.FA_ERR_ALIGN),
+    (dict(lse=A + 2), _lib.FA_ERR_ALIGN),
+    (dict(scale=0.0), _lib.FA_ERR_ARG),
+    (dict(window_left=-2), _lib.FA_ERR_ARG),
+])
+def test_backward_arguments_validated(kw, expect):
+    """Backward arguments are checked on the host, before any GPU work."""
+    assert _bwd(**kw) == expect

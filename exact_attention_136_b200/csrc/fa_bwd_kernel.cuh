@@ -133,13 +133,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   }
   BwdHeader* sh = reinterpret_cast<BwdHeader*>(smem);
   const int warp = threadIdx.x / 32;
-  // longest first: for causal attention key block 0 is seen by every query block
-  const int bh_count = p.B * p.H;
-  const int jk = static_cast<int>(blockIdx.x) / bh_count;
-  const int bh = static_cast<int>(blockIdx.x) - jk * bh_count;
+  // Head-major: the CTAs in flight are the key blocks of one or two heads,
+  // so that head's Q, dO and dQ accumulator stay in L2 (longest first inside
+  // a head: for causal attention key block 0 is seen by every query block).
+  const int jk = static_cast<int>(blockIdx.x) % p.nkb;
+  const int bh = static_cast<int>(blockIdx.x) / p.nkb;
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   int i_lo, i_hi;
   bwd_query_range(jk, p, i_lo, i_hi);
+  // The n-th query block a CTA visits is i_lo + (n + rot) mod cnt: causal
+  // CTAs already start at their own diagonal; the others start at a block
+  // of their own, so CTAs running side by side add into different dQ rows.
+  const int cnt = i_hi - i_lo + 1;
+  const int rot = (p.causal || cnt <= 0) ? 0 : jk % cnt;
   const uint64_t lim = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -186,7 +192,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                          pol_kv);
       }
       int n = 0;
-      for (int i = i_lo; i <= i_hi; ++i, ++n) {
+      for (; n < cnt; ++n) {
+        const int i = i_lo + (n + rot) % cnt;
         const int s = n & 1;
         if (!mbar_wait(smem_u32(&sh->st_empty[s]), ((n >> 1) & 1) ^ 1, lim)) {
           bwd_error(sh, p, ST_TIMEOUT_LOAD);
@@ -222,8 +229,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const uint32_t ds_mn = sdesc_sw128_lo(sbase + C::OFF_DS, C::CHUNK);
       const uint32_t ds_kmaj = sdesc_sw128_lo(sbase + C::OFF_DS, 16);
       bool ok = mbar_wait(smem_u32(&sh->kv_full), 0, lim);
-      int n = 0;
-      for (int i = i_lo; i <= i_hi && ok; ++i, ++n) {
+      for (int n = 0; n < cnt && ok; ++n) {
         const int s = n & 1;
         const uint32_t q_tile = sbase + C::OFF_STAGE + s * 2 * C::TILE;
         const uint32_t do_tile = q_tile + C::TILE;
@@ -297,8 +303,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const long long bhq = static_cast<long long>(bh) * p.Nq;
     bool ok = true;
     bool dq_ok = true;   // the previous block's dQ wait (reported at the next vote)
-    int n = 0;
-    for (int i = i_lo; i <= i_hi; ++i, ++n) {
+    for (int n = 0; n < cnt; ++n) {
+      const int i = i_lo + (n + rot) % cnt;
       const int buf = n & 1;
       // row statistics of query block i (one value per thread); the vote
       // below is also the barrier that publishes them

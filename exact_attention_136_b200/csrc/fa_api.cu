@@ -317,11 +317,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dout, co
                cudaStream_t stream, DeviceState* ds, int bit) {
   using C = BwdCfg<D>;
   const CUtensorMapDataType tdt = DT == DT_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (encode_bnhd(&mq, q, tdt, 2, p.B, p.Nq, p.H, D, 64, 128) ||
       encode_bnhd(&mk, k, tdt, 2, p.B, p.Nk, p.H, D, 64, 128) ||
       encode_bnhd(&mv, v, tdt, 2, p.B, p.Nk, p.H, D, 64, 128) ||
-      encode_bnhd(&mdo, dout, tdt, 2, p.B, p.Nq, p.H, D, 64, 128))
+      encode_bnhd(&mdo, dout, tdt, 2, p.B, p.Nq, p.H, D, 64, 128) ||
+      encode_bnhd(&mdq, p.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.Nq, p.H, D, 32, 128))
     return FA_ERR_CUDA;
   if (!(ds->attr_set & (1u << bit))) {
     if (cudaFuncSetAttribute(fa_bwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
@@ -331,7 +332,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dout, co
   }
   const int64_t grid = static_cast<int64_t>(p.nkb) * p.B * p.H;
   if (grid > 0x7fffffff) return FA_ERR_ARG;
-  fa_bwd_kernel<D, DT><<<static_cast<int>(grid), BWD_THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+  fa_bwd_kernel<D, DT><<<static_cast<int>(grid), BWD_THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, mdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

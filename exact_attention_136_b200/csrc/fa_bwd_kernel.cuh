@@ -13,7 +13,9 @@
 // One CTA per (batch, head, 128-key block): K_j and V_j stay in shared
 // memory and dK_j, dV_j accumulate in tensor memory over the query blocks
 // that see the keys; dQ is a sum over key blocks, so every CTA adds its
-// share into an fp32 buffer with vector reductions (red.global.add.v4.f32).
+// share into an fp32 buffer: the gradient warps stage it through shared
+// memory in 128-byte lines and the TMA adds the boxes into global memory
+// (cp.reduce.async.bulk.tensor .add).
 //
 // Everything is computed transposed (keys on the TMEM lanes).  P^T, written
 // back into tensor memory over S^T by the gradient warps (after each has
@@ -69,7 +71,8 @@ struct BwdHeader {
   uint64_t kv_full;
   uint64_t st_full[2], st_empty[2];   // (Q_i, dO_i) stages
   uint64_t s_full, dp_full;           // S^T, dP^T computed
-  uint64_t grad_ready;                // P^T in TMEM, dS^T in shared memory
+  uint64_t p_ready;                   // P^T in TMEM
+  uint64_t ds_ready;                  // dS^T in shared memory
   uint64_t dq_full, dq_empty;         // dQ partial computed / read out
   uint64_t dkv_full;                  // every MMA of the CTA done
   uint32_t tmem_base;
@@ -101,10 +104,21 @@ __device__ __forceinline__ bool grad_bar_and(bool v) {
   return r != 0u;
 }
 
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+// Bulk tensor reduce-add (TMA) of a shared-memory box into global memory,
+// and the bulk-group bookkeeping around it.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2,
+                                                  int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          map),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
 }
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of every committed bulk operation have been read
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and the operations have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Query blocks that see key block jk: causal keeps queries at or after the
 // key (absolute indices), a left window keeps queries at most window_left
@@ -124,7 +138,7 @@ template <int D, int DT>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {
@@ -156,7 +170,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     mbar_init(smem_u32(&sh->s_full), 1);
     mbar_init(smem_u32(&sh->dp_full), 1);
-    mbar_init(smem_u32(&sh->grad_ready), 256);
+    mbar_init(smem_u32(&sh->p_ready), 256);
+    mbar_init(smem_u32(&sh->ds_ready), 256);
     mbar_init(smem_u32(&sh->dq_full), 1);
     mbar_init(smem_u32(&sh->dq_empty), 256);
     mbar_init(smem_u32(&sh->dkv_full), 1);
@@ -166,6 +181,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
     tma_prefetch_map(&tm_do);
+    tma_prefetch_map(&tm_dq);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&sh->tmem_base), 512);
@@ -228,16 +244,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const uint32_t k_mn = sdesc_sw128_lo(sbase + C::OFF_K, C::CHUNK);
       const uint32_t ds_mn = sdesc_sw128_lo(sbase + C::OFF_DS, C::CHUNK);
       const uint32_t ds_kmaj = sdesc_sw128_lo(sbase + C::OFF_DS, 16);
-      bool ok = mbar_wait(smem_u32(&sh->kv_full), 0, lim);
-      for (int n = 0; n < cnt && ok; ++n) {
-        const int s = n & 1;
-        const uint32_t q_tile = sbase + C::OFF_STAGE + s * 2 * C::TILE;
-        const uint32_t do_tile = q_tile + C::TILE;
-        ok = mbar_wait(smem_u32(&sh->st_full[s]), (n >> 1) & 1, lim);
-        if (!ok) break;
-        tc_fence_after();
-        // S^T = K Q_i^T and dP^T = V dO_i^T (keys on the lanes, 128 queries wide)
-        const uint32_t q_kmaj = sdesc_sw128_lo(q_tile, 16), do_kmaj = sdesc_sw128_lo(do_tile, 16);
+      // S^T = K Q_n^T for the n-th query block (keys on the lanes)
+      auto issue_st = [&](int n) {
+        const uint32_t q_kmaj = sdesc_sw128_lo(sbase + C::OFF_STAGE + (n & 1) * 2 * C::TILE, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int byte = kk * 32;
@@ -245,11 +254,28 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_f16_ss_lo(tbase + C::S_COL, k_kmaj + off, q_kmaj + off, HI, ID_ST, kk > 0);
         }
         mma_commit(smem_u32(&sh->s_full));
+      };
+      // Per query block n: dP^T(n), then on P^T(n): dV(n) and the next
+      // block's S^T (which overwrites S^T(n) under P^T(n), after dV(n) has
+      // read it), then on dS^T(n): dK(n) and dQ(n).  So dV(n) and S^T(n+1)
+      // run while the gradient warps form dS, and dP^T(n+1) while they
+      // compute P(n+1).
+      bool ok = mbar_wait(smem_u32(&sh->kv_full), 0, lim) && mbar_wait(smem_u32(&sh->st_full[0]), 0, lim);
+      if (ok) {
+        tc_fence_after();
+        issue_st(0);
+      }
+      for (int n = 0; n < cnt && ok; ++n) {
+        const int s = n & 1;
+        const uint32_t q_tile = sbase + C::OFF_STAGE + s * 2 * C::TILE;
+        const uint32_t do_tile = q_tile + C::TILE;
         // (D = 128: dP^T's columns hold the previous block's dQ until it is read out)
         if (C::SERIAL_DQ && n > 0 && !mbar_wait(smem_u32(&sh->dq_empty), (n - 1) & 1, lim)) {
           ok = false;
           break;
         }
+        tc_fence_after();
+        const uint32_t do_kmaj = sdesc_sw128_lo(do_tile, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int byte = kk * 32;
@@ -257,26 +283,32 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_f16_ss_lo(tbase + C::DP_COL, v_kmaj + off, do_kmaj + off, HI, ID_ST, kk > 0);
         }
         mma_commit(smem_u32(&sh->dp_full));
-        if (!mbar_wait(smem_u32(&sh->grad_ready), n & 1, lim)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&sh->p_ready), n & 1, lim)) { ok = false; break; }
         tc_fence_after();
-        // dV += P^T dO_i (A from TMEM: 16 queries = 8 columns per step), dK += dS^T Q_i
+        // dV += P^T dO_n (A from TMEM: 16 queries = 8 columns per step)
         const uint32_t q_mn = sdesc_sw128_lo(q_tile, C::CHUNK), do_mn = sdesc_sw128_lo(do_tile, C::CHUNK);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
           mma_f16_ts_lo(tbase + C::DV_COL, tbase + C::P_COL + kk * 8, do_mn + off, HI, ID_KV, n > 0 || kk > 0);
         }
+        if (n + 1 < cnt) {
+          if (!mbar_wait(smem_u32(&sh->st_full[(n + 1) & 1]), ((n + 1) >> 1) & 1, lim)) { ok = false; break; }
+          tc_fence_after();
+          issue_st(n + 1);
+        }
+        if (!mbar_wait(smem_u32(&sh->ds_ready), n & 1, lim)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          // A = dS^T in shared memory, K-major: 16 queries = 32 bytes of a row
+          // dK += dS^T Q_n: A = dS^T in shared memory, K-major (16 queries = 32 bytes of a row)
           const int byte = kk * 32;
           const uint32_t a_off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
           const uint32_t b_off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
           mma_f16_ss_lo(tbase + C::DK_COL, ds_kmaj + a_off, q_mn + b_off, HI, ID_KV, n > 0 || kk > 0);
         }
-        mma_commit(smem_u32(&sh->st_empty[s]));   // last readers of Q_i and dO_i
-        // dQ_i (partial) = dS K_j: A = dS^T in shared memory read query-major,
-        // B = K_j read head-dim-major; 16 keys per step
+        mma_commit(smem_u32(&sh->st_empty[s]));   // last readers of Q_n and dO_n
+        // dQ_n (partial) = dS K_j: A = dS^T read query-major, B = K_j head-dim-major
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
@@ -324,8 +356,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int q0 = i * 128;
       const bool need_mask = (jk * 128 + 128 > p.Nk) || (p.causal && jk * 128 + 127 > q0) ||
                              (p.window_left >= 0 && jk * 128 < q0 + 127 - p.window_left);
-      // (S^T was committed before dP^T)
-      const bool got = mbar_wait(smem_u32(&sh->dp_full), n & 1, lim) && mbar_wait(smem_u32(&sh->s_full), n & 1, lim);
+      const bool got = mbar_wait(smem_u32(&sh->s_full), n & 1, lim);
       if (!grad_bar_and(got && dq_ok)) {
         ok = false;
         break;
@@ -355,6 +386,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int e = 0; e < 16; ++e) pw[e] = pack2<DT>(pv[c * 32 + 2 * e], pv[c * 32 + 2 * e + 1]);
         tmem_st_16x32bx2_x16<32>(tbase + lane_off + C::P_COL + c * 16, pw);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sh->p_ready));
+      // dP^T(n) (committed after S^T(n); a wait that times out leaves dS
+      // unusable, which the next vote reports)
+      dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim)) && dq_ok;
+      tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         // dS^T for queries half * 64 + [16c, 16c + 16)
@@ -375,32 +413,52 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         *reinterpret_cast<uint4*>(ds_row + u0 * 16) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
         *reinterpret_cast<uint4*>(ds_row + u1 * 16) = make_uint4(dw[4], dw[5], dw[6], dw[7]);
       }
-      tmem_wait_st();
       fence_proxy_async_smem();   // dS^T stores visible to the MMA's reads
       tc_fence_before();
-      mbar_arrive(smem_u32(&sh->grad_ready));
-      // dQ_i partial (queries on the lanes): add scale * dS K into dq_acc
-      dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dq_full), n & 1, lim));
-      if (dq_ok) {
-        tc_fence_after();
-        const int q = q0 + r;
-        float* dst = p.dq_acc + ((static_cast<long long>(b) * p.Nq + q) * p.H + h) * D + half * (D / 2);
+      mbar_arrive(smem_u32(&sh->ds_ready));
+      // dQ_i partial (queries on the lanes), staged as scale * dQ through the
+      // dS buffer (its readers, the dK and dQ MMAs, have completed) in boxes
+      // of 32 columns x 128 rows, 128-byte swizzled, and added into dq_acc by
+      // the TMA; rows past N_q are clipped by the map.  Thread (r, half)
+      // holds columns half * D/2 + [0, D/2): round k stages columns
+      // half * D/2 + 32k + [0, 32) as box `half`.  The TMEM columns are
+      // released once the last round's values are in registers.
+      dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dq_full), n & 1, lim)) && dq_ok;
+      tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[16];
-          tmem_ld_16x32bx2_x16<D / 2>(tbase + lane_off + C::DQ_COL + c * 16, v);
-          tmem_wait_ld();
-          if (q < p.Nq) {
+      for (int k = 0; k < D / 64; ++k) {
+        uint8_t* box_row = smem + C::OFF_DS + half * (32 * 128 * 4) + r * 128;
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              red_add_v4(dst + c * 16 + e, p.scale * __uint_as_float(v[e]), p.scale * __uint_as_float(v[e + 1]),
-                         p.scale * __uint_as_float(v[e + 2]), p.scale * __uint_as_float(v[e + 3]));
+        for (int cc = 0; cc < 2; ++cc) {
+          float dqv[16];
+          if (dq_ok) {
+            tmem_ld_16x32bx2_x16<D / 2>(tbase + lane_off + C::DQ_COL + 32 * k + 16 * cc,
+                                        reinterpret_cast<uint32_t*>(dqv));
+            tmem_wait_ld();
           }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<float4*>(box_row + (((4 * cc + u) ^ (r & 7)) * 16)) =
+                make_float4(p.scale * dqv[4 * u], p.scale * dqv[4 * u + 1], p.scale * dqv[4 * u + 2],
+                            p.scale * dqv[4 * u + 3]);
         }
-        tc_fence_before();
+        if (k == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(smem_u32(&sh->dq_empty));
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (t == 0) {
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb)
+            tma_reduce_add_4d(&tm_dq, sbase + C::OFF_DS + hb * (32 * 128 * 4), hb * (D / 2) + 32 * k, h, q0, b);
+          bulk_commit_group();
+          bulk_wait_read_all();   // the buffer may be written again
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
       }
-      mbar_arrive(smem_u32(&sh->dq_empty));
     }
+    if (t == 0) bulk_wait_all();   // every reduction has landed before the CTA exits
     if (!grad_bar_and(ok && dq_ok)) {
       ok = false;
       if (threadIdx.x == 128) bwd_error(sh, p, ST_TIMEOUT_SOFTMAX);

@@ -3,6 +3,7 @@
     from exact_attention_136_b200 import forward, backward
     out, lse = forward(q, k, v, causal=True)      # [batch, seqlen, heads, headdim]
     dq, dk, dv = backward(q, k, v, out, lse, dout, causal=True)
+    out = flash_attn_func(q, k, v, causal=True)  # the pages' call, with autograd
 
 The computation runs in libfa_b200.so (hand-written sm_100a CUDA, C ABI in
 include/fa.h); this package only marshals arguments.
@@ -10,6 +11,7 @@ include/fa.h); this package only marshals arguments.
 
 from .api import (auto_splits, backward, device_status, forward, forward_fp8, forward_host, set_wait_limit_ns,
                   wait_probe)
+from .interface import flash_attn_func
 
-__all__ = ["forward", "forward_fp8", "forward_host", "backward", "auto_splits", "device_status",
+__all__ = ["forward", "forward_fp8", "forward_host", "backward", "flash_attn_func", "auto_splits", "device_status",
            "set_wait_limit_ns", "wait_probe"]

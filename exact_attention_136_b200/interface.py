@@ -1,0 +1,78 @@
+"""The pages' call, ``flash_attn_func``, over this library, with autograd.
+
+Flash Attention | Hermes Skill, Workflow 2, Step 2 calls
+``flash_attn_func(q, k, v, dropout_p=0.0, causal=...)`` on
+``[batch, seqlen, nheads, headdim]`` tensors, and Step 3 adds
+``window_size=(left, right)`` and K/V with fewer heads; the default softmax
+scale is 1/sqrt(headdim) (the page's "auto-scale").  This module gives that
+call, backed by ``forward`` and ``backward`` (argument marshalling only: the
+computation is libfa_b200.so's), so code written against the pages' call can
+switch to this library and train through it.
+
+Readings (the pages leave these open):
+- ``window_size=(left, right)``: ``left`` is the window before the query
+  (-1 = unlimited); with ``causal=True`` the right window is zero whatever
+  ``right`` says (the page pairs causal=True with a two-sided window, which
+  contradict each other; causal wins).  Without causal only ``right = -1``
+  (no right bound) is available.
+- ``dropout_p`` must be 0: the pages give no random-number specification for
+  dropout, and this library does not implement it.
+- The backward takes fp16 / bf16 inputs with as many K/V heads as query heads.
+"""
+
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from .api import backward, forward
+
+
+def _window_left(causal: bool, window_size: Tuple[int, int]) -> int:
+    left, right = (int(window_size[0]), int(window_size[1]))
+    if left < -1 or right < -1:
+        raise ValueError("window_size entries are -1 (unlimited) or >= 0")
+    if not causal and right != -1:
+        raise NotImplementedError("a right window without causal=True is not supported (only left windows)")
+    return left
+
+
+class _FlashAttn(torch.autograd.Function):
+    """O = attention(q, k, v); the backward recomputes from O and the LSE."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale, causal, window_left):
+        out, lse = forward(q, k, v, scale, causal, window_left)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.scale, ctx.causal, ctx.window_left = scale, causal, window_left
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, dlse):
+        if dlse is not None and bool(torch.any(dlse != 0)):
+            raise NotImplementedError("gradients through the returned LSE are not supported")
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left)
+        return dq, dk, dv, None, None, None
+
+
+def flash_attn_func(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dropout_p: float = 0.0,
+                    softmax_scale: Optional[float] = None, causal: bool = False,
+                    window_size: Tuple[int, int] = (-1, -1), return_lse: bool = False):
+    """The pages' flash_attn_func on [batch, seqlen, nheads, headdim] tensors.
+
+    Returns O (and LSE [batch, nheads, seqlen_q], natural log, with
+    return_lse).  Differentiable in q, k, v (fp16 / bf16, equal head counts).
+    """
+    if dropout_p != 0.0:
+        raise NotImplementedError("dropout_p must be 0: no dropout (the pages specify no random generator)")
+    wl = _window_left(bool(causal), window_size)
+    scale = float(softmax_scale) if softmax_scale is not None else q.shape[-1] ** -0.5
+    needs_grad = torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v))
+    if needs_grad:
+        out, lse = _FlashAttn.apply(q, k, v, scale, bool(causal), wl)
+    else:
+        out, lse = forward(q, k, v, scale, bool(causal), wl)
+    return (out, lse) if return_lse else out

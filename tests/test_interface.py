@@ -1,0 +1,91 @@
+"""flash_attn_func (the pages' call) on the CPU: its argument handling and
+autograd plumbing, with the library's forward / backward replaced by the
+fp64 oracle (the GPU entry points themselves are covered by the GPU tests)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_136_b200.interface as itf
+from oracle import attention_backward_ref, attention_ref
+
+
+@pytest.fixture
+def oracle_backend(monkeypatch):
+    calls = []
+
+    def fwd(q, k, v, scale, causal, window_left):
+        calls.append(("fwd", scale, causal, window_left))
+        o, l = attention_ref(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), scale, causal, window_left)
+        return torch.from_numpy(o), torch.from_numpy(l)
+
+    def bwd(q, k, v, out, lse, dout, scale, causal, window_left):
+        calls.append(("bwd", scale, causal, window_left))
+        g = attention_backward_ref(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), dout.numpy(), scale,
+                                   causal, window_left)
+        return tuple(torch.from_numpy(x) for x in g)
+
+    monkeypatch.setattr(itf, "forward", fwd)
+    monkeypatch.setattr(itf, "backward", bwd)
+    return calls
+
+
+def _plain_attention(q, k, v, scale, causal, wl):
+    """Softmax attention with torch ops, [B, N, H, D] (torch autograd differentiates it)."""
+    s = torch.einsum("bihd,bjhd->bhij", q, k) * scale
+    n_q, n_k = q.shape[1], k.shape[1]
+    i = torch.arange(n_q)[:, None]
+    j = torch.arange(n_k)[None, :]
+    vis = torch.ones(n_q, n_k, dtype=torch.bool)
+    if causal:
+        vis &= j <= i
+    if wl >= 0:
+        vis &= j >= i - wl
+    s = s.masked_fill(~vis, float("-inf"))
+    return torch.einsum("bhij,bjhd->bihd", torch.softmax(s, dim=-1), v)
+
+
+@pytest.mark.parametrize("causal, window", [(False, (-1, -1)), (True, (-1, -1)), (True, (3, 3)), (False, (2, -1))])
+def test_gradients_match_torch_autograd(oracle_backend, causal, window):
+    g = torch.Generator().manual_seed(7)
+    q, k, v = (torch.randn(1, 9, 2, 4, generator=g, dtype=torch.float64, requires_grad=True) for _ in range(3))
+    do = torch.randn(1, 9, 2, 4, generator=g, dtype=torch.float64)
+    out = itf.flash_attn_func(q, k, v, causal=causal, window_size=window)
+    out.backward(do)
+    wl = window[0]
+    q2, k2, v2 = (t.detach().clone().requires_grad_() for t in (q, k, v))
+    ref = _plain_attention(q2, k2, v2, 0.5, causal, wl)   # default scale 1/sqrt(4)
+    ref.backward(do)
+    assert torch.allclose(out, ref, atol=1e-12)
+    for a, b in ((q.grad, q2.grad), (k.grad, k2.grad), (v.grad, v2.grad)):
+        assert torch.allclose(a, b, atol=1e-12)
+    # scale, causal and window reach the library unchanged, forward then backward
+    assert oracle_backend == [("fwd", 0.5, causal, wl), ("bwd", 0.5, causal, wl)]
+
+
+def test_no_grad_path_and_lse(oracle_backend):
+    q, k, v = (torch.randn(1, 5, 1, 8, dtype=torch.float64) for _ in range(3))
+    out, lse = itf.flash_attn_func(q, k, v, softmax_scale=0.3, causal=True, return_lse=True)
+    o, l = attention_ref(q.numpy(), k.numpy(), v.numpy(), 0.3, True, -1)
+    assert np.allclose(out.numpy(), o) and np.allclose(lse.numpy(), l)
+    assert oracle_backend == [("fwd", 0.3, True, -1)]   # no autograd record without requires_grad
+
+
+def test_rejected_arguments(oracle_backend):
+    q = torch.zeros(1, 4, 1, 8, dtype=torch.float64)
+    with pytest.raises(NotImplementedError):
+        itf.flash_attn_func(q, q, q, dropout_p=0.1)
+    with pytest.raises(NotImplementedError):
+        itf.flash_attn_func(q, q, q, causal=False, window_size=(2, 2))
+    with pytest.raises(ValueError):
+        itf.flash_attn_func(q, q, q, window_size=(-2, -1))
+    assert oracle_backend == []
+
+
+def test_causal_two_sided_window_reads_as_left_window(oracle_backend):
+    # the pages pair causal=True with window_size=(256, 256); causal wins on the right
+    q = torch.zeros(1, 4, 1, 8, dtype=torch.float64)
+    itf.flash_attn_func(q, q, q, causal=True, window_size=(256, 256))
+    assert oracle_backend == [("fwd", 8 ** -0.5, True, 256)]

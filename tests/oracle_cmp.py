@@ -68,7 +68,7 @@ def compare(out, lse, ref_o, ref_l, rows=None):
 def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, unit_roundoff):
     """Per-element bounds (dq, dk, dv; shaped like q, k, v) on how far a
     backward computed the way the CUDA path does can be from the exact
-    gradients, all arrays float64 numpy, K/V heads equal to query heads.
+    gradients, all arrays float64 numpy.
 
     The path recomputes P = exp(scale q.k - LSE) in fp32 from the forward's
     LSE (relative error e1 <= |LSE_used - LSE| + 1e-6), takes the row term
@@ -81,28 +81,32 @@ def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, u
         |d dS_ik| <= (u + e1)(1 + u) |dS_ik| + (1 + u) P_ik eD_i
         |d dK_kd| <= scale sum_i |d dS_ik| |Q_id|,  |d dQ_id| <= scale sum_k |d dS_ik| |K_kd|
     each plus 1e-5 of the matching sum of absolute products (fp32 sums).
+    With fewer K/V heads than query heads (query head h reads K/V head
+    h // (H / H_kv)) the dK and dV bounds add up over each group's heads.
     """
     from oracle import attention_ref
     u = float(unit_roundoff)
     B, n_q, H, D = q.shape
-    n_k = k.shape[1]
+    n_k, h_kv = k.shape[1], k.shape[2]
+    group = H // h_kv
     bq, bk, bv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
     o_ref, l_ref, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True)
     for b in range(B):
         for h in range(H):
+            hk = h // group
             p = probs[b, h]
             g = do[b, :, h, :]
-            vv = v[b, :, h, :]
+            vv = v[b, :, hk, :]
             qq = q[b, :, h, :]
-            kk = k[b, :, h, :]
+            kk = k[b, :, hk, :]
             dp = g @ vv.T
             ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
             l_diff = np.where(np.isfinite(l_ref[b, h]), np.abs(lse_used[b, h] - l_ref[b, h]), 0.0)
             e1 = (1.01 * l_diff + 1e-6)[:, None]                       # per query row
             e_d = (np.abs(g) * np.abs(o_used[b, :, h, :] - o_ref[b, :, h, :])).sum(axis=1) + \
                 1e-6 * np.abs(g * o_ref[b, :, h, :]).sum(axis=1)
-            bv[b, :, h, :] = ((u + e1) * p).T @ np.abs(g) + 1e-5 * p.T @ np.abs(g)
+            bv[b, :, hk, :] += ((u + e1) * p).T @ np.abs(g) + 1e-5 * p.T @ np.abs(g)
             d_ds = (u + e1) * (1 + u) * np.abs(ds) + (1 + u) * p * e_d[:, None]
-            bk[b, :, h, :] = scale * (d_ds.T @ np.abs(qq) + 1e-5 * np.abs(ds).T @ np.abs(qq))
+            bk[b, :, hk, :] += scale * (d_ds.T @ np.abs(qq) + 1e-5 * np.abs(ds).T @ np.abs(qq))
             bq[b, :, h, :] = scale * (d_ds @ np.abs(kk) + 1e-5 * np.abs(ds) @ np.abs(kk))
     return bq, bk, bv

@@ -18,22 +18,25 @@ def _emulated_backward(q, k, v, do, o_used, scale, causal, dt):
     rnd = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(tdt).double().numpy()
     _, _, probs = attention_ref(q, k, v, scale, causal, -1, return_probs=True)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    group = q.shape[2] // k.shape[2]
     for h in range(q.shape[2]):
+        hk = h // group
         p = probs[0, h]
         g = do[0, :, h]
         delta = (g * o_used[0, :, h]).sum(axis=1)
-        ds = p * (g @ v[0, :, h].T - delta[:, None])
-        dv[0, :, h] = rnd(p).T @ g
-        dk[0, :, h] = scale * rnd(ds).T @ q[0, :, h]
-        dq[0, :, h] = scale * rnd(ds) @ k[0, :, h]
+        ds = p * (g @ v[0, :, hk].T - delta[:, None])
+        dv[0, :, hk] += rnd(p).T @ g
+        dk[0, :, hk] += scale * rnd(ds).T @ q[0, :, h]
+        dq[0, :, h] = scale * rnd(ds) @ k[0, :, hk]
     return dq, dk, dv
 
 
 def test_backward_bounds_cover_emulated_rounding():
     from oracle import attention_backward_ref
     from tests.oracle_cmp import backward_bounds
-    for dt, u, causal in (("bf16", 2.0 ** -8, True), ("fp16", 2.0 ** -11, False)):
-        qkv = inputs.make_qkv(1, 200, 200, 2, 32, dt, seeds=(51, 52, 53))
+    for dt, u, causal, h_kv in (("bf16", 2.0 ** -8, True, 2), ("fp16", 2.0 ** -11, False, 2),
+                                ("bf16", 2.0 ** -8, True, 1)):
+        qkv = inputs.make_qkv(1, 200, 200, 2, 32, dt, seeds=(51, 52, 53), h_kv=h_kv)
         do = inputs.make_qkv(1, 200, 200, 2, 32, dt, seeds=(54, 55, 56)).q
         f = lambda t: t.double().numpy()
         q, k, v, g = f(qkv.q), f(qkv.k), f(qkv.v), f(do)

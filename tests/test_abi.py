@@ -187,3 +187,20 @@ def _bwd(**kw):
 def test_backward_arguments_validated(kw, expect):
     """Backward arguments are checked on the host, before any GPU work."""
     assert _bwd(**kw) == expect
+
+
+def _prototypes():
+    """{name: number of parameters} for every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?[\w\s\*]*?\b(fa_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.M | re.S):
+        params = m.group(2).strip()
+        protos[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_arities_match_the_header():
+    protos = _prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, count in protos.items():
+        assert len(_lib.SIGNATURES[name][1]) == count, name

@@ -204,3 +204,17 @@ def test_binding_arities_match_the_header():
     assert set(protos) == set(declared_functions())
     for name, count in protos.items():
         assert len(_lib.SIGNATURES[name][1]) == count, name
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/fa.h compiles as strict C99 (the ABI has no C++ in it)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_fa.c"
+    src.write_text('#include "fa.h"\nint main(void) { fa_stream_t s = 0; (void)s; return FA_OK; }\n')
+    res = subprocess.run([cc, "-std=c99", "-pedantic", "-Wall", "-Werror", "-fsyntax-only",
+                          "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr

@@ -218,3 +218,40 @@ def test_header_is_plain_c(tmp_path):
     res = subprocess.run([cc, "-std=c99", "-pedantic", "-Wall", "-Werror", "-fsyntax-only",
                           "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_c_program_links_and_calls(tmp_path):
+    """A plain C program links against libfa_b200.so and calls it: version and
+    status strings, and argument errors, which are answered before any GPU
+    work (so this runs without a GPU)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    src = tmp_path / "call_fa.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "fa.h"
+int main(void) {
+  static float buf[64];   /* a 16-byte-aligned dummy pointer; never dereferenced */
+  int bad_batch = fa_fwd(buf, buf, buf, buf, NULL, 0, 16, 16, 2, 64, 0.125f, 0, -1, FA_FP16, NULL);
+  int bad_dim = fa_fwd(buf, buf, buf, buf, NULL, 1, 16, 16, 2, 96, 0.125f, 0, -1, FA_FP16, NULL);
+  int bad_fp8 = fa_fwd_fp8(buf, buf, buf, buf, NULL, 1, 16, 16, 2, 128, 0.1f, 0, -1, 0.0f, 1.0f, 1.0f, NULL);
+  printf("%s|%d|%d|%d|%s\n", fa_version(), bad_batch, bad_dim, bad_fp8, fa_status_string(FA_ERR_ARG));
+  return 0;
+}
+""")
+    exe = tmp_path / "call_fa"
+    res = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                          "-L", lib_dir, "-lfa_b200", "-Wl,-rpath," + lib_dir], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    version, bad_batch, bad_dim, bad_fp8, msg = run.stdout.strip().split("|")
+    assert version and msg
+    assert int(bad_batch) == _lib.FA_ERR_ARG
+    assert int(bad_dim) == _lib.FA_ERR_UNSUPPORTED
+    assert int(bad_fp8) == _lib.FA_ERR_ARG   # zero descale

@@ -213,7 +213,8 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float
  *   workspace: caller-owned device memory of at least
  *     fa_bwd_workspace_bytes(B, N_q, H, D) bytes, 256-byte aligned: an fp32
  *     dQ accumulator and rowsum(dO * O).  The library allocates nothing.
- * Four kernels run in order on `stream`.  Returns FA_ERR_ARG /
+ * Three kernels run in order on `stream` (rowsum(dO * O) and a zeroed
+ * accumulator; dQ, dK, dV; dQ converted to 16-bit).  Returns FA_ERR_ARG /
  * FA_ERR_UNSUPPORTED (FA_E4M3, other head dims) / FA_ERR_ALIGN (16-byte
  * aligned tensors, 4-byte aligned lse) before any GPU work, FA_ERR_CUDA on a
  * launch failure, else FA_OK; waits that time out are reported by

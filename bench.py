@@ -52,8 +52,8 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_TFLOPS = {"fp16": 2250.0, "bf16": 2250.0, "e4m3": 4500.0}
 PROFILE_DIR = os.path.join(ROOT, "profiles")
+# the forward kernel and its host code (the backward's sources are not part of it)
 KERNEL_SOURCES = ["exact_attention_136_b200/csrc/fa_fwd_kernel.cuh", "exact_attention_136_b200/csrc/sm100.cuh",
-                  "exact_attention_136_b200/csrc/fa_bwd_kernel.cuh",
                   "exact_attention_136_b200/csrc/fa_api.cu", "exact_attention_136_b200/csrc/tmap.h"]
 
 
@@ -129,7 +129,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
@@ -206,21 +206,123 @@ def run_reference(args, world, rank):
     wall = time.perf_counter() - t_all
     per_row = 4.0 * w.n_k * w.D * W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left)
     value = per_row * total_rows / total_t / 1e12
-    # one full forward of the workload at this throughput
-    ms_per_step = W.flops(w) / (value * 1e12) * 1e3
     sample = (f"each step: fp64 oracle on {rows_per_step} sampled query rows of one (batch, head), "
               f"cycling over the {len(heads)} heads; {args.steps} steps took {wall:.1f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "desc": w.desc, "rows_per_step": rows_per_step,
-                   "ms_per_step_note": "one full forward of the workload at the sampled throughput"},
+                   "ms_per_step_note": "measured: one sampled step (the rows above), not a full forward"},
+        # one full forward of the workload at the sampled throughput (an extrapolation)
+        "full_forward_ms_extrapolated": W.flops(w) / (value * 1e12) * 1e3,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
     print(json.dumps(line), flush=True)
+
+
+MUFU_EXP_PER_CLK_PER_SM = 16   # ex2.approx results per clock per SM (B200 microbenchmark)
+# configurations measured beside the headline in every run (the other configurations
+# the target names), with the oracle rows per (batch, head) timed for each
+EXTRA_CONFIGS = [("pr1_b1h8n512d64_fp16", 512), ("b2h8n2048d64_fp16", 64),
+                 ("swa4096_b1h32n32768d128_bf16", 16), ("fp8_causal_b2h16n16384d128", 16)]
+
+
+def binding_roofline(w: W.Workload, sms: int, sm_max_mhz: float):
+    """(bound, peak TF/s, source) for a workload: the lower of the tensor-core
+    peak (measured bf16 burst; x2 for e4m3) and the exponential unit's: one
+    ex2 per score, MUFU_EXP_PER_CLK_PER_SM per SM per clock, 4 * D counted
+    FLOP per score (2 D for Q.K, 2 D for P.V), at the maximum SM clock."""
+    tensor, src, _ = measured_peaks(w.dtype)
+    mhz = sm_max_mhz or 1965.0
+    exp_peak = MUFU_EXP_PER_CLK_PER_SM * 4.0 * w.D * sms * mhz * 1e6 / 1e12
+    if exp_peak < tensor:
+        return "exp", exp_peak, (f"MUFU ex2 {MUFU_EXP_PER_CLK_PER_SM}/clk/SM x 4*D={4 * w.D} flop per score x "
+                                 f"{sms} SMs x {mhz:.0f} MHz")
+    return "tensor", tensor, f"{src} bf16 burst" + (" x2 for fp8" if w.dtype == "e4m3" else "")
+
+
+def clock_normalised(value, clocks):
+    """The value scaled to the maximum SM clock (value x max MHz / median MHz under load)."""
+    if not clocks or not clocks.get("sm_mhz") or not clocks.get("sm_max_mhz"):
+        return None
+    return value * clocks["sm_max_mhz"] / clocks["sm_mhz"]
+
+
+def timed(step, steps, dev, stream, local, barrier=lambda: None):
+    """CUDA-event milliseconds of `steps` calls of step() on `stream`, with the
+    SM clocks sampled while they run."""
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    return e0.elapsed_time(e1), sampler.stop()
+
+
+def make_step(w: W.Workload, qkv, q, k, v, out, lse, stream, splits, mask):
+    from exact_attention_136_b200 import forward, forward_fp8
+
+    def step():
+        if w.dtype == "e4m3":
+            forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, w.scale, w.causal, w.window_left,
+                        out=out, lse=lse, stream=stream, num_splits=splits, attn_mask=mask)
+        else:
+            forward(q, k, v, w.scale, w.causal, w.window_left, out=out, lse=lse, stream=stream, num_splits=splits,
+                    attn_mask=mask)
+    return step
+
+
+def device_tensors(w: W.Workload, seeds, dev):
+    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=seeds, h_kv=w.h_kv)
+    q, k, v = (t.pin_memory().to(dev) for t in (qkv.q, qkv.k, qkv.v))
+    out_dtype = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+    out = torch.empty((w.B, w.n_q, w.H, w.D), dtype=out_dtype, device=dev)
+    lse = torch.empty((w.B, w.H, w.n_q), dtype=torch.float32, device=dev)
+    return qkv, q, k, v, out, lse
+
+
+def measure_config(name, cpu_rows, dev, stream, local, sms, with_cpu):
+    """One more configuration: launches timed for about 0.1 s after 5 warm-ups,
+    its binding roofline, clocks, and the oracle on sampled rows."""
+    from exact_attention_136_b200 import device_status
+    w = W.WORKLOADS[name]
+    qkv, q, k, v, out, lse = device_tensors(w, w.seeds, dev)
+    step = make_step(w, qkv, q, k, v, out, lse, stream, w.splits, None)
+    for _ in range(5):
+        step()
+    ms_try, _ = timed(step, 3, dev, stream, local)
+    steps = int(min(2000, max(10, math.ceil(100.0 / max(ms_try / 3, 1e-3)))))
+    ms, clocks = timed(step, steps, dev, stream, local)
+    rc, flags = device_status(device=dev)
+    if rc != 0:
+        raise RuntimeError(f"{name}: device status {rc} flags {flags}")
+    if not bool(torch.isfinite(out).all()):
+        raise RuntimeError(f"{name}: non-finite output")
+    ms_launch = ms / steps
+    tf = W.flops(w) / (ms_launch / 1e3) / 1e12
+    bound, peak, src = binding_roofline(w, sms, (clocks or {}).get("sm_max_mhz"))
+    entry = {"desc": w.desc, "dtype": w.dtype, "launches": steps, "ms_per_launch": ms_launch,
+             "us_per_launch": ms_launch * 1e3, "tflops": tf, "flop_per_launch": W.flops(w),
+             "roofline": {"bound": bound, "peak": peak, "frac": tf / peak, "peak_source": src},
+             "pct_of_nominal_dense_peak": 100.0 * tf / NOMINAL_TFLOPS[w.dtype],
+             "clocks": clocks, "tflops_clock_normalised": clock_normalised(tf, clocks)}
+    if with_cpu:
+        ctf, cdt, n_rows, threads = oracle_rows_tflops(w, qkv, cpu_rows)
+        entry["cpu_oracle"] = {"tflops": ctf, "seconds": cdt, "rows": n_rows, "cores": threads,
+                               "rows_per_head": min(cpu_rows, w.n_q)}
+    del q, k, v, out, lse
+    return entry
 
 
 def main():
@@ -237,6 +339,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling cases)")
     ap.add_argument("--backward", action="store_true", help="time the backward (fa_bwd) instead of the forward")
+    ap.add_argument("--long-seconds", type=float, default=2.2,
+                    help="also time the workload for at least this long (sustained figure; 0 = skip)")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other configurations")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -246,7 +351,7 @@ def main():
         run_reference(args, world, rank)
         return
 
-    from exact_attention_136_b200 import _lib, device_status, forward, forward_fp8, forward_host
+    from exact_attention_136_b200 import _lib, device_status, forward_host
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -255,6 +360,7 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     lib = _lib.lib()  # loud failure when the CUDA library is missing
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     w = W.WORKLOADS[args.workload]
     if args.batch is not None:
@@ -264,25 +370,15 @@ def main():
         run_backward(args, w, world, rank, local, dev)
         return
     seeds = rank_seeds(w, rank)   # each rank: its own batch
-    qkv = inputs.make_qkv(w.B, w.n_q, w.n_k, w.H, w.D, w.dtype, seeds=seeds, h_kv=w.h_kv)
+    qkv, q, k, v, out, lse = device_tensors(w, seeds, dev)
     hq, hk, hv = qkv.q.pin_memory(), qkv.k.pin_memory(), qkv.v.pin_memory()
-    q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
-    out_dtype = torch.float16 if w.dtype == "fp16" else torch.bfloat16
-    out = torch.empty((w.B, w.n_q, w.H, w.D), dtype=out_dtype, device=dev)
-    lse = torch.empty((w.B, w.H, w.n_q), dtype=torch.float32, device=dev)
+    out_dtype = out.dtype
     stream = torch.cuda.current_stream(dev)
 
     splits = w.splits if args.splits is None else args.splits
     mask_cpu = W.make_mask(w)
     mask = mask_cpu.to(dev) if mask_cpu is not None else None
-
-    def step():
-        if w.dtype == "e4m3":
-            forward_fp8(q, k, v, qkv.q_descale, qkv.k_descale, qkv.v_descale, w.scale, w.causal, w.window_left,
-                        out=out, lse=lse, stream=stream, num_splits=splits, attn_mask=mask)
-        else:
-            forward(q, k, v, w.scale, w.causal, w.window_left, out=out, lse=lse, stream=stream, num_splits=splits,
-                    attn_mask=mask)
+    step = make_step(w, qkv, q, k, v, out, lse, stream, splits, mask)
 
     def barrier():
         if world > 1:
@@ -295,21 +391,8 @@ def main():
     if rc != 0:
         raise RuntimeError(f"device status {rc} flags {flags} after warm-up")
 
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    clocks = sampler.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    ms, clocks = timed(step, args.steps, dev, stream, local, barrier)
+    ms = max_over_ranks(ms, dev)
     rc, flags = device_status(device=dev)
     if rc != 0:
         raise RuntimeError(f"device status {rc} flags {flags} in the timed region")
@@ -320,6 +403,16 @@ def main():
     ms_per_step = ms / args.steps
     value = world * flops * args.steps / (ms / 1e3) / 1e12
     per_launch_tflops = flops / (ms_per_step / 1e3) / 1e12
+
+    # the same launches for a few seconds: what the kernel sustains under the power cap
+    long_run = None
+    if args.long_seconds > 0:
+        n_long = int(math.ceil(args.long_seconds * 1e3 / ms_per_step))
+        lms, lclocks = timed(step, n_long, dev, stream, local, barrier)
+        lms = max_over_ranks(lms, dev)
+        lval = world * flops * n_long / (lms / 1e3) / 1e12
+        long_run = {"launches": n_long, "seconds": lms / 1e3, "ms_per_step": lms / n_long, "value": lval,
+                    "clocks": lclocks, "value_clock_normalised": clock_normalised(lval, lclocks)}
 
     # end to end through the host-buffer entry point: H2D inputs, kernel, D2H out + lse
     ho = torch.empty((w.B, w.n_q, w.H, w.D), dtype=out_dtype, pin_memory=True)
@@ -359,6 +452,7 @@ def main():
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     peak, peak_src, sustained = measured_peaks(w.dtype)
+    bound, bpeak, bsrc = binding_roofline(w, sms, (clocks or {}).get("sm_max_mhz"))
     traffic = recorded_traffic(w.name)
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
 
@@ -369,6 +463,24 @@ def main():
                "sample": f"fp64 oracle on {args.cpu_rows} sampled query rows of each of the {w.B * w.H} "
                          f"(batch, head) pairs ({n_rows} rows, {dt:.1f} s); FLOP credited per row = "
                          f"the workload's average 4*N_k*D*block_fraction"}
+    del hq, hk, hv, ho, hl
+
+    # the other configurations, one after another on this GPU (rank 0 of a single-GPU run)
+    configs = None
+    if rank == 0 and world == 1 and not args.no_extras and args.batch is None:
+        del q, k, v, out, lse, staging, step
+        torch.cuda.empty_cache()
+        configs = {w.name: {"desc": w.desc, "dtype": w.dtype, "ms_per_launch": ms_per_step,
+                            "tflops": per_launch_tflops,
+                            "roofline": {"bound": bound, "peak": bpeak, "frac": per_launch_tflops / bpeak,
+                                         "peak_source": bsrc},
+                            "pct_of_nominal_dense_peak": 100.0 * per_launch_tflops / NOMINAL_TFLOPS[w.dtype],
+                            "clocks": clocks, "tflops_clock_normalised": clock_normalised(per_launch_tflops, clocks),
+                            "note": "the headline measurement above"}}
+        for name, rows in EXTRA_CONFIGS:
+            if name != w.name:
+                configs[name] = measure_config(name, rows, dev, stream, local, sms, not args.no_cpu_baseline)
+                torch.cuda.empty_cache()
 
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -379,8 +491,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "desc": w.desc, "B": w.B, "N_q": w.n_q, "N_k": w.n_k, "H": w.H,
-                   "H_kv": w.h_kv, "splits": splits, "mask": w.mask or None, "D": w.D, "causal": w.causal, "window_left": w.window_left, "scale": w.scale,
-                   "flop_per_step": flops,
+                   "H_kv": w.h_kv, "splits": splits, "mask": w.mask or None, "D": w.D, "causal": w.causal,
+                   "window_left": w.window_left, "scale": w.scale, "flop_per_step": flops,
                    "block_fraction": W.block_fraction(w.n_q, w.n_k, w.causal, w.window_left),
                    "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB vs {L2_BYTES / 1e6:.0f} MB), no flush",
                    "pct_of_nominal_dense_peak": 100.0 * per_launch_tflops / NOMINAL_TFLOPS[w.dtype],
@@ -390,10 +502,13 @@ def main():
                 "steps": args.e2e_steps,
                 "api": "fa_fwd_host (pinned host buffers)" if (w.h_kv == w.H and splits == 1 and mask is None)
                        else "pinned host copies + forward"},
-        "roofline": {"bound": "tensor", "achieved": per_launch_tflops, "peak": peak, "unit": UNIT,
-                     "frac": per_launch_tflops / peak, "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 burst" + (" x2 for fp8" if w.dtype == "e4m3" else ""),
-                     "peak_sustained": sustained},
+        "roofline": {"bound": bound, "achieved": per_launch_tflops, "peak": bpeak, "unit": UNIT,
+                     "frac": per_launch_tflops / bpeak, "traffic": traffic, "peak_source": bsrc,
+                     "tensor_peak": peak, "tensor_peak_source": f"{peak_src} bf16 burst" +
+                     (" x2 for fp8" if w.dtype == "e4m3" else ""), "peak_sustained": sustained},
+        "value_clock_normalised": clock_normalised(value, clocks),
+        "long_window": long_run,
+        "configs": configs,
         "cpu_baseline": cpu,
         "clocks": clocks,
         "gpu_launches": args.steps,
@@ -522,11 +637,10 @@ def run_backward(args, w, world, rank, local, dev):
         "roofline": {"bound": "tensor", "achieved": per_step_tflops, "peak": peak, "unit": UNIT,
                      "frac": per_step_tflops / peak, "traffic": None,
                      "peak_source": f"{peak_src} bf16 burst", "peak_sustained": sustained,
-                     "note": "achieved over the whole step (three kernels: row term, main, dQ conversion; "
-                             "the main kernel is ~95 % of it)"},
+                     "note": "achieved over the whole step (three kernels: row term, dK/dV, dQ)"},
         "cpu_baseline": cpu,
         "clocks": clocks,
-        "gpu_launches": 3 * args.steps,   # prologue, fa_bwd_kernel, epilogue per step
+        "gpu_launches": 3 * args.steps,   # row term, dK/dV kernel, dQ kernel per step
         "kernel_hash": kernel_hash(),
     }
     print(json.dumps(line), flush=True)

@@ -46,6 +46,8 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_c_int, _c_int, _c_int, _c_int]),
     "fa_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                         _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
+    "fa_bwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                            _c_int, _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
     "fa_device_status": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_wait_probe": (_c_int, [ctypes.c_ulonglong, _vp]),

@@ -56,29 +56,50 @@ def _outputs(q, B, n_q, H, D, out, lse, want_lse):
 
 def _mask_args(attn_mask: torch.Tensor, q: torch.Tensor, B: int, H: int, n_q: int, n_k: int):
     """attn_mask ([N_q, N_k] or [B or 1, H or 1, N_q, N_k]; bool = attend where True, float = added to
-    the scaled scores) as the library takes it: bytes or the output's 16-bit type, rows padded to
-    16 bytes, broadcast dimensions with stride 0.  Returns (buffer, kind, stride_b, stride_h, stride_q)."""
+    the scaled scores) as the library takes it: bytes or the output's 16-bit type, rows starting on
+    16-byte boundaries, broadcast dimensions with stride 0.  Like SDPA, a float mask must have the
+    inputs' type (the output's 16-bit type for FP8 inputs); no other float type is narrowed
+    silently.  A mask already in that form is passed as it is; otherwise it is copied into a
+    padded buffer.  Returns (buffer, kind, stride_b, stride_h, stride_q)."""
     m = attn_mask
     if m.dim() == 2:
         m = m[None, None]
     if (m.dim() != 4 or m.shape[2] != n_q or m.shape[3] != n_k or m.shape[0] not in (1, B)
             or m.shape[1] not in (1, H)):
         raise ValueError("attn_mask must be [N_q, N_k] or [B or 1, H or 1, N_q, N_k]")
+    out_dt = torch.float16 if q.dtype == torch.float16 else torch.bfloat16
     if m.dtype == torch.bool:
         kind, dt = _lib.FA_MASK_BOOL, torch.uint8
+    elif m.dtype == out_dt:
+        kind, dt = _lib.FA_MASK_ADD, out_dt
     else:
-        kind, dt = _lib.FA_MASK_ADD, (torch.float16 if q.dtype == torch.float16 else torch.bfloat16)
-    per = 16 // torch.empty((), dtype=dt).element_size()
+        raise ValueError(f"attn_mask must be bool or {out_dt} (the inputs' type), not {m.dtype}")
+    es = 1 if dt == torch.uint8 else 2
+    direct = m.view(torch.uint8) if m.dtype == torch.bool else m
+    # broadcast dimensions read with stride 0
+    strides = [direct.stride(i) if direct.shape[i] > 1 else 0 for i in range(4)]
+    if n_q == 1:
+        strides[2] = n_k
+    # passed as it is when its rows are whole 16-byte chunks on 16-byte boundaries
+    if (direct.device == q.device and (n_k * es) % 16 == 0 and direct.stride(3) == 1
+            and direct.data_ptr() % 16 == 0 and all((st * es) % 16 == 0 for st in strides[:3])
+            and strides[2] >= n_k):
+        return direct, kind, strides[0], strides[1], strides[2]
+    per = 16 // es
     n_pad = -(-n_k // per) * per
     buf = torch.zeros((m.shape[0], m.shape[1], n_q, n_pad), dtype=dt, device=q.device)
-    buf[..., :n_k] = m.to(device=q.device, dtype=dt)
+    buf[..., :n_k] = m.to(device=q.device).view(torch.uint8) if m.dtype == torch.bool else m.to(device=q.device)
     sb = buf.stride(0) if m.shape[0] > 1 else 0
     sh = buf.stride(1) if m.shape[1] > 1 else 0
     return buf, kind, sb, sh, buf.stride(2)
 
 
 def _masked(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, dt, descales, attn_mask, s):
-    buf, kind, sb, sh, sq = _mask_args(attn_mask, q, B, H, n_q, n_k)
+    # a padded copy of the mask is made on the launching stream (allocated
+    # there too), so the kernel reads it after the copy and its memory is not
+    # handed out again before the kernel has run
+    with torch.cuda.stream(s):
+        buf, kind, sb, sh, sq = _mask_args(attn_mask, q, B, H, n_q, n_k)
     rc = _lib.lib().fa_fwd_mask(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                 lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, h_kv, D, scale,
                                 int(bool(causal)), int(window_left), dt, float(descales[0]), float(descales[1]),
@@ -102,7 +123,9 @@ def _splitkv(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_l
              num_splits, s):
     """fa_fwd_splitkv with a workspace from PyTorch's allocator."""
     nbytes = _lib.lib().fa_fwd_splitkv_workspace_bytes(B, n_q, n_k, H, D, num_splits)
-    ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=q.device)
+    # allocated on the launching stream: not handed out again before the kernels have used it
+    with torch.cuda.stream(s):
+        ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=q.device)
     rc = _lib.lib().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                    lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, h_kv, D, scale,
                                    int(bool(causal)), int(window_left), dt, float(descales[0]),
@@ -204,11 +227,11 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq, dk, dv) of forward(q, k, v, scale, causal, window_left)
     for the upstream gradient dout, from the forward's out and lse (fp16 /
-    bf16, K/V heads equal to query heads).  The fp32 workspace the library
-    needs is taken from torch's allocator for the call."""
+    bf16).  k and v may have fewer heads than q (grouped-query attention):
+    dk and dv of a K/V head then sum over the query heads that read it.  The
+    fp32 workspace the library needs is taken from torch's allocator for the
+    call."""
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
-    if h_kv != H:
-        raise ValueError("backward needs as many K/V heads as query heads")
     if q.dtype not in (torch.float16, torch.bfloat16):
         raise ValueError("backward takes fp16 or bf16 inputs")
     for name, t in (("out", out), ("dout", dout)):
@@ -221,14 +244,24 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
         nbytes = int(_lib.lib().fa_bwd_workspace_bytes(B, n_q, H, D))
-        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
-        rc = _lib.lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
-                               lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H, D, scale,
-                               int(bool(causal)), int(window_left), _DT[q.dtype], ws.data_ptr(), nbytes,
-                               s.cuda_stream)
-        # keep the workspace alive until the kernels that use it have run
-        ws.record_stream(s)
-    _lib.check(rc, "fa_bwd")
+        with torch.cuda.stream(s):
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+        if h_kv == H:
+            rc = _lib.lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                   lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H, D,
+                                   scale, int(bool(causal)), int(window_left), _DT[q.dtype], ws.data_ptr(), nbytes,
+                                   s.cuda_stream)
+        else:
+            rc = _lib.lib().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H,
+                                       h_kv, D, scale, int(bool(causal)), int(window_left), _DT[q.dtype],
+                                       ws.data_ptr(), nbytes, s.cuda_stream)
+        # the outputs come from the current stream's pool: keep them reserved
+        # until the launching stream's kernels have written them
+        if s != torch.cuda.current_stream(q.device):
+            for t in (dq, dk, dv):
+                t.record_stream(s)
+    _lib.check(rc, "fa_bwd" if h_kv == H else "fa_bwd_gqa")
     return dq, dk, dv
 
 

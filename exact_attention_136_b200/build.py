@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa_b200.so")
 SOURCES = [os.path.join(CSRC, "fa_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_bwd_kernel.cuh", "sm100.cuh", "tmap.h")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_bwd_kernel.cuh", "fa_bwd_api.cuh", "sm100.cuh", "tmap.h")] + [
     os.path.join(os.path.dirname(HERE), "include", "fa.h")]
 
 NVCC_FLAGS = [

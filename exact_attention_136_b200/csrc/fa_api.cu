@@ -3,12 +3,13 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 #include <unordered_map>
+#include <vector>
 
 #include "../../include/fa.h"
 #include "fa_fwd_kernel.cuh"
-#include "fa_bwd_kernel.cuh"
 #include "tmap.h"
 
 namespace fa {
@@ -28,19 +29,22 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 // Scheduler scratch: one {next unit, finished CTAs} pair of counters per
-// stream, from a pool allocated once per device.  Launches on one stream run
-// in order, launches on different streams use different counters, and each
-// launch leaves its counters at zero.
+// stream.  Launches on one stream run in order, launches on different
+// streams use different counters, and each launch leaves its counters at
+// zero.  Pairs come from chunks of kSchedSlots allocated once each; when a
+// chunk is used up the next stream gets a pair from a new chunk, so no two
+// streams ever share one.  A pair is zeroed on its stream when the stream
+// first gets it (cudaMalloc'd memory starts undefined).
 constexpr int kSchedSlots = 256;
 
 struct DeviceState {
-  bool init = false;
+  std::atomic<bool> init{false};
   int num_sms = 0;
-  int* status = nullptr;     // device address of g_status_word
-  unsigned attr_set = 0;     // bit per kernel instantiation
-  unsigned* sched_pool = nullptr;
-  std::unordered_map<cudaStream_t, int> sched_slot;
-  int next_slot = 0;
+  int* status = nullptr;                 // device address of g_status_word
+  std::atomic<unsigned> attr_set{0};     // bit per kernel instantiation with its attributes set
+  std::vector<unsigned*> sched_chunks;   // kSchedSlots pairs each
+  std::unordered_map<cudaStream_t, unsigned*> sched_slot;
+  int used_in_last_chunk = kSchedSlots;
   unsigned* noalloc_scratch = nullptr;   // device address of g_noalloc_scratch
 };
 
@@ -52,14 +56,14 @@ int device_state(DeviceState** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   DeviceState& s = g_dev[dev];
-  if (!s.init) {
+  if (!s.init.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!s.init) {
+    if (!s.init.load(std::memory_order_relaxed)) {
       if (cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return FA_ERR_CUDA;
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.status), g_status_word) != cudaSuccess)
         return FA_ERR_CUDA;
-      s.init = true;
+      s.init.store(true, std::memory_order_release);
     }
   }
   *out = &s;
@@ -68,25 +72,34 @@ int device_state(DeviceState** out) {
 
 int sched_counters(DeviceState* ds, cudaStream_t stream, unsigned** out) {
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!ds->sched_pool) {
-    unsigned* pool = nullptr;
-    const size_t bytes = sizeof(unsigned) * 2 * kSchedSlots;
-    if (cudaMalloc(&pool, bytes) != cudaSuccess) return FA_ERR_CUDA;
-    if (cudaMemset(pool, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
-      cudaFree(pool);
-      return FA_ERR_CUDA;
-    }
-    ds->sched_pool = pool;
-  }
   auto it = ds->sched_slot.find(stream);
-  int slot;
   if (it != ds->sched_slot.end()) {
-    slot = it->second;
-  } else {
-    slot = ds->next_slot++ % kSchedSlots;
-    ds->sched_slot[stream] = slot;
+    *out = it->second;
+    return FA_OK;
   }
-  *out = ds->sched_pool + 2 * slot;
+  if (ds->used_in_last_chunk == kSchedSlots) {
+    unsigned* chunk = nullptr;
+    if (cudaMalloc(&chunk, sizeof(unsigned) * 2 * kSchedSlots) != cudaSuccess) return FA_ERR_CUDA;
+    ds->sched_chunks.push_back(chunk);
+    ds->used_in_last_chunk = 0;
+  }
+  unsigned* pair = ds->sched_chunks.back() + 2 * ds->used_in_last_chunk;
+  // zeroed on the stream that will use it, ahead of its first kernel
+  if (cudaMemsetAsync(pair, 0, 2 * sizeof(unsigned), stream) != cudaSuccess) return FA_ERR_CUDA;
+  ++ds->used_in_last_chunk;
+  ds->sched_slot[stream] = pair;
+  *out = pair;
+  return FA_OK;
+}
+
+// Sets the shared-memory attribute of a kernel instantiation once per device
+// (concurrent first calls may both set it, which is harmless).
+template <typename K>
+int set_smem_attr_once(DeviceState* ds, int bit, K kernel, int smem_bytes) {
+  if (ds->attr_set.load(std::memory_order_acquire) & (1u << bit)) return FA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+    return FA_ERR_CUDA;
+  ds->attr_set.fetch_or(1u << bit, std::memory_order_release);
   return FA_OK;
 }
 
@@ -119,17 +132,15 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
       encode_bnhd(&mk, k, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N) ||
       encode_bnhd(&mv, v, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N))
     return FA_ERR_CUDA;
-  if (!(ds->attr_set & (1u << bit))) {
-    if (cudaFuncSetAttribute(fa_fwd_kernel<D, DT, SPLIT, MASK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
-      return FA_ERR_CUDA;
+  if (!(ds->attr_set.load(std::memory_order_acquire) & (1u << bit))) {
     // The per-role register split (setmaxnreg) redistributes the registers
     // the CTA was launched with; it is only valid for the launch count it
     // was sized for, so a build that came out with another count is refused.
     cudaFuncAttributes fa{};
     if (cudaFuncGetAttributes(&fa, fa_fwd_kernel<D, DT, SPLIT, MASK>) != cudaSuccess) return FA_ERR_CUDA;
     if (fa.numRegs != REGS_LAUNCH) return FA_ERR_UNSUPPORTED;
-    ds->attr_set |= (1u << bit);
+    const int rc = set_smem_attr_once(ds, bit, fa_fwd_kernel<D, DT, SPLIT, MASK>, C::SMEM_BYTES);
+    if (rc != FA_OK) return rc;
   }
   const int grid = p.num_units < ds->num_sms ? p.num_units : ds->num_sms;
   if (sched_override) {
@@ -306,106 +317,10 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
 
 size_t elem_bytes(int dtype) { return dtype == FA_E4M3 ? 1 : 2; }
 
-// Workspace of the backward: fp32 dQ accumulator [B, N_q, H, D] followed by
-// D_i = rowsum(dO * O) [B, H, N_q].
-size_t bwd_workspace_bytes(int B, int Nq, int H, int D) {
-  return static_cast<size_t>(B) * Nq * H * (static_cast<size_t>(D) + 1) * sizeof(float);
-}
-
-template <int D, int DT>
-int launch_bwd(const void* q, const void* k, const void* v, const void* dout, const BwdParams& p,
-               cudaStream_t stream, DeviceState* ds, int bit) {
-  using C = BwdCfg<D>;
-  const CUtensorMapDataType tdt = DT == DT_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUtensorMap mq, mk, mv, mdo, mdq;
-  if (encode_bnhd(&mq, q, tdt, 2, p.B, p.Nq, p.H, D, 64, 128) ||
-      encode_bnhd(&mk, k, tdt, 2, p.B, p.Nk, p.H, D, 64, 128) ||
-      encode_bnhd(&mv, v, tdt, 2, p.B, p.Nk, p.H, D, 64, 128) ||
-      encode_bnhd(&mdo, dout, tdt, 2, p.B, p.Nq, p.H, D, 64, 128) ||
-      encode_bnhd(&mdq, p.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.Nq, p.H, D, 32, 128))
-    return FA_ERR_CUDA;
-  if (!(ds->attr_set & (1u << bit))) {
-    if (cudaFuncSetAttribute(fa_bwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
-    ds->attr_set |= (1u << bit);
-  }
-  const int64_t grid = static_cast<int64_t>(p.nkb) * p.B * p.H;
-  if (grid > 0x7fffffff) return FA_ERR_ARG;
-  fa_bwd_kernel<D, DT><<<static_cast<int>(grid), BWD_THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, mdq, p);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-int backward(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
-             void* dq, void* dk, void* dv, int B, int Nq, int Nk, int H, int D, float scale, int causal,
-             int window_left, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  int rc = validate(q, k, v, const_cast<void*>(out), B, Nq, Nk, H, D, scale, causal, window_left, dtype, H);
-  if (rc != FA_OK) return rc;
-  if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
-  if ((Nq > 0 && (!dout || !lse || !dq)) || (Nk > 0 && (!dk || !dv))) return FA_ERR_ARG;
-  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-    return FA_ERR_ALIGN;
-  const size_t ws = bwd_workspace_bytes(B, Nq, H, D);
-  if (ws > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws))
-    return FA_ERR_ARG;
-  if (Nq == 0 && Nk == 0) return FA_OK;
-  DeviceState* ds = nullptr;
-  rc = device_state(&ds);
-  if (rc != FA_OK) return rc;
-  if (Nq == 0) {
-    // no query sees any key: dK = dV = 0
-    const size_t kv_bytes = static_cast<size_t>(B) * Nk * H * D * 2;
-    if (cudaMemsetAsync(dk, 0, kv_bytes, stream) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, stream) != cudaSuccess)
-      return FA_ERR_CUDA;
-    return FA_OK;
-  }
-  float* dq_acc = static_cast<float*>(workspace);
-  float* delta = dq_acc + static_cast<size_t>(B) * Nq * H * D;
-  const int64_t rows = static_cast<int64_t>(B) * Nq * H;
-  {
-    const int64_t want = (rows + 7) / 8;
-    const int blocks = static_cast<int>(want < 8 * 148 ? want : 8 * 148);
-    if (D == 64) fa_bwd_prologue_kernel<64><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, dq_acc, B, Nq, H);
-    else fa_bwd_prologue_kernel<128><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, dq_acc, B, Nq, H);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  }
-  if (Nk > 0) {
-    BwdParams p{};
-    p.dk = dk;
-    p.dv = dv;
-    p.dq_acc = dq_acc;
-    p.lse = lse;
-    p.delta = delta;
-    p.B = B;
-    p.Nq = Nq;
-    p.Nk = Nk;
-    p.H = H;
-    p.causal = causal;
-    p.window_left = window_left;
-    p.scale = scale;
-    p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    p.nkb = (Nk + 127) / 128;
-    p.wait_limit_ns = g_wait_limit_ns;
-    p.status = ds->status;
-    switch (dtype * 2 + (D == 128 ? 1 : 0)) {
-      case FA_FP16 * 2 + 0: rc = launch_bwd<64, DT_FP16>(q, k, v, dout, p, stream, ds, 20); break;
-      case FA_FP16 * 2 + 1: rc = launch_bwd<128, DT_FP16>(q, k, v, dout, p, stream, ds, 21); break;
-      case FA_BF16 * 2 + 0: rc = launch_bwd<64, DT_BF16>(q, k, v, dout, p, stream, ds, 22); break;
-      case FA_BF16 * 2 + 1: rc = launch_bwd<128, DT_BF16>(q, k, v, dout, p, stream, ds, 23); break;
-      default: return FA_ERR_UNSUPPORTED;
-    }
-    if (rc != FA_OK) return rc;
-  }
-  const long long n = static_cast<long long>(rows) * D;
-  const long long want = (n / 4 + 255) / 256;
-  const int blocks = static_cast<int>(want < 16 * 148 ? want : 16 * 148);
-  fa_bwd_epilogue_kernel<<<blocks, 256, 0, stream>>>(dq_acc, dq, dtype, n);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
 }  // namespace
 }  // namespace fa
+
+#include "fa_bwd_api.cuh"   // backward: validation and launches
 
 extern "C" {
 
@@ -491,7 +406,7 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float
   if (rc != FA_OK) return rc;
   // the scheduler's counters index work units as 32-bit values: problems with
   // more units than that (or a scratch need above the array) are rejected
-  const int64_t units = static_cast<int64_t>((N_q + 255) / 256) * B * H;
+  const int64_t units = static_cast<int64_t>((N_q + 2 * fa::BLOCK_M - 1) / (2 * fa::BLOCK_M)) * B * H;
   if (fa::kSchedWordsNeeded > fa::kNoAllocScratchWords || units > 0x7fff0000LL) return FA_ERR_ARG;
   if (N_q == 0) return FA_OK;
   fa::DeviceState* ds = nullptr;
@@ -516,8 +431,16 @@ size_t fa_bwd_workspace_bytes(int B, int N_q, int H, int D) {
 int fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int D, float scale, int causal,
            int window_left, int dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, D, scale, causal, window_left, dtype,
+  return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, H, D, scale, causal, window_left, dtype,
                       workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int H_kv, int D, float scale,
+               int causal, int window_left, int dtype, void* workspace, size_t workspace_bytes,
+               fa_stream_t stream) {
+  return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, H_kv, D, scale, causal, window_left,
+                      dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_device_status(fa_stream_t stream, int* flags) {

@@ -1,0 +1,121 @@
+// Host side of the backward (included by fa_api.cu after its helpers):
+// argument validation, tensor maps and the three launches of fa_bwd.
+#pragma once
+
+#include "fa_bwd_kernel.cuh"
+
+namespace fa {
+namespace {
+
+// Workspace of the backward: D_i = rowsum(dO * O) [B, H, N_q] fp32.
+size_t bwd_workspace_bytes(int B, int Nq, int H, int D) {
+  (void)D;
+  return static_cast<size_t>(B) * Nq * H * sizeof(float);
+}
+
+// The dK/dV kernel (one CTA per key block) and the dQ kernel (one CTA per
+// query block), both after the prologue; one CTA per SM each (the dQ
+// kernel's shared-memory request is raised to keep a second CTA from
+// waiting on the first's tensor memory).
+template <int D, int DT>
+int launch_bwd(const void* q, const void* k, const void* v, const void* dout, const BwdParams& p,
+               cudaStream_t stream, DeviceState* ds, int bit) {
+  using C = BwdCfg<D>;
+  constexpr int DQ_SMEM_USED = 1024 + 6 * C::TILE;
+  constexpr int DQ_SMEM = DQ_SMEM_USED > 118 * 1024 ? DQ_SMEM_USED : 118 * 1024;
+  const CUtensorMapDataType tdt = DT == DT_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap mq, mk, mv, mdo;
+  if (encode_bnhd(&mq, q, tdt, 2, p.B, p.Nq, p.H, D, 64, 128) ||
+      encode_bnhd(&mk, k, tdt, 2, p.B, p.Nk, p.Hkv, D, 64, 128) ||
+      encode_bnhd(&mv, v, tdt, 2, p.B, p.Nk, p.Hkv, D, 64, 128) ||
+      encode_bnhd(&mdo, dout, tdt, 2, p.B, p.Nq, p.H, D, 64, 128))
+    return FA_ERR_CUDA;
+  if (!(ds->attr_set.load(std::memory_order_acquire) & (1u << bit))) {
+    if (cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    const int rc = set_smem_attr_once(ds, bit, fa_bwd_dq_kernel<D, DT>, DQ_SMEM);
+    if (rc != FA_OK) return rc;
+  }
+  const int64_t grid_kv = static_cast<int64_t>(p.nkb) * p.B * p.Hkv;
+  const int64_t grid_q = static_cast<int64_t>(p.nqb) * p.B * p.H;
+  if (grid_kv > 0x7fffffff || grid_q > 0x7fffffff) return FA_ERR_ARG;
+  fa_bwd_dkdv_kernel<D, DT><<<static_cast<int>(grid_kv), BWD_THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  fa_bwd_dq_kernel<D, DT><<<static_cast<int>(grid_q), BWD_THREADS, DQ_SMEM, stream>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int backward(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+             void* dq, void* dk, void* dv, int B, int Nq, int Nk, int H, int Hkv, int D, float scale, int causal,
+             int window_left, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int rc = validate(q, k, v, const_cast<void*>(out), B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
+  if (rc != FA_OK) return rc;
+  if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
+  if ((Nq > 0 && (!dout || !lse || !dq)) || (Nk > 0 && (!dk || !dv))) return FA_ERR_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return FA_ERR_ALIGN;
+  const size_t ws = bwd_workspace_bytes(B, Nq, H, D);
+  if (ws > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws))
+    return FA_ERR_ARG;
+  if (Nq == 0 && Nk == 0) return FA_OK;
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if (Nq == 0) {
+    // no query sees any key: dK = dV = 0
+    const size_t kv_bytes = static_cast<size_t>(B) * Nk * Hkv * D * 2;
+    if (cudaMemsetAsync(dk, 0, kv_bytes, stream) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  float* delta = static_cast<float*>(workspace);
+  const int64_t rows = static_cast<int64_t>(B) * Nq * H;
+  {
+    const int64_t want = (rows + 7) / 8;
+    const int blocks = static_cast<int>(want < 8 * 148 ? want : 8 * 148);
+    if (D == 64) fa_bwd_prologue_kernel<64><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, B, Nq, H);
+    else fa_bwd_prologue_kernel<128><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, B, Nq, H);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (Nk == 0) {
+    // no key: dQ = 0
+    if (cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * D * 2, stream) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  {
+    BwdParams p{};
+    p.dk = dk;
+    p.dv = dv;
+    p.dq = dq;
+    p.lse = lse;
+    p.delta = delta;
+    p.B = B;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.H = H;
+    p.Hkv = Hkv;
+    p.qpk = H / Hkv;
+    p.causal = causal;
+    p.window_left = window_left;
+    p.scale = scale;
+    p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.nkb = (Nk + 127) / 128;
+    p.nqb = (Nq + 127) / 128;
+    p.wait_limit_ns = g_wait_limit_ns;
+    p.status = ds->status;
+    switch (dtype * 2 + (D == 128 ? 1 : 0)) {
+      case FA_FP16 * 2 + 0: rc = launch_bwd<64, DT_FP16>(q, k, v, dout, p, stream, ds, 20); break;
+      case FA_FP16 * 2 + 1: rc = launch_bwd<128, DT_FP16>(q, k, v, dout, p, stream, ds, 21); break;
+      case FA_BF16 * 2 + 0: rc = launch_bwd<64, DT_BF16>(q, k, v, dout, p, stream, ds, 22); break;
+      case FA_BF16 * 2 + 1: rc = launch_bwd<128, DT_BF16>(q, k, v, dout, p, stream, ds, 23); break;
+      default: return FA_ERR_UNSUPPORTED;
+    }
+    if (rc != FA_OK) return rc;
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fa

@@ -1048,6 +1048,18 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
 }
 
 // ------------------------------------------------------------------ kernel
+// Called once per CTA by thread 0 when the CTA claims no more units: the
+// last CTA of the launch to get here zeroes the scheduler scratch for the
+// next launch (every CTA gets here: all waits are bounded).
+__device__ __forceinline__ void cta_finished(const FwdParams& p) {
+  __threadfence();
+  if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+    atomicExch(p.sched, 0u);
+    atomicExch(p.sched + 1, 0u);
+    __threadfence();
+  }
+}
+
 template <int D, int DT, bool SPLIT, int MASK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -1055,8 +1067,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   using C = Cfg<D, DT>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {
-    // 128-byte swizzled tiles need 1024-byte alignment; never expected
-    if (threadIdx.x == 0) atomicOr(p.status, ST_SMEM_MISALIGNED);
+    // 128-byte swizzled tiles need 1024-byte alignment; never expected.  The
+    // CTA still counts itself finished, so the scratch is left at zero.
+    if (threadIdx.x == 0) {
+      atomicOr(p.status, ST_SMEM_MISALIGNED);
+      cta_finished(p);
+    }
     return;
   }
   SharedHeader* sh = reinterpret_cast<SharedHeader*>(smem);
@@ -1122,17 +1138,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0)
     for (int i = 0; i < 64; ++i) atomicAdd(&g_stats[i], static_cast<unsigned long long>(sh->stats[i]));
 #endif
-  if (threadIdx.x == 0) {
-    // this CTA claims no more units; the last CTA to get here zeroes the
-    // scheduler scratch for the next launch (every CTA gets here: all waits
-    // are bounded)
-    __threadfence();
-    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-      atomicExch(p.sched, 0u);
-      atomicExch(p.sched + 1, 0u);
-      __threadfence();
-    }
-  }
+  if (threadIdx.x == 0) cta_finished(p);
 }
 
 // Combines the key-range slices of a split forward.  One warp per output

@@ -211,10 +211,10 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float
  *     H, D, scale, causal, window_left, dtype); lse is required here.
  *   dout, dq: [B, N_q, H, D]; dk, dv: [B, N_k, H, D]; 16-bit like q.
  *   workspace: caller-owned device memory of at least
- *     fa_bwd_workspace_bytes(B, N_q, H, D) bytes, 256-byte aligned: an fp32
- *     dQ accumulator and rowsum(dO * O).  The library allocates nothing.
- * Three kernels run in order on `stream` (rowsum(dO * O) and a zeroed
- * accumulator; dQ, dK, dV; dQ converted to 16-bit).  Returns FA_ERR_ARG /
+ *     fa_bwd_workspace_bytes(B, N_q, H, D) bytes, 256-byte aligned: the fp32
+ *     row term rowsum(dO * O), [B, H, N_q].  The library allocates nothing.
+ * Three kernels run in order on `stream`: the row term; dK and dV (one CTA
+ * per key block); dQ (one CTA per query block).  Returns FA_ERR_ARG /
  * FA_ERR_UNSUPPORTED (FA_E4M3, other head dims) / FA_ERR_ALIGN (16-byte
  * aligned tensors, 4-byte aligned lse) before any GPU work, FA_ERR_CUDA on a
  * launch failure, else FA_OK; waits that time out are reported by
@@ -225,6 +225,20 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* out, const v
            const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int D,
            float scale, int causal, int window_left, int dtype, void* workspace,
            size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fa_bwd_gqa -- fa_bwd for grouped K/V heads (the forward of fa_fwd_gqa;
+ * multi-query / grouped-query attention, Flash Attention | Hermes Skill,
+ * Workflow 2, Step 3): k, v, dk, dv are [B, N_k, H_kv, D] with H a multiple
+ * of H_kv, and query head h reads K/V head h / (H / H_kv).  dk and dv of a
+ * K/V head are the sums of the gradients of every query head that reads it.
+ * Workspace, ownership, kernels and return values as fa_bwd; FA_ERR_ARG also
+ * when H_kv < 1 or H is not a multiple of H_kv.
+ */
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* out, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H,
+               int H_kv, int D, float scale, int causal, int window_left, int dtype,
+               void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fa_device_status -- synchronises `stream`, then reads and clears the

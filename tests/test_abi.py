@@ -153,8 +153,8 @@ def test_mask_arguments_validated(kind, mask, sb, sh, sq):
 
 def test_backward_workspace_size():
     f = _lib.lib().fa_bwd_workspace_bytes
-    # fp32 dQ accumulator [B, N_q, H, D] plus the row term [B, H, N_q]
-    assert f(2, 300, 4, 128) == 2 * 300 * 4 * 129 * 4
+    # the fp32 row term rowsum(dO * O), [B, H, N_q]
+    assert f(2, 300, 4, 128) == 2 * 300 * 4 * 4
     assert f(1, 0, 1, 64) == 0
     assert f(0, 10, 1, 64) == 0 and f(1, 10, 1, 96) == 0
 
@@ -187,6 +187,17 @@ def _bwd(**kw):
 def test_backward_arguments_validated(kw, expect):
     """Backward arguments are checked on the host, before any GPU work."""
     assert _bwd(**kw) == expect
+
+
+@pytest.mark.parametrize("H, H_kv, expect", [(4, 3, _lib.FA_ERR_ARG), (4, 0, _lib.FA_ERR_ARG),
+                                             (2, 4, _lib.FA_ERR_ARG), (4, 2, _lib.FA_ERR_UNSUPPORTED)])
+def test_backward_gqa_heads_validated(H, H_kv, expect):
+    """fa_bwd_gqa checks the head grouping before any GPU work (D = 96 makes a
+    valid grouping stop at the head-dim check instead of launching)."""
+    D = 96 if expect == _lib.FA_ERR_UNSUPPORTED else 64
+    f = _lib.lib().fa_bwd_gqa
+    assert f(A, A, A, A, A, A, A, A, A, 1, 16, 16, H, H_kv, D, 0.125, 0, -1, _lib.FA_FP16, A, 1 << 20,
+             None) == expect
 
 
 def _prototypes():

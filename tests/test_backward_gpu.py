@@ -18,8 +18,8 @@ U = {"fp16": 2.0 ** -11, "bf16": 2.0 ** -8}
 DEV = torch.device("cuda", 0)
 
 
-def _run_and_check(B, n_q, n_k, H, D, dt, causal, wl, seed=0, scale=None):
-    qkv = inputs.make_qkv(B, n_q, n_k, H, D, dt, seeds=(500 + seed, 501 + seed, 502 + seed))
+def _run_and_check(B, n_q, n_k, H, D, dt, causal, wl, seed=0, scale=None, h_kv=0):
+    qkv = inputs.make_qkv(B, n_q, n_k, H, D, dt, seeds=(500 + seed, 501 + seed, 502 + seed), h_kv=h_kv or H)
     do = inputs.make_qkv(B, n_q, n_q, H, D, dt, seeds=(503 + seed, 504 + seed, 505 + seed)).q
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     q, k, v, g = (t.to(DEV) for t in (qkv.q, qkv.k, qkv.v, do))
@@ -73,9 +73,25 @@ def test_backward_many_key_blocks_accumulate_dq():
     _run_and_check(1, 1024, 1024, 1, 64, "fp16", False, -1, seed=3)
 
 
-def test_backward_rejects_fp8_and_gqa():
-    q = torch.zeros((1, 128, 2, 128), device=DEV, dtype=torch.bfloat16)
-    k = torch.zeros((1, 128, 1, 128), device=DEV, dtype=torch.bfloat16)
+GQA_CASES = [
+    # B, N_q, N_k, H, H_kv, D, dtype, causal, window_left
+    (1, 256, 256, 4, 2, 128, "bf16", True, -1),
+    (2, 300, 300, 4, 1, 64, "fp16", True, -1),
+    (1, 411, 257, 6, 2, 128, "fp16", False, -1),
+    (1, 520, 520, 4, 4, 64, "bf16", True, 130),
+    (1, 384, 384, 8, 2, 128, "bf16", False, 100),
+]
+
+
+@pytest.mark.parametrize("B,n_q,n_k,H,h_kv,D,dt,causal,wl", GQA_CASES)
+def test_backward_gqa_matches_oracle(B, n_q, n_k, H, h_kv, D, dt, causal, wl):
+    """Grouped K/V heads: dK and dV of a K/V head sum the gradients of every
+    query head of its group (fa_bwd_gqa), element by element under the bounds."""
+    _run_and_check(B, n_q, n_k, H, D, dt, causal, wl, seed=11, h_kv=h_kv)
+
+
+def test_backward_rejects_fp8():
+    q = torch.zeros((1, 128, 2, 128), device=DEV, dtype=torch.float8_e4m3fn)
     lse = torch.zeros((1, 2, 128), device=DEV)
     with pytest.raises(ValueError):
-        backward(q, k, k, q, lse, q)
+        backward(q, q, q, q, lse, q)

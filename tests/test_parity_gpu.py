@@ -241,6 +241,68 @@ def test_attn_mask_parity(case):
     assert d_l <= TOL_LSE, f"max|dLSE| {d_l:.3e} > {TOL_LSE}"
 
 
+def test_float_mask_of_another_type_is_rejected():
+    """Like SDPA, an additive mask must have the inputs' 16-bit type: an fp32
+    mask is refused rather than silently rounded."""
+    dev = torch.device("cuda", 0)
+    q = torch.zeros((1, 64, 2, 64), dtype=torch.bfloat16, device=dev)
+    with pytest.raises(ValueError):
+        forward(q, q, q, 0.125, False, -1, attn_mask=torch.zeros((64, 64), dtype=torch.float32, device=dev))
+    with pytest.raises(ValueError):
+        forward(q, q, q, 0.125, False, -1, attn_mask=torch.zeros((64, 64), dtype=torch.float16, device=dev))
+
+
+def test_mask_passed_in_place_equals_padded_copy():
+    """A mask whose rows are whole 16-byte chunks goes to the kernel as it is;
+    a strided view of the same values is copied first.  Same result."""
+    dev = torch.device("cuda", 0)
+    qkv = inputs.make_qkv(1, 256, 512, 2, 128, "bf16", seeds=(31, 32, 33))
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    g = torch.Generator().manual_seed(34)
+    wide = (2.0 * torch.randn((2, 256, 1024), generator=g)).to(torch.bfloat16).to(dev)
+    dense = wide[:, :, :512].contiguous()[None]         # [1, 2, 256, 512], taken as it is
+    strided = wide[:, :, ::2][None]                     # last dim strided: copied
+    strided_vals = strided.contiguous()
+    o1, l1 = forward(q, k, v, 0.09, False, -1, attn_mask=dense)
+    o2, l2 = forward(q, k, v, 0.09, False, -1, attn_mask=dense[:, :, :, :].expand(1, 2, 256, 512))
+    o3, l3 = forward(q, k, v, 0.09, False, -1, attn_mask=strided)
+    o4, l4 = forward(q, k, v, 0.09, False, -1, attn_mask=strided_vals)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(o3, o4) and torch.equal(l3, l4)
+    ref_o, ref_l = oracle(qkv, 0.09, False, -1, mask=dense.to(torch.float64).cpu().numpy())
+    d_o, d_l = compare(o1, l1, ref_o, ref_l)
+    assert d_o <= TOL_O["bf16"] and d_l <= TOL_LSE
+
+
+def test_temporaries_survive_a_side_stream():
+    """The split forward's workspace and a padded mask copy are freed when the
+    call returns; on a stream other than the current one they must stay
+    reserved until the kernels have run, even if the caller allocates and
+    overwrites memory right away."""
+    dev = torch.device("cuda", 0)
+    qkv = inputs.make_qkv(1, 128, 8192, 8, 128, "bf16", seeds=(41, 42, 43))
+    q, k, v = qkv.q.to(dev), qkv.k.to(dev), qkv.v.to(dev)
+    # N_k - 3 keys: the boolean mask's rows are not whole 16-byte chunks, so it is copied
+    mask = (torch.rand((1, 1, 128, 8192 - 3), generator=torch.Generator().manual_seed(44)) > 0.2).to(dev)
+    kq, vm = k[:, :8192 - 3].contiguous(), v[:, :8192 - 3].contiguous()
+    ref_s, ref_sl = forward(q, k, v, 0.09, False, -1, num_splits=8)
+    ref_m, ref_ml = forward(q, kq, vm, 0.09, False, -1, attn_mask=mask)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    for _ in range(3):
+        o_s, l_s = forward(q, k, v, 0.09, False, -1, num_splits=8, stream=side)
+        o_m, l_m = forward(q, kq, vm, 0.09, False, -1, attn_mask=mask, stream=side)
+        # both streams allocate at once and scribble on what they get
+        junk = [torch.full((1 << 22,), float("nan"), device=dev) for _ in range(8)]
+        with torch.cuda.stream(side):
+            junk += [torch.full((1 << 22,), float("nan"), device=dev) for _ in range(8)]
+        del junk
+        side.synchronize()
+        assert torch.equal(o_s, ref_s) and torch.equal(l_s, ref_sl)
+        assert torch.equal(o_m, ref_m) and torch.equal(l_m, ref_ml)
+
+
 def test_causal_pattern_mask_equals_causal():
     """A boolean mask holding the causal pattern gives the causal forward (to rounding)."""
     qkv = inputs.make_qkv(1, 640, 640, 2, 128, "bf16", seeds=(95, 96, 97))

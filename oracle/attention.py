@@ -52,6 +52,19 @@ and H_kv key/value heads (H a multiple of H_kv), query head h uses key/value
 head h // (H / H_kv).  H_kv = 1 is multi-query attention, H_kv = H the
 ordinary case.
 
+Dropout (the ``dropout_p`` argument of the pages' flash_attn_func, Flash
+Attention | Hermes Skill, Workflow 2, Step 2; the pages define neither the
+operation nor its random numbers).  The reading here is the usual one for
+attention dropout: after the softmax, each probability P_ij is kept with
+probability 1 - p and then divided by 1 - p, or set to 0, independently:
+
+    O_i = sum_j (Z_ij / (1 - p)) P_ij V[b,j,h,:],   Z_ij in {0, 1}
+
+with P and LSE exactly as above (the softmax normaliser counts every visible
+key; dropout does not change LSE).  The keep bits Z come from the
+counter-based generator in ``philox.py`` keyed by (seed, offset) and indexed
+by (batch, query head, row, key), so any implementation can reproduce them.
+
 Layouts follow the pages' flash_attn_func layout ``[batch, seqlen, nheads,
 headdim]`` for Q, K, V and O (Workflow 2, Step 2), and ``[batch, heads,
 N_q]`` for LSE (the pages print no LSE layout; this is our reading).
@@ -67,6 +80,8 @@ import math
 from typing import Iterable
 
 import numpy as np
+
+from .philox import dropout_keep
 
 __all__ = [
     "visibility",
@@ -95,7 +110,8 @@ def visibility(rows: Iterable[int], n_k: int, causal: bool, window_left: int) ->
 
 
 def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
-                  rows=None, return_probs: bool = False, mask=None):
+                  rows=None, return_probs: bool = False, mask=None, dropout_p: float = 0.0,
+                  seed: int = 0, offset: int = 0):
     """Exact attention forward in float64 (definition in the module docstring).
 
     q: [B, N_q, H, D]; k, v: [B, N_k, H_kv, D] with H a multiple of H_kv
@@ -105,8 +121,10 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
           (used for long sequences where the full N_q x N_k matrix is large).
     mask: optional boolean (True = attend) or real array broadcastable to
           [B, H, N_q, N_k]; a real mask is added to the scaled scores.
+    dropout_p, seed, offset: dropout of the probabilities (0 = none), keep
+          bits from philox.dropout_keep.
     Returns (O [B, R, H, D], LSE [B, H, R]) with R = len(rows) (or N_q), and
-    with ``return_probs`` also P [B, H, R, N_k].
+    with ``return_probs`` also the softmax P [B, H, R, N_k] (before dropout).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -155,7 +173,11 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
             e = np.where(vis, np.exp(s - m[:, None]), 0.0)
             l = e.sum(axis=1)
             p = e / np.where(seen, l, 1.0)[:, None]
-            out[b, :, h, :] = p @ v[b, :, hk, :]
+            if dropout_p > 0.0:
+                keep = dropout_keep(seed, offset, b, h, H, rows, n_k, dropout_p)
+                out[b, :, h, :] = (np.where(keep, p, 0.0) / (1.0 - dropout_p)) @ v[b, :, hk, :]
+            else:
+                out[b, :, h, :] = p @ v[b, :, hk, :]
             lse[b, h, :] = np.where(seen, m + np.log(np.where(seen, l, 1.0)), -np.inf)
             if return_probs:
                 probs[b, h] = p
@@ -164,7 +186,8 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
     return out, lse
 
 
-def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_left: int = -1, mask=None):
+def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_left: int = -1, mask=None,
+                         dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
     """Pure-Python triple loop over (query, key, dim), for tiny shapes only.
 
     Written independently of ``attention_ref``: nested lists, ``math.exp``, no
@@ -173,7 +196,8 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
     ``attention_ref``'s outputs.  K and V may have fewer heads than Q (query
     head h then reads head h * H_kv // H, the same contiguous groups).  mask:
     optional nested [B or 1][H or 1][N_q][N_k] of booleans (keep where True)
-    or numbers (added to the scaled score).
+    or numbers (added to the scaled score).  dropout_p > 0: each weight is
+    kept where philox.dropout_keep says so and then divided by 1 - dropout_p.
     """
     B = len(q)
     n_q = len(q[0])
@@ -186,6 +210,7 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
     for b in range(B):
         for h in range(H):
             g = h * h_kv // H
+            kept = dropout_keep(seed, offset, b, h, H, range(n_q), n_k, dropout_p) if dropout_p > 0 else None
             for i in range(n_q):
                 weights = []
                 for j in range(n_k):
@@ -214,12 +239,17 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
                 for d in range(D):
                     acc = 0.0
                     for j, w in weights:
+                        if kept is not None:
+                            if not kept[i][j]:
+                                continue
+                            w = w / (1.0 - dropout_p)
                         acc += w * float(v[b][j][g][d])
                     O[b][i][h][d] = acc / total
     return O, L
 
 
-def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, window_left: int = -1):
+def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, window_left: int = -1,
+                           dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
     """Gradients of the exact attention forward, in float64.
 
     The pages name the backward pass only by its method: the speed and memory
@@ -240,7 +270,10 @@ def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, wind
     with P, S, visibility and the K/V head of each query head exactly as in
     ``attention_ref``; a K/V head shared by a group of query heads gets the sum
     of their dK and dV.  Invisible (i, j) pairs have P_ij = 0 and contribute
-    nothing, and a row with no visible key contributes nothing at all.
+    nothing, and a row with no visible key contributes nothing at all.  With
+    dropout (keep bits Z, probability p) the forward uses Pd = Z P / (1 - p),
+    so dV = Pd^T dO, dP = Z (dO V^T) / (1 - p), and dS, dQ, dK follow as above
+    (sum_j' P_ij' dP_ij' is still sum_d dO_id O_id).
 
     q, do: [B, N_q, H, D]; k, v: [B, N_k, H_kv, D].  Returns (dQ, dK, dV)
     shaped like q, k, v.
@@ -254,6 +287,7 @@ def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, wind
     if do.shape != q.shape:
         raise ValueError("do must be shaped like q")
     _, _, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True)
+    rows = np.arange(n_q, dtype=np.int64)
     group = H // h_kv
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
@@ -263,8 +297,13 @@ def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, wind
             hk = h // group
             p = probs[b, h]                       # [N_q, N_k], zero where invisible
             g = do[b, :, h, :]                    # [N_q, D]
-            dv[b, :, hk, :] += p.T @ g
             dp = g @ v[b, :, hk, :].T             # [N_q, N_k]
+            if dropout_p > 0.0:
+                z = dropout_keep(seed, offset, b, h, H, rows, n_k, dropout_p) / (1.0 - dropout_p)
+                dv[b, :, hk, :] += (z * p).T @ g
+                dp = z * dp
+            else:
+                dv[b, :, hk, :] += p.T @ g
             ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
             dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])
             dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])

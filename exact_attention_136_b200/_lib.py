@@ -51,6 +51,7 @@ SIGNATURES = {
     "fa_device_status": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_wait_probe": (_c_int, [ctypes.c_ulonglong, _vp]),
+    "fa_exp2_check": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_version": (ctypes.c_char_p, []),
 }

@@ -470,6 +470,16 @@ int fa_wait_probe(unsigned long long limit_ns, fa_stream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_exp2_check(const float* x, float* poly, float* mufu, int n, int degree, fa_stream_t stream) {
+  if (n < 0 || (degree != 2 && degree != 3)) return FA_ERR_ARG;
+  if (n == 0) return FA_OK;
+  if (!x || !poly || !mufu) return FA_ERR_ARG;
+  const int threads = 256;
+  const int blocks = static_cast<int>(((n + 1) / 2 + threads - 1) / threads < 1024 ? ((n + 1) / 2 + threads - 1) / threads : 1024);
+  fa::fa_exp2_check_kernel<<<blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, poly, mufu, n, degree);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 const char* fa_status_string(int status) {
   switch (status) {
     case FA_OK: return "ok";

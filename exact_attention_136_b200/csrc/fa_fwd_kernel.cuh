@@ -97,6 +97,18 @@ struct FwdParams {
   float mask_scale;    // 1 / (scale * q_descale * k_descale)
 };
 
+// Exponentials taken on the FMA pipe (see Cfg::EMU_FROM): pairs i >= this of
+// every 8, per instantiation; 8 = none.
+#ifndef FA_EMU_FROM_D128
+#define FA_EMU_FROM_D128 8
+#endif
+#ifndef FA_EMU_FROM_D64
+#define FA_EMU_FROM_D64 8
+#endif
+#ifndef FA_EMU_FROM_E4M3
+#define FA_EMU_FROM_E4M3 8
+#endif
+
 constexpr int BLOCK_M = 128;   // query rows per tile
 constexpr int BLOCK_N = 128;   // keys per block
 constexpr int NUM_THREADS = 640;   // warpgroup 0: load + MMA; 2 warpgroups per Q tile
@@ -132,12 +144,18 @@ struct Cfg {
   // Measured on B200: faster for 16-bit inputs; for e4m3, whose PV is only
   // four MMAs, the extra hand-over costs more than the overlap gains.
   static constexpr bool PSPLIT = DT != DT_E4M3;
+  // Exponentials on the FMA pipe: pairs i >= EMU_FROM of every 8 in a block
+  // without masked keys take exp2_poly instead of MUFU (8 = none), with a
+  // polynomial of degree EMU_DEG (P is rounded to e4m3's 3-bit mantissa in
+  // the FP8 path, so degree 2 is ample there).
+  static constexpr int EMU_FROM = DT == DT_E4M3 ? FA_EMU_FROM_E4M3 : (D == 64 ? FA_EMU_FROM_D64 : FA_EMU_FROM_D128);
+  static constexpr int EMU_DEG = DT == DT_E4M3 ? 2 : 3;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(D == 64 || D == 128, "head dim");
 };
 
 struct SharedHeader {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];   // per Q tile: loaded / read by the tile's last S
   uint64_t kv_full[12], kv_empty[12];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t p_half[2];   // first half of P_t stored (keys k of the block with k mod 64 < 32)
@@ -232,7 +250,7 @@ constexpr int kTraceSlice = 16384;
 #define FA_TRACE_DECL unsigned trace_n = 0
 #define FA_TRACE(who, ev, j)                                                                          \
   do {                                                                                                \
-    if (blockIdx.x == 0 && ((who) >= 2 || (threadIdx.x & 127) == 0) && g_trace && trace_n < kTraceSlice) \
+    if (blockIdx.x == 0 && ((who) >= 2 || threadIdx.x == 128u + 256u * (who)) && g_trace && trace_n < kTraceSlice) \
       g_trace[(who) * kTraceSlice + trace_n++] =                                                      \
           (static_cast<unsigned long long>((ev) & 0xff) << 48) |                                     \
           (static_cast<unsigned long long>((j) & 0xffff) << 32) |                                    \
@@ -306,7 +324,8 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
   uint32_t q_uses = 0;
   uint32_t issued_mask = 0;   // bit s: slot s has had a load
   uint32_t phase_mask = 0;    // bit s: parity of slot s's latest load
-  bool q_outstanding = false;
+  uint32_t q_loaded = 0;       // bit t: Q tile t has had a load
+  uint32_t q_phase = 0;        // bit t: parity of Q tile t's latest load
   bool ok = true;
   FA_TRACE_DECL;
   const uint64_t pol_kv = policy_evict_last();
@@ -336,18 +355,23 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
       continue;
     }
     if (aborted(sh)) { ok = false; break; }
-    // Q tiles (wait until the previous unit's S MMAs have read them)
-    if (!mbar_wait(smem_u32(&sh->q_empty), (q_uses & 1u) ^ 1u, p.wait_limit_ns)) {
-      record_error(sh, p, ST_TIMEOUT_LOAD); ok = false; break;
-    }
-    mbar_arrive_expect_tx(smem_u32(&sh->q_full), 2 * C::TILE_BYTES);
+    // Q tiles, each as soon as the previous unit's last S of that tile has
+    // read it (tile 0's last S of a causal unit comes a key block before
+    // tile 1's, so its next Q loads during the unit's last block)
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+    for (int t = 0; t < 2 && ok; ++t) {
+      if (!mbar_wait(smem_u32(&sh->q_empty[t]), (q_uses & 1u) ^ 1u, p.wait_limit_ns)) {
+        record_error(sh, p, ST_TIMEOUT_LOAD); ok = false; break;
+      }
+      mbar_arrive_expect_tx(smem_u32(&sh->q_full[t]), C::TILE_BYTES);
 #pragma unroll
       for (int c = 0; c < C::NCHUNK; ++c)
-        tma_load_4d_hint(smem_u32(sq + t * C::TILE_BYTES + c * C::CHUNK_BYTES), mq, smem_u32(&sh->q_full),
+        tma_load_4d_hint(smem_u32(sq + t * C::TILE_BYTES + c * C::CHUNK_BYTES), mq, smem_u32(&sh->q_full[t]),
                          c * C::BOX_INNER, w.h, w.q0 + t * BLOCK_M, w.b, pol_q);
-    q_outstanding = true;
+      q_loaded |= 1u << t;
+      q_phase = (q_phase & ~(1u << t)) | ((q_uses & 1u) << t);
+    }
+    if (!ok) break;
     ++q_uses;
     // K_j, V_j for the union of the tiles' block ranges
     for (int j = w.jlo; j <= w.jhi && ok; ++j) {
@@ -395,8 +419,10 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
       if (((issued_mask >> s) & 1u) &&
           !mbar_wait(smem_u32(&sh->kv_full[s]), (phase_mask >> s) & 1u, p.wait_limit_ns))
         record_error(sh, p, ST_TIMEOUT_DRAIN);
-    if (q_outstanding && !mbar_wait(smem_u32(&sh->q_full), (q_uses - 1u) & 1u, p.wait_limit_ns))
-      record_error(sh, p, ST_TIMEOUT_DRAIN);
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      if (((q_loaded >> t) & 1u) && !mbar_wait(smem_u32(&sh->q_full[t]), (q_phase >> t) & 1u, p.wait_limit_ns))
+        record_error(sh, p, ST_TIMEOUT_DRAIN);
   }
   FA_TRACE(3, 15, 0);
 }
@@ -502,6 +528,7 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
   const uint32_t kv_empty0 = smem_u32(&sh->kv_empty[0]);
   const uint32_t s_full0 = smem_u32(&sh->s_full[0]), p_full0 = smem_u32(&sh->p_full[0]);
   const uint32_t p_half0 = smem_u32(&sh->p_half[0]);
+  const uint32_t q_empty0 = smem_u32(&sh->q_empty[0]);
   const uint64_t lim = p.wait_limit_ns;
   uint32_t q_uses = 0;
   uint32_t p_waits[2] = {0, 0};
@@ -523,16 +550,22 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
     const Unit w = get_unit<SPLIT>(u, us, p);
     if (w.jhi < 0) continue;
     if (aborted(sh)) { ok = false; break; }
-    if (!mbar_wait(smem_u32(&sh->q_full), q_uses & 1u, lim)) {
+    if (!mbar_wait(smem_u32(&sh->q_full[0]), q_uses & 1u, lim) ||
+        !mbar_wait(smem_u32(&sh->q_full[1]), q_uses & 1u, lim)) {
       record_error(sh, p, ST_TIMEOUT_MMA); ok = false; break;
     }
     ++q_uses;
-    // Steady key blocks: both tiles issue PV(j-1) and S(j), and j-1 is
+    // a tile without key blocks here does not read its Q tile (it has landed)
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      if (!w.valid[t]) mbar_arrive(smem_u32(&sh->q_empty[t]));
+    // Steady key blocks: both tiles issue PV(j-1) and S(j), j-1 is
     // neither tile's first block (O starts from zero there, after the
-    // previous unit's epilogue has read it) nor its last (O is handed over).
+    // previous unit's epilogue has read it) nor its last (O is handed over),
+    // and j is neither tile's last (its S releases the tile's Q buffer).
     const bool both = w.valid[0] && w.valid[1];
     const int js = both ? max(w.lo[0], w.lo[1]) + 2 : 0x7fffffff;
-    const int je = both ? min(w.hi[0], w.hi[1]) : -1;
+    const int je = both ? min(w.hi[0], w.hi[1]) - 1 : -1;
     for (int j = w.jlo; j <= w.jhi + 1 && ok; ++j) {
       const uint32_t vfull = kv_full0 + 8u * vslot, kfull = kv_full0 + 8u * kslot;
       if (j >= js && j <= je) {
@@ -624,6 +657,7 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
             }
             issue_s<D, DT>(tbase + 128 * t, opaque(q_desc0) + t * SLOT_DESC, k_desc, hi);
             mma_commit(s_full0 + 8u * t);
+            if (j == w.hi[t]) mma_commit(q_empty0 + 8u * t);   // the tile's last read of its Q tile
             if (t == 1 || !s_use[1]) {
               mma_commit(kv_empty0 + 8u * kslot);   // last reader of K_j
               k_done = true;
@@ -654,7 +688,6 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
       }
     }
     if (!ok) break;
-    mma_commit(smem_u32(&sh->q_empty));
   }
   FA_TRACE(2, 15, 0);
   // all issued MMAs complete before the CTA releases TMEM
@@ -710,12 +743,16 @@ __device__ __forceinline__ void store_part_row16(float* dst, const float* o, flo
         make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
 }
 
+// Coefficients of 2^f on f in [-1/2, 1/2], fitted by the Remez exchange on
+// relative error (csrc/gen_exp2_poly.py): degree 3, max relative error
+// 7.5e-5 (below the 16-bit P rounding); degree 2, 1.7e-3 (far below e4m3's).
+
 // 2^x on the FMA pipe for a pair of finite x (unmasked blocks only).
 // Range reduction for base 2 is exact: x = j + f with j = round(x) and
-// f in [-1/2, 1/2]; 2^j is added into the exponent field and 2^f is a cubic
-// fitted by the Remez exchange on relative error (csrc/gen_exp2_poly.py:
-// max relative error 7.5e-5, below the 16-bit P rounding).  x is clamped to
-// -125 first so 2^j stays a normal number; those terms are < 2^-124.
+// f in [-1/2, 1/2]; 2^j is added into the exponent field and 2^f is the
+// polynomial above.  x is clamped to -125 first so 2^j stays a normal
+// number; those terms are < 2^-124.
+template <int DEG>
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
   x.x = fmaxf(x.x, -125.0f);
@@ -723,10 +760,18 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
   const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
   const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
-  float2 q = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
-                        make_float2(0.2426111251115799f, 0.2426111251115799f));
-  q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  q = __ffma2_rn(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  float2 q;
+  if constexpr (DEG == 3) {
+    q = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                   make_float2(0.2426111251115799f, 0.2426111251115799f));
+    q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    q = __ffma2_rn(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  } else {
+    static_assert(DEG == 2, "polynomial degree");
+    q = __ffma2_rn(make_float2(0.23842893540859222f, 0.23842893540859222f), f,
+                   make_float2(0.7034479975700378f, 0.7034479975700378f));
+    q = __ffma2_rn(q, f, make_float2(1.0004431009292603f, 1.0004431009292603f));
+  }
   // t's low mantissa bits hold j; shifting by 23 moves j into the exponent field
   return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
@@ -744,18 +789,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // threads 0-15, the same lanes half a row of P further for threads 16-31)
 // and return their fp32 sum twice: exact, and over the values P*V uses
 // (different only for e4m3, whose 3-bit mantissa would otherwise bias O).
-// Pairs i >= FA_EMU_FROM of every 8 (unmasked blocks) take exp2_poly2 on the
-// FMA pipe instead of MUFU.  Default 8 = none: in the full kernel, where the
-// two tiles' softmax warps share every scheduler, the emulation's extra
-// instructions cost more than the MUFU time they free (B200, causal D=128
-// bf16: 988 TF/s without, 939 with 3 of 8 pairs emulated; D=64 fp16 and FP8
-// the same way).  Kept as a build option for configurations where MUFU is
-// the binding limit.
-#ifndef FA_EMU_FROM
-#define FA_EMU_FROM 8
-#endif
-
-template <int DT, bool EMULATE, int Q0, int NQ>
+// With EMULATE (blocks without masked keys), pairs i >= EMU_FROM of every 8
+// take exp2_poly2 on the FMA pipe instead of MUFU.
+template <int DT, bool EMULATE, int Q0, int NQ, int EMU_FROM = 8, int EMU_DEG = 3>
 __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_mref, uint32_t p_addr) {
   const float2 cc2 = make_float2(cc, cc);
   const float2 nm2 = make_float2(neg_mref, neg_mref);
@@ -770,8 +806,8 @@ __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_m
       const int c = q * 16 + 2 * i;
       const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), cc2, nm2);
       float2 e;
-      if (EMULATE && i >= FA_EMU_FROM) {
-        e = exp2_poly2(x);
+      if (EMULATE && i >= EMU_FROM) {
+        e = exp2_poly2<EMU_DEG>(x);
       } else {
         e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       }
@@ -963,7 +999,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       // the split hand-over, P over keys k with k mod 64 < 32 goes first
       constexpr int NQ0 = C::PSPLIT ? 2 : 4;
       float2 lsum = need_mask ? exp_half<DT, false, 0, NQ0>(s, cc, -mref, p_addr)
-                              : exp_half<DT, true, 0, NQ0>(s, cc, -mref, p_addr);
+                              : exp_half<DT, true, 0, NQ0, C::EMU_FROM, C::EMU_DEG>(s, cc, -mref, p_addr);
       float alpha = 1.f;
       if (warp_rescale) alpha = (m_cand == -INFINITY) ? 1.f : ex2_approx(m_old - m_cand);
       // O rescale of this thread's half row (only when some row of this warp
@@ -993,7 +1029,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
         mbar_arrive(smem_u32(&sh->p_half[t]));
         FA_TRACE(t, 12, j);
         const float2 ls2 = need_mask ? exp_half<DT, false, 2, 2>(s, cc, -mref, p_addr)
-                                     : exp_half<DT, true, 2, 2>(s, cc, -mref, p_addr);
+                                     : exp_half<DT, true, 2, 2, C::EMU_FROM, C::EMU_DEG>(s, cc, -mref, p_addr);
         lsum = make_float2(lsum.x + ls2.x, lsum.y + ls2.y);
       }
       FA_TRACE(t, 4, j);
@@ -1015,27 +1051,26 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     FA_TRACE(t, 6, 0);
     tc_fence_after();
     const float inv = (lq_row > 0.f ? 1.f / lq_row : 0.f) * p.out_scale;
-    if constexpr (SPLIT) {
-      float* part_row = p.o_part + part_rows() * D + o_elem();
+    // the thread's whole half row of O in one round trip (its scores are
+    // dead by now, so the registers are free), then O_t is released
+    uint32_t o[HALF_D];
 #pragma unroll
-      for (int c = 0; c < HALF_D; c += 16) {
-        uint32_t o[16];
-        tmem_ld_16x32bx2_x16<HALF_D>(o_addr + c, o);
-        tmem_wait_ld();
-        if (row_ok) store_part_row16(part_row + c, reinterpret_cast<float*>(o), inv);
-      }
-    } else {
-      uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem() * OUT_ES;
-#pragma unroll
-      for (int c = 0; c < HALF_D; c += 16) {
-        uint32_t o[16];
-        tmem_ld_16x32bx2_x16<HALF_D>(o_addr + c, o);
-        tmem_wait_ld();
-        if (row_ok) store_out_row16<DT>(out_row + c * OUT_ES, reinterpret_cast<float*>(o), inv);
-      }
-    }
+    for (int c = 0; c < HALF_D; c += 32) tmem_ld_16x32bx2_x32<HALF_D>(o_addr + c, o + c);
+    tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(smem_u32(&sh->o_empty[t]));
+    if (row_ok) {
+      if constexpr (SPLIT) {
+        float* part_row = p.o_part + part_rows() * D + o_elem();
+#pragma unroll
+        for (int c = 0; c < HALF_D; c += 16) store_part_row16(part_row + c, reinterpret_cast<float*>(o + c), inv);
+      } else {
+        uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem() * OUT_ES;
+#pragma unroll
+        for (int c = 0; c < HALF_D; c += 16)
+          store_out_row16<DT>(out_row + c * OUT_ES, reinterpret_cast<float*>(o + c), inv);
+      }
+    }
     if (row_ok && half == 0) {
       // natural log of sum_j exp(scale * s_j) = (m_used + log2(l) - PSHIFT) * ln 2
       const float lse_v = l_row > 0.f ? (m_used + __log2f(l_row) - C::PSHIFT) * 0.69314718055994531f : -INFINITY;
@@ -1080,8 +1115,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x / 32;
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&sh->q_full), 1);
-    mbar_init(smem_u32(&sh->q_empty), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&sh->q_full[t]), 1);
+      mbar_init(smem_u32(&sh->q_empty[t]), 1);
+    }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_u32(&sh->kv_full[s]), 1);
       mbar_init(smem_u32(&sh->kv_empty[s]), 1);
@@ -1208,6 +1245,22 @@ __global__ void fa_empty_kernel(void* out, float* lse, int B, int Nq, int H) {
       const int64_t n = bn % Nq;
       const int64_t b = bn / Nq;
       lse[(b * H + h) * Nq + n] = -INFINITY;
+    }
+  }
+}
+
+// The kernel's two ways of taking 2^x, side by side: the FMA-pipe
+// polynomial of the given degree (2 or 3) and MUFU's ex2.approx.ftz.
+__global__ void fa_exp2_check_kernel(const float* __restrict__ x, float* __restrict__ poly,
+                                     float* __restrict__ mufu, int n, int degree) {
+  for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * gridDim.x * blockDim.x) {
+    const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+    const float2 r = degree == 2 ? exp2_poly2<2>(v) : exp2_poly2<3>(v);
+    poly[i] = r.x;
+    mufu[i] = ex2_approx(v.x);
+    if (i + 1 < n) {
+      poly[i + 1] = r.y;
+      mufu[i + 1] = ex2_approx(v.y);
     }
   }
 }

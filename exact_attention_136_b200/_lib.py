@@ -38,6 +38,8 @@ SIGNATURES = {
     "fa_fwd_mask": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                              _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp, _c_int,
                              ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, _vp]),
+    "fa_fwd_dropout": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                _c_float, _c_int, _c_int, _c_int, _c_float, ctypes.c_ulonglong, ctypes.c_uint, _vp]),
     "fa_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                              _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, _c_float,
                              _c_float, _vp]),
@@ -48,6 +50,9 @@ SIGNATURES = {
                         _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
     "fa_bwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                             _c_int, _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
+    "fa_bwd_dropout": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
+                                _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, ctypes.c_ulonglong,
+                                ctypes.c_uint, _vp, ctypes.c_size_t, _vp]),
     "fa_device_status": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_wait_probe": (_c_int, [ctypes.c_ulonglong, _vp]),

@@ -138,7 +138,8 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
             causal: bool = False, window_left: int = -1, out: Optional[torch.Tensor] = None,
             lse: Optional[torch.Tensor] = None, return_lse: bool = True,
             stream: Optional[torch.cuda.Stream] = None, num_splits: int = 1,
-            attn_mask: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            attn_mask: Optional[torch.Tensor] = None, dropout_p: float = 0.0, seed: Optional[int] = None,
+            offset: int = 0) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Exact attention forward; returns (out, lse).
 
     scale=None means 1/sqrt(headdim), the pages' auto scale (Workflow 2,
@@ -151,8 +152,15 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
     attn_mask: the pages' SDPA mask (Workflow 1, Step 2) -- bool (attend where
     True) or float (added to the scaled scores), [N_q, N_k] or
     [B or 1, H or 1, N_q, N_k]; not combined with num_splits.
+    dropout_p > 0: dropout of the attention probabilities (fa_fwd_dropout;
+    fp16 / bf16, not combined with attn_mask or num_splits), with the keep
+    bits drawn from the 64-bit seed (required) and the 32-bit offset; the
+    backward needs the same seed and offset.
     """
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
+    if dropout_p:
+        return _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, stream, num_splits,
+                                attn_mask, dropout_p, seed, offset)
     if num_splits == 0:
         num_splits = auto_splits(B, n_q, n_k, H, q.device)
     if q.dtype == torch.float8_e4m3fn:
@@ -181,6 +189,29 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
                                        n_k, H, h_kv, D, scale, int(bool(causal)), int(window_left), _DT[q.dtype],
                                        1.0, 1.0, 1.0, s.cuda_stream)
     _lib.check(rc, "fa_fwd" if h_kv == H else "fa_fwd_gqa")
+    return out, lse
+
+
+def _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, stream, num_splits, attn_mask,
+                     dropout_p, seed, offset):
+    B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
+    if not (0.0 <= dropout_p < 1.0):
+        raise ValueError("dropout_p must be in [0, 1)")
+    if q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("dropout takes fp16 or bf16 inputs")
+    if attn_mask is not None or num_splits not in (0, 1):
+        raise ValueError("dropout is not combined with attn_mask or num_splits")
+    if seed is None:
+        raise ValueError("dropout needs an explicit seed (and offset) so the backward can redraw the mask")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out, lse = _outputs(q, B, n_q, H, D, out, lse, return_lse)
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        rc = _lib.lib().fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                       lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, h_kv, D, scale,
+                                       int(bool(causal)), int(window_left), _DT[q.dtype], float(dropout_p),
+                                       int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF, s.cuda_stream)
+    _lib.check(rc, "fa_fwd_dropout")
     return out, lse
 
 
@@ -224,13 +255,15 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
 
 def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
              dout: torch.Tensor, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,
-             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+             stream: Optional[torch.cuda.Stream] = None, dropout_p: float = 0.0, seed: Optional[int] = None,
+             offset: int = 0) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq, dk, dv) of forward(q, k, v, scale, causal, window_left)
     for the upstream gradient dout, from the forward's out and lse (fp16 /
     bf16).  k and v may have fewer heads than q (grouped-query attention):
-    dk and dv of a K/V head then sum over the query heads that read it.  The
-    fp32 workspace the library needs is taken from torch's allocator for the
-    call."""
+    dk and dv of a K/V head then sum over the query heads that read it.
+    dropout_p, seed, offset: those of a dropout forward (fa_bwd_dropout redraws
+    its keep bits).  The fp32 workspace the library needs is taken from
+    torch's allocator for the call."""
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
     if q.dtype not in (torch.float16, torch.bfloat16):
         raise ValueError("backward takes fp16 or bf16 inputs")
@@ -246,7 +279,15 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
         nbytes = int(_lib.lib().fa_bwd_workspace_bytes(B, n_q, H, D))
         with torch.cuda.stream(s):
             ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
-        if h_kv == H:
+        if dropout_p:
+            if seed is None:
+                raise ValueError("a dropout backward needs the forward's seed (and offset)")
+            rc = _lib.lib().fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H,
+                                           h_kv, D, scale, int(bool(causal)), int(window_left), _DT[q.dtype],
+                                           float(dropout_p), int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF,
+                                           ws.data_ptr(), nbytes, s.cuda_stream)
+        elif h_kv == H:
             rc = _lib.lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
                                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H, D,
                                    scale, int(bool(causal)), int(window_left), _DT[q.dtype], ws.data_ptr(), nbytes,
@@ -261,7 +302,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
         if s != torch.cuda.current_stream(q.device):
             for t in (dq, dk, dv):
                 t.record_stream(s)
-    _lib.check(rc, "fa_bwd" if h_kv == H else "fa_bwd_gqa")
+    _lib.check(rc, "fa_bwd_dropout" if dropout_p else ("fa_bwd" if h_kv == H else "fa_bwd_gqa"))
     return dq, dk, dv
 
 

@@ -183,10 +183,16 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
             int H, int Hkv, int D, float scale, int causal, int window_left, int dtype, float qd, float kd,
             float vd, cudaStream_t stream, unsigned* sched_override = nullptr, int splits = 1,
             void* workspace = nullptr, size_t workspace_bytes = 0, const void* mask = nullptr,
-            int mask_type = 0, long long mask_sb = 0, long long mask_sh = 0, long long mask_sq = 0) {
+            int mask_type = 0, long long mask_sb = 0, long long mask_sh = 0, long long mask_sq = 0,
+            float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0) {
   int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
   if (rc != FA_OK) return rc;
   if (splits < 1) return FA_ERR_ARG;
+  // dropout: 0 <= p < 1, 16-bit inputs, not combined with a mask or a split key range
+  if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_ARG;
+  const bool dropout = dropout_p > 0.f;
+  if (dropout && (mask_type != 0 || splits != 1)) return FA_ERR_ARG;
+  if (dropout && dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
   if (mask_type != 0) {
     // byte (boolean) or 16-bit (additive) elements; every row of the mask
     // starts on a 16-byte boundary and holds N_k elements
@@ -265,6 +271,22 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   p.mask_sh = mask_sh;
   p.mask_sq = mask_sq;
   p.mask_scale = static_cast<float>(1.0 / (static_cast<double>(scale) * qd * kd));
+  if (dropout) {
+    // keep key j when its 16-bit random value is >= round(p * 65536) (ties
+    // to even); kept probabilities are scaled by 1 / (1 - p)
+    p.drop_threshold = static_cast<unsigned>(std::nearbyint(static_cast<double>(dropout_p) * 65536.0));
+    p.seed_lo = static_cast<unsigned>(seed & 0xffffffffull);
+    p.seed_hi = static_cast<unsigned>(seed >> 32);
+    p.drop_offset = offset;
+    p.out_scale = static_cast<float>(static_cast<double>(vd) / (1.0 - static_cast<double>(dropout_p)));
+    switch (dtype * 2 + (D == 128 ? 1 : 0)) {
+      case FA_FP16 * 2 + 0: return launch<64, DT_FP16, false, MASK_DROPOUT>(q, k, v, p, stream, ds, 24, sched_override);
+      case FA_FP16 * 2 + 1: return launch<128, DT_FP16, false, MASK_DROPOUT>(q, k, v, p, stream, ds, 25, sched_override);
+      case FA_BF16 * 2 + 0: return launch<64, DT_BF16, false, MASK_DROPOUT>(q, k, v, p, stream, ds, 26, sched_override);
+      case FA_BF16 * 2 + 1: return launch<128, DT_BF16, false, MASK_DROPOUT>(q, k, v, p, stream, ds, 27, sched_override);
+      default: return FA_ERR_UNSUPPORTED;
+    }
+  }
   if (mask_type != 0) {
     // masked forwards: every key block in the causal / window range is
     // computed (the mask decides inside the blocks)
@@ -373,6 +395,14 @@ int fa_fwd_mask(const void* q, const void* k, const void* v, void* out, float* l
                      mask_type, mask_stride_b, mask_stride_h, mask_stride_q);
 }
 
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q, int N_k,
+                   int H, int H_kv, int D, float scale, int causal, int window_left, int dtype, float dropout_p,
+                   unsigned long long seed, unsigned offset, fa_stream_t stream) {
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, 1.f, 1.f, 1.f,
+                     reinterpret_cast<cudaStream_t>(stream), nullptr, 1, nullptr, 0, nullptr, 0, 0, 0, 0, dropout_p,
+                     seed, offset);
+}
+
 int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,
                 void* dv, void* dout, float* dlse, int B, int N_q, int N_k, int H, int D, float scale,
                 int causal, int window_left, int dtype, float q_descale, float k_descale,
@@ -441,6 +471,15 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* out, con
                fa_stream_t stream) {
   return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, H_kv, D, scale, causal, window_left,
                       dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int H_kv, int D,
+                   float scale, int causal, int window_left, int dtype, float dropout_p, unsigned long long seed,
+                   unsigned offset, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, H_kv, D, scale, causal, window_left,
+                      dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), dropout_p, seed,
+                      offset);
 }
 
 int fa_device_status(fa_stream_t stream, int* flags) {

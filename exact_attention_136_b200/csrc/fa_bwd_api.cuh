@@ -17,7 +17,7 @@ size_t bwd_workspace_bytes(int B, int Nq, int H, int D) {
 // query block), both after the prologue; one CTA per SM each (the dQ
 // kernel's shared-memory request is raised to keep a second CTA from
 // waiting on the first's tensor memory).
-template <int D, int DT>
+template <int D, int DT, bool DROP>
 int launch_bwd(const void* q, const void* k, const void* v, const void* dout, const BwdParams& p,
                cudaStream_t stream, DeviceState* ds, int bit) {
   using C = BwdCfg<D>;
@@ -31,27 +31,30 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dout, co
       encode_bnhd(&mdo, dout, tdt, 2, p.B, p.Nq, p.H, D, 64, 128))
     return FA_ERR_CUDA;
   if (!(ds->attr_set.load(std::memory_order_acquire) & (1u << bit))) {
-    if (cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+    if (cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D, DT, DROP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
       return FA_ERR_CUDA;
-    const int rc = set_smem_attr_once(ds, bit, fa_bwd_dq_kernel<D, DT>, DQ_SMEM);
+    const int rc = set_smem_attr_once(ds, bit, fa_bwd_dq_kernel<D, DT, DROP>, DQ_SMEM);
     if (rc != FA_OK) return rc;
   }
   const int64_t grid_kv = static_cast<int64_t>(p.nkb) * p.B * p.Hkv;
   const int64_t grid_q = static_cast<int64_t>(p.nqb) * p.B * p.H;
   if (grid_kv > 0x7fffffff || grid_q > 0x7fffffff) return FA_ERR_ARG;
-  fa_bwd_dkdv_kernel<D, DT><<<static_cast<int>(grid_kv), BWD_THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+  fa_bwd_dkdv_kernel<D, DT, DROP><<<static_cast<int>(grid_kv), BWD_THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  fa_bwd_dq_kernel<D, DT><<<static_cast<int>(grid_q), BWD_THREADS, DQ_SMEM, stream>>>(mq, mk, mv, mdo, p);
+  fa_bwd_dq_kernel<D, DT, DROP><<<static_cast<int>(grid_q), BWD_THREADS, DQ_SMEM, stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int backward(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
              void* dq, void* dk, void* dv, int B, int Nq, int Nk, int H, int Hkv, int D, float scale, int causal,
-             int window_left, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+             int window_left, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+             float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0) {
   int rc = validate(q, k, v, const_cast<void*>(out), B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
   if (rc != FA_OK) return rc;
   if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
+  if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_ARG;
+  const bool drop = dropout_p > 0.f;
   if ((Nq > 0 && (!dout || !lse || !dq)) || (Nk > 0 && (!dk || !dv))) return FA_ERR_ARG;
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
@@ -105,11 +108,23 @@ int backward(const void* q, const void* k, const void* v, const void* out, const
     p.nqb = (Nq + 127) / 128;
     p.wait_limit_ns = g_wait_limit_ns;
     p.status = ds->status;
-    switch (dtype * 2 + (D == 128 ? 1 : 0)) {
-      case FA_FP16 * 2 + 0: rc = launch_bwd<64, DT_FP16>(q, k, v, dout, p, stream, ds, 20); break;
-      case FA_FP16 * 2 + 1: rc = launch_bwd<128, DT_FP16>(q, k, v, dout, p, stream, ds, 21); break;
-      case FA_BF16 * 2 + 0: rc = launch_bwd<64, DT_BF16>(q, k, v, dout, p, stream, ds, 22); break;
-      case FA_BF16 * 2 + 1: rc = launch_bwd<128, DT_BF16>(q, k, v, dout, p, stream, ds, 23); break;
+    if (drop) {
+      // the forward's keep rule (fa_fwd_dropout) and 1 / (1 - p)
+      p.drop_threshold = static_cast<unsigned>(std::nearbyint(static_cast<double>(dropout_p) * 65536.0));
+      p.seed_lo = static_cast<unsigned>(seed & 0xffffffffull);
+      p.seed_hi = static_cast<unsigned>(seed >> 32);
+      p.drop_offset = offset;
+      p.drop_scale = static_cast<float>(1.0 / (1.0 - static_cast<double>(dropout_p)));
+    }
+    switch ((dtype * 2 + (D == 128 ? 1 : 0)) * 2 + (drop ? 1 : 0)) {
+      case (FA_FP16 * 2 + 0) * 2 + 0: rc = launch_bwd<64, DT_FP16, false>(q, k, v, dout, p, stream, ds, 20); break;
+      case (FA_FP16 * 2 + 1) * 2 + 0: rc = launch_bwd<128, DT_FP16, false>(q, k, v, dout, p, stream, ds, 21); break;
+      case (FA_BF16 * 2 + 0) * 2 + 0: rc = launch_bwd<64, DT_BF16, false>(q, k, v, dout, p, stream, ds, 22); break;
+      case (FA_BF16 * 2 + 1) * 2 + 0: rc = launch_bwd<128, DT_BF16, false>(q, k, v, dout, p, stream, ds, 23); break;
+      case (FA_FP16 * 2 + 0) * 2 + 1: rc = launch_bwd<64, DT_FP16, true>(q, k, v, dout, p, stream, ds, 28); break;
+      case (FA_FP16 * 2 + 1) * 2 + 1: rc = launch_bwd<128, DT_FP16, true>(q, k, v, dout, p, stream, ds, 29); break;
+      case (FA_BF16 * 2 + 0) * 2 + 1: rc = launch_bwd<64, DT_BF16, true>(q, k, v, dout, p, stream, ds, 30); break;
+      case (FA_BF16 * 2 + 1) * 2 + 1: rc = launch_bwd<128, DT_BF16, true>(q, k, v, dout, p, stream, ds, 31); break;
       default: return FA_ERR_UNSUPPORTED;
     }
     if (rc != FA_OK) return rc;

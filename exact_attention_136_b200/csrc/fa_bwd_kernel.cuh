@@ -51,6 +51,10 @@ struct BwdParams {
   int nqb;                  // query blocks per (batch, head)
   unsigned long long wait_limit_ns;
   int* status;
+  // dropout (DROP kernels): the forward's keep bits (keep_bits8 with these
+  // values) and 1 / (1 - p)
+  unsigned drop_threshold, seed_lo, seed_hi, drop_offset;
+  float drop_scale;
 };
 
 template <int D>
@@ -122,7 +126,7 @@ __device__ __forceinline__ void bwd_query_range(int jk, const BwdParams& p, int&
   if (jk * 128 >= p.Nk) i_hi = i_lo - 1;   // (not launched: the grid covers N_k)
 }
 
-template <int D, int DT>
+template <int D, int DT, bool DROP>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -355,11 +359,42 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
         pv[e] = pe;
       }
+      // dropout keep bits of this thread's key for its 64 queries (bit e:
+      // query q0 + 64 * half + e).  The generator gives 8 keys of one query
+      // per call, so in round m lane L draws query 8m + (L mod 8) for its
+      // 8-key group, and the 8 lanes of the group exchange bits
+      uint32_t keep[2] = {0u, 0u};
+      if constexpr (DROP) {
+        const int lane8 = lane & 7;
+        const uint32_t grp = static_cast<uint32_t>(jk * 128 + quad * 32 + sub * 16 + (lane & 8)) / 8u;
+        const uint32_t bh = static_cast<uint32_t>(b * p.H + hq);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t qq = static_cast<uint32_t>(q0 + half * 64 + 8 * m + lane8);
+          const uint32_t mine8 = keep_bits8(grp, qq, bh, p.drop_offset, p.seed_lo, p.seed_hi, p.drop_threshold);
+          uint32_t got8 = 0;
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const uint32_t v8 = __shfl_sync(0xffffffffu, mine8, (lane & ~7) + x);
+            got8 |= ((v8 >> lane8) & 1u) << x;
+          }
+          keep[m / 4] |= got8 << (8 * (m % 4));
+        }
+      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pw[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pw[e] = pack2<DT>(pv[c * 32 + 2 * e], pv[c * 32 + 2 * e + 1]);
+        for (int e = 0; e < 16; ++e) {
+          float p0 = pv[c * 32 + 2 * e], p1 = pv[c * 32 + 2 * e + 1];
+          if constexpr (DROP) {
+            // dV takes the kept probabilities, scaled by 1 / (1 - p)
+            const uint32_t kb = keep[c] >> (2 * e);
+            p0 = (kb & 1u) ? p0 * p.drop_scale : 0.f;
+            p1 = (kb & 2u) ? p1 * p.drop_scale : 0.f;
+          }
+          pw[e] = pack2<DT>(p0, p1);
+        }
         tmem_st_16x32bx2_x16<32>(tbase + lane_off + C::P_COL + c * 16, pw);
       }
       tmem_wait_st();
@@ -381,8 +416,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           const int ql = half * 64 + c * 16 + e;
-          const float d0 = pv[c * 16 + e] * (__uint_as_float(dpv[e]) - sh->delta[buf][ql]);
-          const float d1 = pv[c * 16 + e + 1] * (__uint_as_float(dpv[e + 1]) - sh->delta[buf][ql + 1]);
+          float g0 = __uint_as_float(dpv[e]), g1 = __uint_as_float(dpv[e + 1]);
+          if constexpr (DROP) {
+            // dP of the dropped forward: Z / (1 - p) times dO V^T
+            const uint32_t kb = keep[(c * 16 + e) / 32] >> ((c * 16 + e) % 32);
+            g0 = (kb & 1u) ? g0 * p.drop_scale : 0.f;
+            g1 = (kb & 2u) ? g1 * p.drop_scale : 0.f;
+          }
+          const float d0 = pv[c * 16 + e] * (g0 - sh->delta[buf][ql]);
+          const float d1 = pv[c * 16 + e + 1] * (g1 - sh->delta[buf][ql + 1]);
           dw[e / 2] = pack2<DT>(d0, d1);
         }
         // row r of dS^T, two 16-byte units of the 128-byte row, XOR-swizzled
@@ -453,7 +495,7 @@ struct DqHeader {
   int abort_flag;
 };
 
-template <int D, int DT>
+template <int D, int DT, bool DROP>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -617,6 +659,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         ok = false;
         break;
       }
+      // dropout keep bits of this row's keys k0 + 64 * half + [0, 64)
+      uint32_t keep[2] = {0u, 0u};
+      if constexpr (DROP) {
+        const uint32_t g0 = static_cast<uint32_t>(k0 + half * 64) / 8u;
+        const uint32_t bhq = static_cast<uint32_t>(b * p.H + h);
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          keep[g / 4] |= keep_bits8(g0 + g, static_cast<uint32_t>(q), bhq, p.drop_offset, p.seed_lo, p.seed_hi,
+                                    p.drop_threshold)
+                         << (8 * (g % 4));
+      }
       tc_fence_after();
       // the whole half row of S (keys half * 64 + [0, 64)) before any dS store
       float pv[64];
@@ -640,9 +693,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tmem_wait_ld();
         uint32_t dw[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2)
-          dw[e / 2] = pack2<DT>(pv[c * 16 + e] * (__uint_as_float(dpv[e]) - dlt),
-                                pv[c * 16 + e + 1] * (__uint_as_float(dpv[e + 1]) - dlt));
+        for (int e = 0; e < 16; e += 2) {
+          float g0 = __uint_as_float(dpv[e]), g1 = __uint_as_float(dpv[e + 1]);
+          if constexpr (DROP) {
+            // dP of the dropped forward: Z / (1 - p) times dO V^T
+            const uint32_t kb = keep[(c * 16 + e) / 32] >> ((c * 16 + e) % 32);
+            g0 = (kb & 1u) ? g0 * p.drop_scale : 0.f;
+            g1 = (kb & 2u) ? g1 * p.drop_scale : 0.f;
+          }
+          dw[e / 2] = pack2<DT>(pv[c * 16 + e] * (g0 - dlt), pv[c * 16 + e + 1] * (g1 - dlt));
+        }
         tmem_st_16x32bx2_x8<32>(tbase + lane_off + C::P_COL + c * 8, dw);
       }
       tmem_wait_st();

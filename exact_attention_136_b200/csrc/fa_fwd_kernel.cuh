@@ -50,8 +50,9 @@ namespace fa {
 
 enum : int { DT_FP16 = 0, DT_BF16 = 1, DT_E4M3 = 2 };
 
-// attention-mask kinds of the masked kernel instantiations
-enum : int { MASK_NONE = 0, MASK_BOOL = 1, MASK_ADD = 2 };
+// kernel instantiations with a mask on the scores or the probabilities:
+// an attention mask (boolean, additive) or dropout of the probabilities
+enum : int { MASK_NONE = 0, MASK_BOOL = 1, MASK_ADD = 2, MASK_DROPOUT = 3 };
 
 // device status word: bit flags of the role whose wait timed out
 enum : int {
@@ -95,6 +96,12 @@ struct FwdParams {
   const void* mask;
   long long mask_sb, mask_sh, mask_sq;
   float mask_scale;    // 1 / (scale * q_descale * k_descale)
+  // dropout (MASK_DROPOUT kernels): key j of row i of (batch b, query head
+  // h) is kept when a 16-bit value of Philox4x32-10 at counter
+  // (j / 8, i, b * H + h, drop_offset) under key (seed_lo, seed_hi) is at
+  // least drop_threshold; out_scale already holds the 1 / (1 - p)
+  unsigned drop_threshold;
+  unsigned seed_lo, seed_hi, drop_offset;
 };
 
 // Exponentials taken on the FMA pipe (see Cfg::EMU_FROM): pairs i >= this of
@@ -695,6 +702,41 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
   if (!mbar_wait(smem_u32(&sh->mma_done), 0, lim)) record_error(sh, p, ST_TIMEOUT_DRAIN);
 }
 
+// ------------------------------------------------------------------ dropout
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel Random
+// Numbers: As Easy as 1, 2, 3", SC 2011): each round multiplies counter
+// words 0 and 2 by two fixed odd constants and mixes the high and low
+// halves of the products with words 1 and 3 and the key; the key is bumped
+// by two Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// Keep bits of 8 consecutive keys 8g .. 8g+7 of one row: bit e for key
+// 8g + e, from the 16-bit halves of the four output words (low half first).
+__device__ __forceinline__ uint32_t keep_bits8(uint32_t g, uint32_t row, uint32_t bh, uint32_t offset,
+                                               uint32_t seed_lo, uint32_t seed_hi, uint32_t t) {
+  const uint4 w = philox4x32_10(make_uint4(g, row, bh, offset), seed_lo, seed_hi);
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+  uint32_t bits = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    bits |= ((words[e] & 0xffffu) >= t ? 1u : 0u) << (2 * e);
+    bits |= ((words[e] >> 16) >= t ? 1u : 0u) << (2 * e + 1);
+  }
+  return bits;
+}
+
 // ------------------------------------------------------------------ softmax
 template <int DT>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -791,8 +833,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // (different only for e4m3, whose 3-bit mantissa would otherwise bias O).
 // With EMULATE (blocks without masked keys), pairs i >= EMU_FROM of every 8
 // take exp2_poly2 on the FMA pipe instead of MUFU.
-template <int DT, bool EMULATE, int Q0, int NQ, int EMU_FROM = 8, int EMU_DEG = 3>
-__device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_mref, uint32_t p_addr) {
+template <int DT, bool EMULATE, int Q0, int NQ, int EMU_FROM = 8, int EMU_DEG = 3, bool DROP = false>
+__device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_mref, uint32_t p_addr,
+                                           const uint32_t* keep = nullptr) {
   const float2 cc2 = make_float2(cc, cc);
   const float2 nm2 = make_float2(neg_mref, neg_mref);
   float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -812,6 +855,12 @@ __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_m
         e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       }
       acc[i & 1] = __fadd2_rn(acc[i & 1], e);
+      if constexpr (DROP) {
+        // dropped keys add nothing to P V (the row sum keeps them)
+        const uint32_t kb = keep[c / 32] >> (c % 32);
+        e.x = (kb & 1u) ? e.x : 0.f;
+        e.y = (kb & 2u) ? e.y : 0.f;
+      }
       if constexpr (DT == DT_E4M3) {
         if (i & 1) {
           pw[i / 2] = pack4_e4m3(prev.x, prev.y, e.x, e.y);
@@ -906,9 +955,11 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     float lq = 0.f;             // ... of the stored P values (differs for e4m3)
     // this thread's mask row (its 64 keys of each block start at key
     // k0 + 64 * half); rows past N_q read nothing
+    constexpr bool ATTN_MASK = MASK == MASK_BOOL || MASK == MASK_ADD;
+    constexpr bool DROP = MASK == MASK_DROPOUT;
     constexpr int MES = MASK == MASK_BOOL ? 1 : 2;   // mask element bytes
     const uint8_t* mask_row = nullptr;
-    if constexpr (MASK != MASK_NONE) {
+    if constexpr (ATTN_MASK) {
       if (row_ok)
         mask_row = static_cast<const uint8_t*>(p.mask) +
                    (static_cast<int64_t>(w.b) * p.mask_sb + static_cast<int64_t>(w.h) * p.mask_sh +
@@ -922,9 +973,9 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
                              (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
       // the mask values of this block, loaded while S is computed (16-byte
       // chunks that start at or past N_k are not read)
-      constexpr int MCHUNKS = MASK == MASK_NONE ? 1 : HALF_N * MES / 16;
+      constexpr int MCHUNKS = ATTN_MASK ? HALF_N * MES / 16 : 1;
       uint4 mk[MCHUNKS];
-      if constexpr (MASK != MASK_NONE) {
+      if constexpr (ATTN_MASK) {
 #pragma unroll
         for (int c = 0; c < MCHUNKS; ++c) {
           const int key = k0 + half * HALF_N + c * (16 / MES);
@@ -932,6 +983,18 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
                       ? __ldg(reinterpret_cast<const uint4*>(mask_row + static_cast<int64_t>(k0) * MES) + c)
                       : make_uint4(0u, 0u, 0u, 0u);
         }
+      }
+      // dropout keep bits of this thread's keys (bit c: key k0 + 64 * half + c),
+      // generated while S is computed
+      uint32_t keep[2] = {0u, 0u};
+      if constexpr (DROP) {
+        const uint32_t g0 = static_cast<uint32_t>(k0 + half * HALF_N) / 8u;
+        const uint32_t bh = static_cast<uint32_t>(w.b * p.H + w.h);
+#pragma unroll
+        for (int g = 0; g < HALF_N / 8; ++g)
+          keep[g / 4] |= keep_bits8(g0 + g, static_cast<uint32_t>(row), bh, p.drop_offset, p.seed_lo, p.seed_hi,
+                                    p.drop_threshold)
+                         << (8 * (g % 4));
       }
       bool got = mbar_wait(smem_u32(&sh->s_full[t]), s_waits & 1u, p.wait_limit_ns);
       got = __all_sync(0xffffffffu, got);
@@ -998,8 +1061,8 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       // chunks of 16 scores exponentiated before the first hand-over: with
       // the split hand-over, P over keys k with k mod 64 < 32 goes first
       constexpr int NQ0 = C::PSPLIT ? 2 : 4;
-      float2 lsum = need_mask ? exp_half<DT, false, 0, NQ0>(s, cc, -mref, p_addr)
-                              : exp_half<DT, true, 0, NQ0, C::EMU_FROM, C::EMU_DEG>(s, cc, -mref, p_addr);
+      float2 lsum = need_mask ? exp_half<DT, false, 0, NQ0, 8, 3, DROP>(s, cc, -mref, p_addr, keep)
+                              : exp_half<DT, true, 0, NQ0, C::EMU_FROM, C::EMU_DEG, DROP>(s, cc, -mref, p_addr, keep);
       float alpha = 1.f;
       if (warp_rescale) alpha = (m_cand == -INFINITY) ? 1.f : ex2_approx(m_old - m_cand);
       // O rescale of this thread's half row (only when some row of this warp
@@ -1028,8 +1091,8 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
         tc_fence_before();
         mbar_arrive(smem_u32(&sh->p_half[t]));
         FA_TRACE(t, 12, j);
-        const float2 ls2 = need_mask ? exp_half<DT, false, 2, 2>(s, cc, -mref, p_addr)
-                                     : exp_half<DT, true, 2, 2, C::EMU_FROM, C::EMU_DEG>(s, cc, -mref, p_addr);
+        const float2 ls2 = need_mask ? exp_half<DT, false, 2, 2, 8, 3, DROP>(s, cc, -mref, p_addr, keep)
+                                     : exp_half<DT, true, 2, 2, C::EMU_FROM, C::EMU_DEG, DROP>(s, cc, -mref, p_addr, keep);
         lsum = make_float2(lsum.x + ls2.x, lsum.y + ls2.y);
       }
       FA_TRACE(t, 4, j);

@@ -15,9 +15,12 @@ Readings (the pages leave these open):
   ``right`` says (the page pairs causal=True with a two-sided window, which
   contradict each other; causal wins).  Without causal only ``right = -1``
   (no right bound) is available.
-- ``dropout_p`` must be 0: the pages give no random-number specification for
-  dropout, and this library does not implement it.
-- The backward takes fp16 / bf16 inputs with as many K/V heads as query heads.
+- ``dropout_p``: the usual attention dropout, each softmax probability kept
+  with probability 1 - p and scaled by 1 / (1 - p) (fa_fwd_dropout).  The
+  pages name no random generator; each call draws a 64-bit seed from
+  torch's default generator (so ``torch.manual_seed`` makes runs
+  repeatable) and the backward redraws the same keep bits from it.
+- The backward takes fp16 / bf16 inputs; K/V may have fewer heads than Q.
 """
 
 from __future__ import annotations
@@ -42,10 +45,14 @@ class _FlashAttn(torch.autograd.Function):
     """O = attention(q, k, v); the backward recomputes from O and the LSE."""
 
     @staticmethod
-    def forward(ctx, q, k, v, scale, causal, window_left):
-        out, lse = forward(q, k, v, scale, causal, window_left)
+    def forward(ctx, q, k, v, scale, causal, window_left, dropout_p, seed):
+        if dropout_p:
+            out, lse = forward(q, k, v, scale, causal, window_left, dropout_p=dropout_p, seed=seed)
+        else:
+            out, lse = forward(q, k, v, scale, causal, window_left)
         ctx.save_for_backward(q, k, v, out, lse)
         ctx.scale, ctx.causal, ctx.window_left = scale, causal, window_left
+        ctx.dropout_p, ctx.seed = dropout_p, seed
         ctx.mark_non_differentiable(lse)
         return out, lse
 
@@ -54,8 +61,12 @@ class _FlashAttn(torch.autograd.Function):
         if dlse is not None and bool(torch.any(dlse != 0)):
             raise NotImplementedError("gradients through the returned LSE are not supported")
         q, k, v, out, lse = ctx.saved_tensors
-        dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left)
-        return dq, dk, dv, None, None, None
+        if ctx.dropout_p:
+            dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left,
+                                  dropout_p=ctx.dropout_p, seed=ctx.seed)
+        else:
+            dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left)
+        return dq, dk, dv, None, None, None, None, None
 
 
 def flash_attn_func(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dropout_p: float = 0.0,
@@ -64,15 +75,21 @@ def flash_attn_func(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dropout_p
     """The pages' flash_attn_func on [batch, seqlen, nheads, headdim] tensors.
 
     Returns O (and LSE [batch, nheads, seqlen_q], natural log, with
-    return_lse).  Differentiable in q, k, v (fp16 / bf16, equal head counts).
+    return_lse).  Differentiable in q, k, v (fp16 / bf16).  dropout_p > 0
+    drops attention probabilities (a fresh seed from torch's default
+    generator per call).
     """
-    if dropout_p != 0.0:
-        raise NotImplementedError("dropout_p must be 0: no dropout (the pages specify no random generator)")
+    dropout_p = float(dropout_p)
+    if not (0.0 <= dropout_p < 1.0):
+        raise ValueError("dropout_p must be in [0, 1)")
     wl = _window_left(bool(causal), window_size)
     scale = float(softmax_scale) if softmax_scale is not None else q.shape[-1] ** -0.5
+    seed = int(torch.randint(0, 2 ** 62, (1,)).item()) if dropout_p > 0.0 else 0
     needs_grad = torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v))
     if needs_grad:
-        out, lse = _FlashAttn.apply(q, k, v, scale, bool(causal), wl)
+        out, lse = _FlashAttn.apply(q, k, v, scale, bool(causal), wl, dropout_p, seed)
+    elif dropout_p > 0.0:
+        out, lse = forward(q, k, v, scale, bool(causal), wl, dropout_p=dropout_p, seed=seed)
     else:
         out, lse = forward(q, k, v, scale, bool(causal), wl)
     return (out, lse) if return_lse else out

@@ -158,6 +158,30 @@ int fa_fwd_mask(const void* q, const void* k, const void* v, void* out, float* l
                 long long mask_stride_q, fa_stream_t stream);
 
 /*
+ * fa_fwd_dropout -- the forward with dropout of the attention probabilities
+ * (the dropout_p argument of the pages' flash_attn_func, Flash Attention |
+ * Hermes Skill, Workflow 2, Step 2, which gives no definition; this
+ * library's reading): after the softmax, each probability P_ij is kept with
+ * probability 1 - p and divided by 1 - p, or dropped, independently:
+ *     O_i = sum_j (Z_ij / (1 - p)) P_ij V_j,   LSE as without dropout.
+ * Z_ij = 1 when the 16-bit value for key j of row i of (batch b, query head
+ * h) is >= round(p * 65536) (ties to even; p taken as the float given).
+ * The values come from Philox4x32-10 (Salmon et al., "Parallel Random
+ * Numbers: As Easy as 1, 2, 3", SC 2011) at counter
+ * (j / 8, i, b * H + h, offset) with key (seed mod 2^32, seed / 2^32): the
+ * (j mod 2) half (low half first) of output word (j mod 8) / 2.  Calls with
+ * the same seed and offset drop the same keys (fa_bwd_dropout needs them);
+ * change offset (or seed) for a new mask.
+ *   Arguments as fa_fwd_gqa (FA_FP16 / FA_BF16 only) plus dropout_p in
+ * [0, 1) (0 = plain forward), seed and offset.  Returns FA_ERR_ARG for p out
+ * of range, FA_ERR_UNSUPPORTED for FA_E4M3, else as fa_fwd_gqa.
+ */
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* out, float* lse,
+                   int B, int N_q, int N_k, int H, int H_kv, int D, float scale, int causal,
+                   int window_left, int dtype, float dropout_p, unsigned long long seed,
+                   unsigned offset, fa_stream_t stream);
+
+/*
  * fa_fwd_host -- the same forward on HOST buffers: copies q, k, v from host
  * to the caller's device buffers dq, dk, dv, runs fa_fwd / fa_fwd_fp8 into
  * dout / dlse, and copies out (and lse, when both lse and dlse are non-NULL)
@@ -239,6 +263,21 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* out, con
                const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H,
                int H_kv, int D, float scale, int causal, int window_left, int dtype,
                void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fa_bwd_dropout -- fa_bwd_gqa for the forward of fa_fwd_dropout: the same
+ * dropout_p, seed and offset redraw the forward's keep bits, and the
+ * gradients are those of O = (Z / (1 - p) * P) V: dV = (Z P / (1 - p))^T dO,
+ * dP = Z / (1 - p) * (dO V^T), dS = P * (dP - rowsum(dO * O)), dQ, dK as
+ * fa_bwd.  out and lse are the dropout forward's.  dropout_p = 0 is fa_bwd_gqa.
+ * Workspace, kernels and return values as fa_bwd; FA_ERR_ARG for p outside
+ * [0, 1).
+ */
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                   const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H,
+                   int H_kv, int D, float scale, int causal, int window_left, int dtype,
+                   float dropout_p, unsigned long long seed, unsigned offset, void* workspace,
+                   size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fa_device_status -- synchronises `stream`, then reads and clears the

@@ -65,7 +65,8 @@ def compare(out, lse, ref_o, ref_l, rows=None):
     return d_o, d_l
 
 
-def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, unit_roundoff):
+def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, unit_roundoff, dropout_p=0.0,
+                    seed=0, offset=0):
     """Per-element bounds (dq, dk, dv; shaped like q, k, v) on how far a
     backward computed the way the CUDA path does can be from the exact
     gradients, all arrays float64 numpy.
@@ -83,14 +84,18 @@ def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, u
     each plus 1e-5 of the matching sum of absolute products (fp32 sums).
     With fewer K/V heads than query heads (query head h reads K/V head
     h // (H / H_kv)) the dK and dV bounds add up over each group's heads.
+    With dropout (keep bits Z) the same steps apply to the dropped forward:
+    P in dV becomes Z P / (1 - p) and dP becomes Z dP / (1 - p).
     """
+    from oracle import dropout_keep
     from oracle import attention_ref
     u = float(unit_roundoff)
     B, n_q, H, D = q.shape
     n_k, h_kv = k.shape[1], k.shape[2]
     group = H // h_kv
     bq, bk, bv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
-    o_ref, l_ref, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True)
+    o_ref, l_ref, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True, dropout_p=dropout_p,
+                                        seed=seed, offset=offset)
     for b in range(B):
         for h in range(H):
             hk = h // group
@@ -100,12 +105,17 @@ def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, u
             qq = q[b, :, h, :]
             kk = k[b, :, hk, :]
             dp = g @ vv.T
+            pd = p
+            if dropout_p > 0.0:
+                z = dropout_keep(seed, offset, b, h, H, np.arange(n_q), n_k, dropout_p) / (1.0 - dropout_p)
+                pd = z * p
+                dp = z * dp
             ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
             l_diff = np.where(np.isfinite(l_ref[b, h]), np.abs(lse_used[b, h] - l_ref[b, h]), 0.0)
             e1 = (1.01 * l_diff + 1e-6)[:, None]                       # per query row
             e_d = (np.abs(g) * np.abs(o_used[b, :, h, :] - o_ref[b, :, h, :])).sum(axis=1) + \
                 1e-6 * np.abs(g * o_ref[b, :, h, :]).sum(axis=1)
-            bv[b, :, hk, :] += ((u + e1) * p).T @ np.abs(g) + 1e-5 * p.T @ np.abs(g)
+            bv[b, :, hk, :] += ((u + e1) * pd).T @ np.abs(g) + 1e-5 * pd.T @ np.abs(g)
             d_ds = (u + e1) * (1 + u) * np.abs(ds) + (1 + u) * p * e_d[:, None]
             bk[b, :, hk, :] += scale * (d_ds.T @ np.abs(qq) + 1e-5 * np.abs(ds).T @ np.abs(qq))
             bq[b, :, h, :] = scale * (d_ds @ np.abs(kk) + 1e-5 * np.abs(ds) @ np.abs(kk))

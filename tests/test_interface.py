@@ -16,15 +16,16 @@ from oracle import attention_backward_ref, attention_ref
 def oracle_backend(monkeypatch):
     calls = []
 
-    def fwd(q, k, v, scale, causal, window_left):
-        calls.append(("fwd", scale, causal, window_left))
-        o, l = attention_ref(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), scale, causal, window_left)
+    def fwd(q, k, v, scale, causal, window_left, dropout_p=0.0, seed=None, offset=0):
+        calls.append(("fwd", scale, causal, window_left) + ((dropout_p, seed, offset) if dropout_p else ()))
+        o, l = attention_ref(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), scale, causal, window_left,
+                             dropout_p=dropout_p, seed=seed or 0, offset=offset)
         return torch.from_numpy(o), torch.from_numpy(l)
 
-    def bwd(q, k, v, out, lse, dout, scale, causal, window_left):
-        calls.append(("bwd", scale, causal, window_left))
+    def bwd(q, k, v, out, lse, dout, scale, causal, window_left, dropout_p=0.0, seed=None, offset=0):
+        calls.append(("bwd", scale, causal, window_left) + ((dropout_p, seed, offset) if dropout_p else ()))
         g = attention_backward_ref(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), dout.numpy(), scale,
-                                   causal, window_left)
+                                   causal, window_left, dropout_p=dropout_p, seed=seed or 0, offset=offset)
         return tuple(torch.from_numpy(x) for x in g)
 
     monkeypatch.setattr(itf, "forward", fwd)
@@ -75,8 +76,9 @@ def test_no_grad_path_and_lse(oracle_backend):
 
 def test_rejected_arguments(oracle_backend):
     q = torch.zeros(1, 4, 1, 8, dtype=torch.float64)
-    with pytest.raises(NotImplementedError):
-        itf.flash_attn_func(q, q, q, dropout_p=0.1)
+    for bad_p in (-0.1, 1.0):
+        with pytest.raises(ValueError):
+            itf.flash_attn_func(q, q, q, dropout_p=bad_p)
     with pytest.raises(NotImplementedError):
         itf.flash_attn_func(q, q, q, causal=False, window_size=(2, 2))
     with pytest.raises(ValueError):
@@ -89,3 +91,32 @@ def test_causal_two_sided_window_reads_as_left_window(oracle_backend):
     q = torch.zeros(1, 4, 1, 8, dtype=torch.float64)
     itf.flash_attn_func(q, q, q, causal=True, window_size=(256, 256))
     assert oracle_backend == [("fwd", 8 ** -0.5, True, 256)]
+
+
+def test_dropout_gradients_and_seed_plumbing(oracle_backend):
+    """dropout_p > 0: the forward and the backward get the same seed (drawn
+    from torch's default generator), and the gradients are torch autograd's
+    of softmax * Z / (1 - p) @ V with the oracle's keep bits Z."""
+    from oracle import dropout_keep
+    g = torch.Generator().manual_seed(9)
+    B, n, H, D, p = 1, 10, 2, 4, 0.3
+    q, k, v = (torch.randn(B, n, H, D, generator=g, dtype=torch.float64, requires_grad=True) for _ in range(3))
+    do = torch.randn(B, n, H, D, generator=g, dtype=torch.float64)
+    torch.manual_seed(1234)
+    out = itf.flash_attn_func(q, k, v, dropout_p=p, causal=True)
+    out.backward(do)
+    (_, _, _, _, p_f, seed_f, off_f), (_, _, _, _, p_b, seed_b, off_b) = oracle_backend
+    assert (p_f, seed_f, off_f) == (p_b, seed_b, off_b) == (p, seed_f, 0)
+    # the same torch seed gives the same dropout seed
+    torch.manual_seed(1234)
+    again = itf.flash_attn_func(q.detach(), k.detach(), v.detach(), dropout_p=p, causal=True)
+    assert oracle_backend[-1][5] == seed_f and torch.equal(again, out.detach())
+    q2, k2, v2 = (t.detach().clone().requires_grad_() for t in (q, k, v))
+    s = torch.einsum("bihd,bjhd->bhij", q2, k2) * D ** -0.5
+    s = s.masked_fill(~torch.tril(torch.ones(n, n, dtype=torch.bool)), float("-inf"))
+    z = torch.stack([torch.from_numpy(dropout_keep(seed_f, 0, 0, h, H, np.arange(n), n, p)) for h in range(H)])[None]
+    ref = torch.einsum("bhij,bjhd->bihd", torch.softmax(s, dim=-1) * z / (1 - p), v2)
+    ref.backward(do)
+    assert torch.allclose(out, ref, atol=1e-12)
+    for a, b in ((q.grad, q2.grad), (k.grad, k2.grad), (v.grad, v2.grad)):
+        assert torch.allclose(a, b, atol=1e-12)

@@ -38,6 +38,8 @@ SIGNATURES = {
     "fa_fwd_mask": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                              _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp, _c_int,
                              ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, _vp]),
+    "fa_fwd_varlen": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                               _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
     "fa_fwd_dropout": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _c_float, _c_int, _c_int, _c_int, _c_float, ctypes.c_ulonglong, ctypes.c_uint, _vp]),
     "fa_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,

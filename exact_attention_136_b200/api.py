@@ -215,6 +215,44 @@ def _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, 
     return out, lse
 
 
+def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                   cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int, scale: Optional[float] = None,
+                   causal: bool = False, window_left: int = -1, descales=(1.0, 1.0, 1.0),
+                   stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Attention over a packed batch of sequences (fa_fwd_varlen): q [total_q,
+    H, D], k, v [total_k, H_kv, D]; sequence b owns rows cu_seqlens_q[b] ..
+    cu_seqlens_q[b+1] and keys cu_seqlens_k[b] .. cu_seqlens_k[b+1] (int32 CUDA
+    tensors of B + 1 entries).  Returns (out [total_q, H, D], lse [H, total_q])."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor [total, heads, headdim]")
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _DT:
+        raise ValueError("q, k, v must share one dtype: float16, bfloat16 or float8_e4m3fn")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if not t.is_cuda or t.dtype != torch.int32 or t.dim() != 1 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 >= 2 entries")
+    total_q, H, D = q.shape
+    total_k, h_kv = k.shape[0], k.shape[1]
+    if v.shape != k.shape or k.shape[2] != D or h_kv < 1 or H % h_kv != 0:
+        raise ValueError("k and v must be [total_k, H_kv, D] with H a multiple of H_kv")
+    B = cu_seqlens_q.numel() - 1
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out_dtype = torch.float16 if q.dtype == torch.float16 else torch.bfloat16
+    out = torch.empty((total_q, H, D), dtype=out_dtype, device=q.device)
+    lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        rc = _lib.lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                      cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+                                      int(max_seqlen_k), total_q, total_k, H, h_kv, D, scale, int(bool(causal)),
+                                      int(window_left), _DT[q.dtype], float(descales[0]), float(descales[1]),
+                                      float(descales[2]), s.cuda_stream)
+    _lib.check(rc, "fa_fwd_varlen")
+    return out, lse
+
+
 def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale: float, k_descale: float,
                 v_descale: float, scale: Optional[float] = None, causal: bool = False,
                 window_left: int = -1, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,

@@ -128,9 +128,12 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
                                   : DT == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUtensorMap mq, mk, mv;
-  if (encode_bnhd(&mq, q, tdt, C::ES, p.B, p.Nq, p.H, D, C::BOX_INNER, BLOCK_M) ||
-      encode_bnhd(&mk, k, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N) ||
-      encode_bnhd(&mv, v, tdt, C::ES, p.B, p.Nk, p.Hkv, D, C::BOX_INNER, BLOCK_N))
+  // packed variable-length batches: one batch of total_q rows / total_k keys
+  const int mb = p.cu_q ? 1 : p.B;
+  const int mnq = p.cu_q ? p.total_q : p.Nq, mnk = p.cu_q ? p.total_k : p.Nk;
+  if (encode_bnhd(&mq, q, tdt, C::ES, mb, mnq, p.H, D, C::BOX_INNER, BLOCK_M) ||
+      encode_bnhd(&mk, k, tdt, C::ES, mb, mnk, p.Hkv, D, C::BOX_INNER, BLOCK_N) ||
+      encode_bnhd(&mv, v, tdt, C::ES, mb, mnk, p.Hkv, D, C::BOX_INNER, BLOCK_N))
     return FA_ERR_CUDA;
   if (!(ds->attr_set.load(std::memory_order_acquire) & (1u << bit))) {
     // The per-role register split (setmaxnreg) redistributes the registers
@@ -184,8 +187,12 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
             float vd, cudaStream_t stream, unsigned* sched_override = nullptr, int splits = 1,
             void* workspace = nullptr, size_t workspace_bytes = 0, const void* mask = nullptr,
             int mask_type = 0, long long mask_sb = 0, long long mask_sh = 0, long long mask_sq = 0,
-            float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0) {
-  int rc = validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
+            float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0, const int* cu_q = nullptr,
+            const int* cu_k = nullptr, int total_q = 0, int total_k = 0) {
+  // (packed batches are validated by fa_fwd_varlen, with N_q and N_k the
+  // longest sequences; here only their totals address the tensors)
+  int rc = cu_q ? validate(q, k, v, out, 1, total_q, total_k, H, D, scale, causal, window_left, dtype, Hkv)
+                : validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
   if (rc != FA_OK) return rc;
   if (splits < 1) return FA_ERR_ARG;
   // dropout: 0 <= p < 1, 16-bit inputs, not combined with a mask or a split key range
@@ -213,11 +220,17 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
       (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
        workspace_bytes < splitkv_workspace_bytes(B, Nq, H, D, used_splits)))
     return FA_ERR_ARG;
-  if (Nq == 0) return FA_OK;
+  if (cu_q ? total_q == 0 : Nq == 0) return FA_OK;
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc != FA_OK) return rc;
-  if (Nk == 0) {
+  if (cu_q ? total_k == 0 : Nk == 0) {
+    // no keys anywhere: O = 0, LSE = -inf ([H, total_q] for packed batches,
+    // the same layout as one batch of total_q rows)
+    if (cu_q) {
+      B = 1;
+      Nq = total_q;
+    }
     const int threads = 256;
     const int64_t rows = static_cast<int64_t>(B) * Nq * H;
     const int blocks = static_cast<int>(rows / threads + 1 < 4096 ? rows / threads + 1 : 4096);
@@ -266,6 +279,10 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   }
   p.wait_limit_ns = g_wait_limit_ns;
   p.status = ds->status;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
   p.mask = mask;
   p.mask_sb = mask_sb;
   p.mask_sh = mask_sh;
@@ -401,6 +418,23 @@ int fa_fwd_dropout(const void* q, const void* k, const void* v, void* out, float
   return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, 1.f, 1.f, 1.f,
                      reinterpret_cast<cudaStream_t>(stream), nullptr, 1, nullptr, 0, nullptr, 0, 0, 0, 0, dropout_p,
                      seed, offset);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int H,
+                  int H_kv, int D, float scale, int causal, int window_left, int dtype, float q_descale,
+                  float k_descale, float v_descale, fa_stream_t stream) {
+  if (B < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return FA_ERR_ARG;
+  if (!cu_seqlens_q || !cu_seqlens_k || (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return FA_ERR_ARG;
+  if ((total_q > 0 && max_seqlen_q < 1) || max_seqlen_q > total_q || max_seqlen_k > total_k) return FA_ERR_ARG;
+  // the work units cover max_seqlen_q rows of every sequence
+  const int64_t units = static_cast<int64_t>((max_seqlen_q + 2 * fa::BLOCK_M - 1) / (2 * fa::BLOCK_M)) * B * H;
+  if (units > 0x7fffffff) return FA_ERR_ARG;
+  return fa::forward(q, k, v, out, lse, B, max_seqlen_q, max_seqlen_k, H, H_kv, D, scale, causal, window_left, dtype,
+                     q_descale, k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream), nullptr, 1, nullptr, 0,
+                     nullptr, 0, 0, 0, 0, 0.f, 0, 0, cu_seqlens_q, cu_seqlens_k, total_q, total_k);
 }
 
 int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,

@@ -102,6 +102,13 @@ struct FwdParams {
   // least drop_threshold; out_scale already holds the 1 / (1 - p)
   unsigned drop_threshold;
   unsigned seed_lo, seed_hi, drop_offset;
+  // packed variable-length batches (cu_q non-null): sequence b holds query
+  // rows [cu_q[b], cu_q[b+1]) of q / out ([total_q, H, D]) and keys
+  // [cu_k[b], cu_k[b+1]) of k / v ([total_k, H_kv, D]); LSE is [H, total_q];
+  // N_q is then the longest sequence (it sizes the work units)
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
 };
 
 // Exponentials taken on the FMA pipe (see Cfg::EMU_FROM): pairs i >= this of
@@ -180,12 +187,16 @@ static_assert(sizeof(SharedHeader) <= HEADER_BYTES, "header");
 
 // One 128-row query tile of a work unit and its key-block range.
 struct Tile {
-  int b, h, qs;    // batch, head, first query row
+  int b, h, qs;    // batch (sequence), head, first query row (within the sequence)
   int hk;          // key/value head of this query head
   int lo, hi;      // inclusive key-block range
   int split;       // key-range slice (0 when not split)
-  bool rows;       // tile has rows (qs < N_q)
+  bool rows;       // tile has rows (qs < nq)
   bool valid;      // ... and at least one key block
+  int nq, nk;      // the sequence's query rows and keys
+  int qrow0, krow0, tb;   // TMA row of its first query / key, and TMA batch coordinate
+  int64_t orow0;   // out row (of [rows, H, D]) of its first query
+  int64_t lse0;    // LSE element of its first query
 };
 
 // Work-unit order.  Units are numbered group by group, a group being
@@ -209,21 +220,42 @@ __device__ __forceinline__ Tile get_tile(int u, int split, int t, const FwdParam
   w.h = bh - w.b * p.H;
   w.hk = w.h / p.qpk;
   w.qs = m * (2 * BLOCK_M) + t * BLOCK_M;
-  w.rows = w.qs < p.Nq;
-  const int qe = min(w.qs + BLOCK_M - 1, p.Nq - 1);
+  if (p.cu_q) {
+    // a packed sequence: its rows and keys, clamped into the packed tensors
+    const int q_start = min(max(__ldg(p.cu_q + w.b), 0), p.total_q);
+    const int k_start = min(max(__ldg(p.cu_k + w.b), 0), p.total_k);
+    w.nq = min(max(__ldg(p.cu_q + w.b + 1), q_start), p.total_q) - q_start;
+    w.nk = min(max(__ldg(p.cu_k + w.b + 1), k_start), p.total_k) - k_start;
+    w.qrow0 = q_start;
+    w.krow0 = k_start;
+    w.tb = 0;
+    w.orow0 = q_start;
+    w.lse0 = static_cast<int64_t>(w.h) * p.total_q + q_start;
+  } else {
+    w.nq = p.Nq;
+    w.nk = p.Nk;
+    w.qrow0 = 0;
+    w.krow0 = 0;
+    w.tb = w.b;
+    w.orow0 = static_cast<int64_t>(w.b) * p.Nq;
+    w.lse0 = (static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq;
+  }
+  w.rows = w.qs < w.nq;
+  const int qe = min(w.qs + BLOCK_M - 1, w.nq - 1);
   w.lo = p.window_left >= 0 ? max(0, w.qs - p.window_left) / BLOCK_N : 0;
-  w.hi = p.causal ? min(qe, p.Nk - 1) / BLOCK_N : (p.Nk - 1) / BLOCK_N;
+  w.hi = p.causal ? min(qe, w.nk - 1) / BLOCK_N : (w.nk - 1) / BLOCK_N;
   if (SPLIT) {
     w.lo = max(w.lo, w.split * p.split_blocks);
     w.hi = min(w.hi, (w.split + 1) * p.split_blocks - 1);
   }
-  w.valid = w.rows && p.Nk > 0 && w.lo <= w.hi;
+  w.valid = w.rows && w.nk > 0 && w.lo <= w.hi;
   return w;
 }
 
 // Both tiles of a work unit and the union of their key-block ranges.
 struct Unit {
   int b, h, hk, q0;
+  int qrow0, krow0, tb;   // TMA row of the sequence's first query / key, TMA batch coordinate
   int lo[2], hi[2];
   bool valid[2];
   int jlo, jhi;    // empty (jhi < 0) when neither tile has work
@@ -238,6 +270,9 @@ __device__ __forceinline__ Unit get_unit(int u, int split, const FwdParams& p) {
   w.h = a.h;
   w.hk = a.hk;
   w.q0 = a.qs;
+  w.qrow0 = a.qrow0;
+  w.krow0 = a.krow0;
+  w.tb = a.tb;
   w.lo[0] = a.lo; w.hi[0] = a.hi; w.valid[0] = a.valid;
   w.lo[1] = c.lo; w.hi[1] = c.hi; w.valid[1] = c.valid;
   w.jlo = a.valid ? a.lo : (c.valid ? c.lo : 0);
@@ -374,7 +409,7 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
 #pragma unroll
       for (int c = 0; c < C::NCHUNK; ++c)
         tma_load_4d_hint(smem_u32(sq + t * C::TILE_BYTES + c * C::CHUNK_BYTES), mq, smem_u32(&sh->q_full[t]),
-                         c * C::BOX_INNER, w.h, w.q0 + t * BLOCK_M, w.b, pol_q);
+                         c * C::BOX_INNER, w.h, w.qrow0 + w.q0 + t * BLOCK_M, w.tb, pol_q);
       q_loaded |= 1u << t;
       q_phase = (q_phase & ~(1u << t)) | ((q_uses & 1u) << t);
     }
@@ -396,7 +431,7 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d_hint(smem_u32(ring + slot * C::TILE_BYTES + c * C::CHUNK_BYTES), map, bar,
-                           c * C::BOX_INNER, w.hk, j * BLOCK_N, w.b, pol_kv);
+                           c * C::BOX_INNER, w.hk, w.krow0 + j * BLOCK_N, w.tb, pol_kv);
         issued_mask |= 1u << slot;
         phase_mask = (phase_mask & ~(1u << slot)) | ((round & 1u) << slot);
         ++kv_it;
@@ -412,7 +447,7 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
           for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int c = 0; c < C::NCHUNK; ++c)
-              tma_prefetch_l2_4d(mq, c * C::BOX_INNER, wn.h, wn.q0 + t * BLOCK_M, wn.b);
+              tma_prefetch_l2_4d(mq, c * C::BOX_INNER, wn.h, wn.qrow0 + wn.q0 + t * BLOCK_M, wn.tb);
         }
       }
     }
@@ -921,14 +956,15 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     const Tile w = get_tile<SPLIT>(u, us, t, p);
     if (!w.rows) continue;
     const int row = w.qs + r;
-    const bool row_ok = row < p.Nq;
+    const bool row_ok = row < w.nq;
     // this row's O and LSE elements (in the output, or in this key slice's
-    // partials, which hold part_rows() more rows per slice); taken where
-    // they are used, so nothing extra stays live through the block loop
-    auto o_elem = [&]() {
-      return ((static_cast<int64_t>(w.b) * p.Nq + row) * p.H + w.h) * (int64_t)D + half * HALF_D;
+    // partials, which hold part_rows() more rows per slice), from a tile
+    // recomputed where they are used, so nothing extra stays live through
+    // the block loop
+    auto o_elem = [&](const Tile& x) {
+      return ((x.orow0 + row) * p.H + x.h) * (int64_t)D + half * HALF_D;
     };
-    auto l_elem = [&]() { return (static_cast<int64_t>(w.b) * p.H + w.h) * p.Nq + row; };
+    auto l_elem = [&](const Tile& x) { return x.lse0 + row; };
     auto part_rows = [&]() { return static_cast<int64_t>(w.split) * p.B * p.Nq * p.H; };
     if (!w.valid) {
       // no visible key for any row of this tile (in this slice)
@@ -938,13 +974,13 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
         for (int i = 0; i < 16; ++i) z[i] = 0.f;
         if constexpr (SPLIT) {
 #pragma unroll
-          for (int c = 0; c < HALF_D; c += 16) store_part_row16(p.o_part + part_rows() * D + o_elem() + c, z, 0.f);
-          if (half == 0) p.lse_part[part_rows() + l_elem()] = -INFINITY;
+          for (int c = 0; c < HALF_D; c += 16) store_part_row16(p.o_part + part_rows() * D + o_elem(w) + c, z, 0.f);
+          if (half == 0) p.lse_part[part_rows() + l_elem(w)] = -INFINITY;
         } else {
-          uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem() * OUT_ES;
+          uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem(w) * OUT_ES;
 #pragma unroll
           for (int c = 0; c < HALF_D; c += 16) store_out_row16<DT>(out_row + c * OUT_ES, z, 0.f);
-          if (p.lse && half == 0) p.lse[l_elem()] = -INFINITY;
+          if (p.lse && half == 0) p.lse[l_elem(w)] = -INFINITY;
         }
       }
       continue;
@@ -969,7 +1005,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       // boundary blocks (causal diagonal, window edge, key tail), decided
       // before S arrives
       const int k0 = j * BLOCK_N;
-      const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
+      const bool need_mask = (k0 + BLOCK_N > w.nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
                              (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
       // the mask values of this block, loaded while S is computed (16-byte
       // chunks that start at or past N_k are not read)
@@ -979,7 +1015,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
 #pragma unroll
         for (int c = 0; c < MCHUNKS; ++c) {
           const int key = k0 + half * HALF_N + c * (16 / MES);
-          mk[c] = (mask_row && key < p.Nk)
+          mk[c] = (mask_row && key < w.nk)
                       ? __ldg(reinterpret_cast<const uint4*>(mask_row + static_cast<int64_t>(k0) * MES) + c)
                       : make_uint4(0u, 0u, 0u, 0u);
         }
@@ -1031,7 +1067,7 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       }
       if (need_mask) {
         const int kh = k0 + half * HALF_N;
-        const int hi_c = min(p.Nk - kh, p.causal ? row - kh + 1 : HALF_N);
+        const int hi_c = min(w.nk - kh, p.causal ? row - kh + 1 : HALF_N);
         const int lo_c = p.window_left >= 0 ? row - p.window_left - kh : 0;
 #pragma unroll
         for (int c = 0; c < HALF_N; ++c)
@@ -1122,13 +1158,14 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(smem_u32(&sh->o_empty[t]));
+    const Tile we = get_tile<SPLIT>(static_cast<int>(opaque(static_cast<uint32_t>(u))), us, t, p);
     if (row_ok) {
       if constexpr (SPLIT) {
-        float* part_row = p.o_part + part_rows() * D + o_elem();
+        float* part_row = p.o_part + part_rows() * D + o_elem(we);
 #pragma unroll
         for (int c = 0; c < HALF_D; c += 16) store_part_row16(part_row + c, reinterpret_cast<float*>(o + c), inv);
       } else {
-        uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem() * OUT_ES;
+        uint8_t* out_row = reinterpret_cast<uint8_t*>(p.out) + o_elem(we) * OUT_ES;
 #pragma unroll
         for (int c = 0; c < HALF_D; c += 16)
           store_out_row16<DT>(out_row + c * OUT_ES, reinterpret_cast<float*>(o + c), inv);
@@ -1137,8 +1174,8 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     if (row_ok && half == 0) {
       // natural log of sum_j exp(scale * s_j) = (m_used + log2(l) - PSHIFT) * ln 2
       const float lse_v = l_row > 0.f ? (m_used + __log2f(l_row) - C::PSHIFT) * 0.69314718055994531f : -INFINITY;
-      if constexpr (SPLIT) p.lse_part[part_rows() + l_elem()] = lse_v;
-      else if (p.lse) p.lse[l_elem()] = lse_v;
+      if constexpr (SPLIT) p.lse_part[part_rows() + l_elem(we)] = lse_v;
+      else if (p.lse) p.lse[l_elem(we)] = lse_v;
     }
     FA_TRACE(t, 7, 0);
   }

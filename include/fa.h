@@ -158,6 +158,34 @@ int fa_fwd_mask(const void* q, const void* k, const void* v, void* out, float* l
                 long long mask_stride_q, fa_stream_t stream);
 
 /*
+ * fa_fwd_varlen -- the forward over a packed batch of sequences of different
+ * lengths (the pages recommend the library for long sequences and batched
+ * inference, Flash Attention | Hermes Skill, "When to use" / "Common
+ * issues"; the packed layout is this library's reading).  Sequence b owns
+ * query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) of q and out, and keys
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]) of k and v; attention, causal and
+ * window rules apply within each sequence, with indices counted from its
+ * first row / key (as fa_fwd does for one batch).
+ *   q, out: [total_q, H, D]; k, v: [total_k, H_kv, D] (16-byte aligned,
+ *     contiguous; out bf16 for FA_E4M3, else the input type).
+ *   lse: [H, total_q] fp32, may be NULL.
+ *   cu_seqlens_q, cu_seqlens_k: DEVICE arrays of B + 1 int32, 4-byte
+ *     aligned, starting at 0, non-decreasing, ending at total_q / total_k.
+ *     The kernels read them and clamp every sequence into [0, total]; values
+ *     that break these rules give wrong results, never accesses outside the
+ *     tensors.
+ *   max_seqlen_q >= every sequence's query count (rows past it are not
+ *     computed); max_seqlen_k >= every key count (it sizes the L2 grouping).
+ * dtype, descales and the rest as fa_fwd_gqa.  Returns FA_ERR_ARG for bad
+ * sizes or pointers (before any GPU work), else as fa_fwd_gqa.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int H, int H_kv, int D, float scale,
+                  int causal, int window_left, int dtype, float q_descale, float k_descale,
+                  float v_descale, fa_stream_t stream);
+
+/*
  * fa_fwd_dropout -- the forward with dropout of the attention probabilities
  * (the dropout_p argument of the pages' flash_attn_func, Flash Attention |
  * Hermes Skill, Workflow 2, Step 2, which gives no definition; this

@@ -266,3 +266,24 @@ int main(void) {
     assert int(bad_batch) == _lib.FA_ERR_ARG
     assert int(bad_dim) == _lib.FA_ERR_UNSUPPORTED
     assert int(bad_fp8) == _lib.FA_ERR_ARG   # zero descale
+
+
+@pytest.mark.parametrize("kw, expect", [
+    (dict(B=0), _lib.FA_ERR_ARG),
+    (dict(cu_q=None), _lib.FA_ERR_ARG),
+    (dict(cu_k=A + 2), _lib.FA_ERR_ARG),            # int32 arrays: 4-byte aligned
+    (dict(max_q=0), _lib.FA_ERR_ARG),               # rows but no row per sequence
+    (dict(max_q=5000), _lib.FA_ERR_ARG),            # longer than the packed rows
+    (dict(max_k=9000), _lib.FA_ERR_ARG),
+    (dict(D=96), _lib.FA_ERR_UNSUPPORTED),
+    (dict(H=3, H_kv=2), _lib.FA_ERR_ARG),
+])
+def test_varlen_arguments_validated(kw, expect):
+    """fa_fwd_varlen checks its sizes and pointers on the host, before any GPU work."""
+    a = dict(q=A, k=A, v=A, out=A, lse=None, cu_q=A, cu_k=A, B=2, max_q=100, max_k=100, total_q=150, total_k=150,
+             H=2, H_kv=2, D=64, scale=0.1, causal=0, wl=-1, dt=_lib.FA_FP16)
+    a.update(kw)
+    f = _lib.lib().fa_fwd_varlen
+    assert f(a["q"], a["k"], a["v"], a["out"], a["lse"], a["cu_q"], a["cu_k"], a["B"], a["max_q"], a["max_k"],
+             a["total_q"], a["total_k"], a["H"], a["H_kv"], a["D"], a["scale"], a["causal"], a["wl"], a["dt"], 1.0,
+             1.0, 1.0, None) == expect

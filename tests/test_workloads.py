@@ -74,3 +74,27 @@ def test_fp8_quantisation():
     err = (deq - src.double()).abs()
     assert float((err / src.double().abs().clamp_min(1e-2 * x.q_descale * 64)).max()) <= 2 ** -4 + 1e-6
     assert float(x.q.to(torch.float32).abs().max()) <= 448.0
+
+
+def test_binding_roofline_picks_the_exponential_unit_where_it_is_lower():
+    """The bench line's roofline: one ex2 per score at 16 per clock per SM, 4 D
+    counted FLOP per score; the lower of that and the tensor peak binds."""
+    import bench
+    tensor, _, _ = bench.measured_peaks("bf16")
+    d64 = W.WORKLOADS["b2h8n2048d64_fp16"]
+    bound, peak, _ = bench.binding_roofline(d64, 148, 1965.0)
+    assert bound == "exp" and abs(peak - 16 * 4 * 64 * 148 * 1965e6 / 1e12) < 1e-6
+    c3 = W.WORKLOADS["causal_b4h32n8192d128_bf16"]
+    exp128 = 16 * 4 * 128 * 148 * 1965e6 / 1e12
+    bound, peak, _ = bench.binding_roofline(c3, 148, 1965.0)
+    assert (bound, peak) == (("tensor", tensor) if tensor < exp128 else ("exp", exp128))
+    fp8 = W.WORKLOADS["fp8_causal_b2h16n16384d128"]
+    bound, peak, _ = bench.binding_roofline(fp8, 148, 1965.0)
+    assert peak == min(2 * tensor, exp128)
+
+
+def test_clock_normalised_value():
+    import bench
+    assert bench.clock_normalised(1000.0, {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0}) == 1000.0 * 1965.0 / 1500.0
+    assert bench.clock_normalised(1000.0, None) is None
+    assert bench.clock_normalised(1000.0, {"sm_mhz": None, "sm_max_mhz": 1965.0}) is None

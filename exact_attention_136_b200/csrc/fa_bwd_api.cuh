@@ -21,7 +21,7 @@ template <int D, int DT, bool DROP>
 int launch_bwd(const void* q, const void* k, const void* v, const void* dout, const BwdParams& p,
                cudaStream_t stream, DeviceState* ds, int bit) {
   using C = BwdCfg<D>;
-  constexpr int DQ_SMEM_USED = 1024 + 6 * C::TILE;
+  constexpr int DQ_SMEM_USED = DqCfg<D>::SMEM_USED;
   constexpr int DQ_SMEM = DQ_SMEM_USED > 118 * 1024 ? DQ_SMEM_USED : 118 * 1024;
   const CUtensorMapDataType tdt = DT == DT_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap mq, mk, mv, mdo;
@@ -76,7 +76,7 @@ int backward(const void* q, const void* k, const void* v, const void* out, const
   float* delta = static_cast<float*>(workspace);
   const int64_t rows = static_cast<int64_t>(B) * Nq * H;
   {
-    const int64_t want = (rows + 7) / 8;
+    const int64_t want = (rows * (D / 8) + 255) / 256;   // D / 8 threads per row
     const int blocks = static_cast<int>(want < 8 * 148 ? want : 8 * 148);
     if (D == 64) fa_bwd_prologue_kernel<64><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, B, Nq, H);
     else fa_bwd_prologue_kernel<128><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, B, Nq, H);

@@ -22,11 +22,13 @@
 // block pair, were bounded by the L2's reduction throughput.
 //
 // dK/dV kernel: scores are computed transposed (keys on the TMEM lanes).
-// P^T, written back into tensor memory over S^T by the gradient warps (after
-// each has read its whole half row of S^T), is the A operand of
-// dV += P^T dO; dS^T goes to shared memory in the 128-byte-swizzled layout,
-// read K-major as the A operand of dK += dS^T Q.  Tensor memory: S^T [0,128)
-// with P^T (16-bit) over [64,128), dP^T [128,256), dV [256,256+D),
+// P^T goes to shared memory in the 128-byte-swizzled layout, read K-major as
+// the A operand of dV += P^T dO; dS^T, written back into tensor memory over
+// the upper half of dP^T by the gradient warps (after each warp has read all
+// of its dP^T), is the A operand of dK += dS^T Q.  S^T is released as soon as
+// the gradient warps hold it in registers, so the next block's S^T is
+// computed while they form P and dS.  Tensor memory: S^T [0,128),
+// dP^T [128,256) with dS^T (16-bit) over [192,256), dV [256,256+D),
 // dK [256+D,256+2D).
 //
 // dQ kernel: queries on the lanes, like the forward: S [0,128), dP [128,256),
@@ -35,6 +37,16 @@
 #pragma once
 
 namespace fa {
+
+// Timeline records of CTA 0 (see the forward's tracer); compiled out unless
+// FA_TRACE_BUILD is defined.
+#ifdef FA_TRACE_BUILD
+#define FA_BTRACE_DECL FA_TRACE_DECL
+#define FA_BTRACE(who, ev, j) FA_TRACE(who, ev, j)
+#else
+#define FA_BTRACE_DECL do { } while (0)
+#define FA_BTRACE(who, ev, j) do { } while (0)
+#endif
 
 struct BwdParams {
   void* dk;                 // [B, N_k, H, D], 16-bit like the inputs
@@ -66,11 +78,10 @@ struct BwdCfg {
   static constexpr int OFF_K = HDR;
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_STAGE = OFF_V + TILE;  // 2 stages of (Q_i, dO_i)
-  static constexpr int OFF_DS = OFF_STAGE + 2 * 2 * TILE;
-  static constexpr int SMEM = OFF_DS + 128 * 128 * 2;
-  static constexpr int S_COL = 0, P_COL = 64, DP_COL = 128;
+  static constexpr int OFF_PT = OFF_STAGE + 2 * 2 * TILE;   // P^T, 128 keys x 128 queries
+  static constexpr int SMEM = OFF_PT + 128 * 128 * 2;
+  static constexpr int S_COL = 0, DP_COL = 128, DS_COL = 192;   // dS^T (16-bit) over dP^T's upper half
   static constexpr int DV_COL = 256, DK_COL = 256 + D;
-  static constexpr int DQ_COL = 256;             // dQ kernel
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(D == 64 || D == 128, "head dim");
 };
@@ -79,15 +90,21 @@ struct BwdHeader {
   uint64_t kv_full;
   uint64_t st_full[2], st_empty[2];   // (Q_i, dO_i) stages
   uint64_t s_full, dp_full;           // S^T, dP^T computed
-  uint64_t p_ready;                   // P^T in TMEM
-  uint64_t ds_ready;                  // dS^T in shared memory
-  uint64_t ds_free;                   // the MMAs that read dS^T have completed
+  uint64_t s_free;                    // every gradient thread holds S^T in registers
+  uint64_t p_ready;                   // P^T in shared memory
+  uint64_t pt_free;                   // dV has read P^T
+  uint64_t ds_ready;                  // dS^T in TMEM
   uint64_t dkv_full;                  // every MMA of the CTA done
   uint32_t tmem_base;
   int abort_flag;
-  float lse2[2][128];                 // LSE * log2(e) of the query block (+inf: row contributes nothing)
-  float delta[2][128];
+  // -LSE * log2(e) (-inf: the row contributes nothing) and -D of the query
+  // block, query q at stat_slot(q): the two half-warps, which read queries
+  // e and 64 + e together, hit different banks and read four at a time
+  alignas(16) float nlse2[2][128];
+  alignas(16) float ndelta[2][128];
 };
+
+__device__ __forceinline__ int stat_slot(int q) { return ((q & 63) >> 2) * 8 + (q >> 6) * 4 + (q & 3); }
 static_assert(sizeof(BwdHeader) <= 3072, "backward header");
 
 constexpr int BWD_THREADS = 384;      // warpgroup 0: load + MMA; warps 4-11: gradients
@@ -140,8 +157,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   BwdHeader* sh = reinterpret_cast<BwdHeader*>(smem);
   const int warp = threadIdx.x / 32;
   // Head-major: the CTAs in flight are the key blocks of one or two heads,
-  // so that head's Q, dO and dQ accumulator stay in L2 (longest first inside
-  // a head: for causal attention key block 0 is seen by every query block).
+  // so that head's Q and dO stay in L2 (longest first inside a head: for
+  // causal attention key block 0 is seen by every query block).
   const int jk = static_cast<int>(blockIdx.x) % p.nkb;
   const int bhk = static_cast<int>(blockIdx.x) / p.nkb;   // (batch, K/V head)
   const int b = bhk / p.Hkv, hk = bhk - (bhk / p.Hkv) * p.Hkv;
@@ -149,7 +166,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   bwd_query_range(jk, p, i_lo, i_hi);
   // The n-th query block a CTA visits is i_lo + (n + rot) mod cnt: causal
   // CTAs already start at their own diagonal; the others start at a block
-  // of their own, so CTAs running side by side add into different dQ rows.
+  // of their own, so CTAs running side by side read different Q blocks.
   const int cnt = i_hi - i_lo + 1;
   const int rot = (p.causal || cnt <= 0) ? 0 : jk % cnt;
   // every query head of the K/V head's group, cnt query blocks each: visit n
@@ -164,10 +181,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_init(smem_u32(&sh->st_empty[s]), 1);
     }
     mbar_init(smem_u32(&sh->s_full), 1);
+    mbar_init(smem_u32(&sh->s_free), 256);
     mbar_init(smem_u32(&sh->dp_full), 1);
     mbar_init(smem_u32(&sh->p_ready), 256);
+    mbar_init(smem_u32(&sh->pt_free), 1);
     mbar_init(smem_u32(&sh->ds_ready), 256);
-    mbar_init(smem_u32(&sh->ds_free), 1);
     mbar_init(smem_u32(&sh->dkv_full), 1);
     sh->abort_flag = 0;
     fence_mbar_init();
@@ -228,72 +246,81 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane_id() == 0 && i_lo <= i_hi) {
+      FA_BTRACE_DECL;
       constexpr uint32_t FMT = DT == DT_BF16 ? 1u : 0u;
       constexpr uint32_t ID_ST = make_idesc(FMT, false, 128, 128);          // S^T, dP^T: both K-major
-      constexpr uint32_t ID_KV = make_idesc(FMT, true, 128, D);             // dV, dK: A in TMEM, B M/N-major
+      constexpr uint32_t ID_KV = make_idesc(FMT, true, 128, D);             // dV, dK: B M/N-major
       constexpr uint32_t HI = sdesc_sw128_hi(1024);
       const uint32_t k_kmaj = sdesc_sw128_lo(sbase + C::OFF_K, 16);
       const uint32_t v_kmaj = sdesc_sw128_lo(sbase + C::OFF_V, 16);
-      const uint32_t ds_kmaj = sdesc_sw128_lo(sbase + C::OFF_DS, 16);
-      // S^T = K Q_n^T for the n-th query block (keys on the lanes)
-      auto issue_st = [&](int n) {
-        const uint32_t q_kmaj = sdesc_sw128_lo(sbase + C::OFF_STAGE + (n & 1) * 2 * C::TILE, 16);
+      const uint32_t pt_kmaj = sdesc_sw128_lo(sbase + C::OFF_PT, 16);
+      const uint32_t q_tile0 = sbase + C::OFF_STAGE;
+      // S^T = K Q_n^T and dP^T = V dO_n^T for the n-th query block (keys on
+      // the lanes); both K-major
+      auto issue_kmaj = [&](uint32_t col, uint32_t a_kmaj, uint32_t b_tile) {
+        const uint32_t b_kmaj = sdesc_sw128_lo(b_tile, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int byte = kk * 32;
           const uint32_t off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
-          mma_f16_ss_lo(tbase + C::S_COL, k_kmaj + off, q_kmaj + off, HI, ID_ST, kk > 0);
+          mma_f16_ss_lo(tbase + col, a_kmaj + off, b_kmaj + off, HI, ID_ST, kk > 0);
         }
-        mma_commit(smem_u32(&sh->s_full));
       };
-      // Per query block n: dP^T(n), then on P^T(n): dV(n) and the next
-      // block's S^T (which overwrites S^T(n) under P^T(n), after dV(n) has
-      // read it), then on dS^T(n): dK(n).  So dV(n) and S^T(n+1) run while
-      // the gradient warps form dS, and dP^T(n+1) while they compute P(n+1).
+      // Per query block n, in pipe order: S^T(n+1) (as soon as the gradient
+      // warps hold S^T(n) in registers), dV(n) on P^T(n), dK(n) on dS^T(n),
+      // then dP^T(n+1) over dP^T(n) and dS^T(n).  The gradient warps form
+      // P(n+1) while dV(n), dK(n) and dP^T(n+1) run.
       bool ok = mbar_wait(smem_u32(&sh->kv_full), 0, lim) && mbar_wait(smem_u32(&sh->st_full[0]), 0, lim);
       if (ok && visits > 0) {
         tc_fence_after();
-        issue_st(0);
+        issue_kmaj(C::S_COL, k_kmaj, q_tile0);
+        mma_commit(smem_u32(&sh->s_full));
+        issue_kmaj(C::DP_COL, v_kmaj, q_tile0 + C::TILE);
+        mma_commit(smem_u32(&sh->dp_full));
       }
       for (int n = 0; n < visits && ok; ++n) {
-        const int s = n & 1;
-        const uint32_t q_tile = sbase + C::OFF_STAGE + s * 2 * C::TILE;
-        const uint32_t do_tile = q_tile + C::TILE;
-        tc_fence_after();
-        const uint32_t do_kmaj = sdesc_sw128_lo(do_tile, 16);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int byte = kk * 32;
-          const uint32_t off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
-          mma_f16_ss_lo(tbase + C::DP_COL, v_kmaj + off, do_kmaj + off, HI, ID_ST, kk > 0);
-        }
-        mma_commit(smem_u32(&sh->dp_full));
-        if (!mbar_wait(smem_u32(&sh->p_ready), n & 1, lim)) { ok = false; break; }
-        tc_fence_after();
-        // dV += P^T dO_n (A from TMEM: 16 queries = 8 columns per step)
-        const uint32_t q_mn = sdesc_sw128_lo(q_tile, C::CHUNK), do_mn = sdesc_sw128_lo(do_tile, C::CHUNK);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
-          mma_f16_ts_lo(tbase + C::DV_COL, tbase + C::P_COL + kk * 8, do_mn + off, HI, ID_KV, n > 0 || kk > 0);
-        }
+        const uint32_t q_tile = q_tile0 + (n & 1) * 2 * C::TILE;
+        const uint32_t q_next = q_tile0 + ((n + 1) & 1) * 2 * C::TILE;
         if (n + 1 < visits) {
-          if (!mbar_wait(smem_u32(&sh->st_full[(n + 1) & 1]), ((n + 1) >> 1) & 1, lim)) { ok = false; break; }
+          FA_BTRACE(2, 0, n);
+          if (!mbar_wait(smem_u32(&sh->s_free), n & 1, lim) ||
+              !mbar_wait(smem_u32(&sh->st_full[(n + 1) & 1]), ((n + 1) >> 1) & 1, lim)) {
+            ok = false;
+            break;
+          }
+          FA_BTRACE(2, 1, n);
           tc_fence_after();
-          issue_st(n + 1);
+          issue_kmaj(C::S_COL, k_kmaj, q_next);
+          mma_commit(smem_u32(&sh->s_full));
         }
-        if (!mbar_wait(smem_u32(&sh->ds_ready), n & 1, lim)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&sh->p_ready), n & 1, lim)) { ok = false; break; }
+        FA_BTRACE(2, 2, n);
         tc_fence_after();
+        const uint32_t q_mn = sdesc_sw128_lo(q_tile, C::CHUNK), do_mn = sdesc_sw128_lo(q_tile + C::TILE, C::CHUNK);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          // dK += dS^T Q_n: A = dS^T in shared memory, K-major (16 queries = 32 bytes of a row)
+          // dV += P^T dO_n: A = P^T in shared memory, K-major (16 queries = 32 bytes of a row)
           const int byte = kk * 32;
           const uint32_t a_off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
           const uint32_t b_off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
-          mma_f16_ss_lo(tbase + C::DK_COL, ds_kmaj + a_off, q_mn + b_off, HI, ID_KV, n > 0 || kk > 0);
+          mma_f16_ss_lo(tbase + C::DV_COL, pt_kmaj + a_off, do_mn + b_off, HI, ID_KV, n > 0 || kk > 0);
         }
-        mma_commit(smem_u32(&sh->st_empty[s]));   // last readers of Q_n and dO_n
-        mma_commit(smem_u32(&sh->ds_free));       // ... and of dS^T(n)
+        mma_commit(smem_u32(&sh->pt_free));
+        if (!mbar_wait(smem_u32(&sh->ds_ready), n & 1, lim)) { ok = false; break; }
+        FA_BTRACE(2, 3, n);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          // dK += dS^T Q_n: A = dS^T (16-bit) in TMEM, 16 queries = 8 columns per step
+          const uint32_t off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
+          mma_f16_ts_lo(tbase + C::DK_COL, tbase + C::DS_COL + kk * 8, q_mn + off, HI, ID_KV, n > 0 || kk > 0);
+        }
+        mma_commit(smem_u32(&sh->st_empty[n & 1]));   // last readers of Q_n and dO_n
+        if (n + 1 < visits) {
+          issue_kmaj(C::DP_COL, v_kmaj, q_next + C::TILE);
+          mma_commit(smem_u32(&sh->dp_full));
+        }
+        FA_BTRACE(2, 4, n);
       }
       if (!ok) bwd_error(sh, p, ST_TIMEOUT_MMA);
       mma_commit(smem_u32(&sh->dkv_full));   // also: every MMA done before TMEM is released
@@ -305,60 +332,40 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int sub = (warp - 4) >> 2;
     const int lane = static_cast<int>(lane_id());
     const int half = lane >> 4;
-    const int r = quad * 32 + sub * 16 + (lane & 15);           // TMEM lane: key (S^T, dK, dV) or query (dQ)
+    const int r = quad * 32 + sub * 16 + (lane & 15);           // TMEM lane: key
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32 + sub * 16) << 16;
     const int t = static_cast<int>(threadIdx.x) - 128;          // 0..255
     const int key = jk * 128 + r;
     const float c2 = p.score_scale;
-    uint8_t* ds_row = smem + C::OFF_DS + half * C::CHUNK + r * 128;
+    uint8_t* pt_row = smem + C::OFF_PT + half * C::CHUNK + r * 128;
     bool ok = true;
     bool dq_ok = true;   // this block's later waits (reported at the next vote)
+    // one row statistic per thread (threads 0-127: LSE, 128-255: D) of
+    // visit m, loaded a visit ahead
+    auto load_stat = [&](int m) -> float {
+      const int hq = hk * p.qpk + m / cnt;
+      const int q = (i_lo + (m % cnt + rot) % cnt) * 128 + (t & 127);
+      if (q >= p.Nq) return t < 128 ? -INFINITY : 0.f;   // rows past N_q contribute nothing
+      const long long at = (static_cast<long long>(b) * p.H + hq) * p.Nq + q;
+      if (t >= 128) return -p.delta[at];
+      const float l = p.lse[at];
+      return l != -INFINITY ? l * -1.4426950408889634f : -INFINITY;
+    };
+    float stat = visits > 0 ? load_stat(0) : 0.f;
+    FA_BTRACE_DECL;
     for (int n = 0; n < visits; ++n) {
+      FA_BTRACE(0, 0, n);
       const int hq = hk * p.qpk + n / cnt;
       const int i = i_lo + (n % cnt + rot) % cnt;
-      const long long bhq = (static_cast<long long>(b) * p.H + hq) * p.Nq;
       const int buf = n & 1;
-      // row statistics of query block i (one value per thread); the vote
-      // below is also the barrier that publishes them
-      {
-        const int q = i * 128 + (t & 127);
-        if (t < 128) {
-          float v = INFINITY;   // rows past N_q or without a visible key contribute nothing
-          if (q < p.Nq) {
-            const float l = p.lse[bhq + q];
-            if (l != -INFINITY) v = l * 1.4426950408889634f;
-          }
-          sh->lse2[buf][t] = v;
-        } else {
-          sh->delta[buf][t - 128] = q < p.Nq ? p.delta[bhq + q] : 0.f;
-        }
-      }
+      // row statistics of query block i; the vote below is also the
+      // barrier that publishes them (buffer buf was last read in visit
+      // n - 2, before every thread's vote of visit n - 1)
+      (t < 128 ? sh->nlse2[buf] : sh->ndelta[buf])[stat_slot(t & 127)] = stat;
+      if (n + 1 < visits) stat = load_stat(n + 1);
       const int q0 = i * 128;
       const bool need_mask = (jk * 128 + 128 > p.Nk) || (p.causal && jk * 128 + 127 > q0) ||
                              (p.window_left >= 0 && jk * 128 < q0 + 127 - p.window_left);
-      const bool got = mbar_wait(smem_u32(&sh->s_full), n & 1, lim);
-      if (!grad_bar_and(got && dq_ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // the thread's half row of S^T (queries half * 64 + [0, 64)) in
-      // registers before any P^T store lands over its upper half
-      float pv[64];
-      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::S_COL, reinterpret_cast<uint32_t*>(pv));
-      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::S_COL + 32, reinterpret_cast<uint32_t*>(pv + 32));
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const int ql = half * 64 + e;
-        float pe = ex2_approx(pv[e] * c2 - sh->lse2[buf][ql]);
-        if (need_mask) {
-          const int q = q0 + ql;
-          const bool vis = key < p.Nk && (!p.causal || key <= q) && (p.window_left < 0 || key >= q - p.window_left);
-          pe = vis ? pe : 0.f;
-        }
-        pv[e] = pe;
-      }
       // dropout keep bits of this thread's key for its 64 queries (bit e:
       // query q0 + 64 * half + e).  The generator gives 8 keys of one query
       // per call, so in round m lane L draws query 8m + (L mod 8) for its
@@ -381,61 +388,109 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           keep[m / 4] |= got8 << (8 * (m % 4));
         }
       }
+      const bool got = mbar_wait(smem_u32(&sh->s_full), n & 1, lim);
+      if (!grad_bar_and(got && dq_ok)) {
+        ok = false;
+        break;
+      }
+      FA_BTRACE(0, 1, n);
+      tc_fence_after();
+      // the thread's half row of S^T (queries half * 64 + [0, 64)); the MMA
+      // may overwrite S^T with the next block's once every thread has it
+      float pv[64];
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::S_COL, reinterpret_cast<uint32_t*>(pv));
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::S_COL + 32, reinterpret_cast<uint32_t*>(pv + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sh->s_free));
+      if (need_mask) {
+        // keys a query may not see: a score of -inf gives P = 0
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pw[16];
+        for (int e = 0; e < 64; ++e) {
+          const int q = q0 + half * 64 + e;
+          const bool vis = key < p.Nk && (!p.causal || key <= q) && (p.window_left < 0 || key >= q - p.window_left);
+          pv[e] = vis ? pv[e] : -INFINITY;
+        }
+      }
+      // P = 2^(S c2 - LSE log2 e), the statistic held negated; queries
+      // e..e+3 at [2 (e / 4)]
+      const float4* nl4 = reinterpret_cast<const float4*>(sh->nlse2[buf]) + half;
+      const float2 c2v = make_float2(c2, c2);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float p0 = pv[c * 32 + 2 * e], p1 = pv[c * 32 + 2 * e + 1];
+      for (int e4 = 0; e4 < 16; ++e4) {
+        const float4 l4 = nl4[2 * e4];
+        const float2 x0 = __ffma2_rn(make_float2(pv[4 * e4], pv[4 * e4 + 1]), c2v, make_float2(l4.x, l4.y));
+        const float2 x1 = __ffma2_rn(make_float2(pv[4 * e4 + 2], pv[4 * e4 + 3]), c2v, make_float2(l4.z, l4.w));
+        pv[4 * e4] = ex2_approx(x0.x);
+        pv[4 * e4 + 1] = ex2_approx(x0.y);
+        pv[4 * e4 + 2] = ex2_approx(x1.x);
+        pv[4 * e4 + 3] = ex2_approx(x1.y);
+      }
+      FA_BTRACE(0, 2, n);
+      // P^T(n - 1) in shared memory has been read by dV(n - 1)
+      if (n > 0) dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->pt_free), (n - 1) & 1, lim)) && dq_ok;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        // P^T for queries half * 64 + [16c, 16c + 16) (dV takes the kept
+        // probabilities, scaled by 1 / (1 - p)): row r, two 16-byte units of
+        // the 128-byte row, XOR-swizzled by (r mod 8) like a TMA 128B tile
+        uint32_t pw[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float p0 = pv[c * 16 + e], p1 = pv[c * 16 + e + 1];
           if constexpr (DROP) {
-            // dV takes the kept probabilities, scaled by 1 / (1 - p)
-            const uint32_t kb = keep[c] >> (2 * e);
+            const uint32_t kb = keep[(c * 16 + e) / 32] >> ((c * 16 + e) % 32);
             p0 = (kb & 1u) ? p0 * p.drop_scale : 0.f;
             p1 = (kb & 2u) ? p1 * p.drop_scale : 0.f;
           }
-          pw[e] = pack2<DT>(p0, p1);
+          pw[e / 2] = pack2<DT>(p0, p1);
         }
-        tmem_st_16x32bx2_x16<32>(tbase + lane_off + C::P_COL + c * 16, pw);
+        const int u0 = (2 * c) ^ (r & 7), u1 = (2 * c + 1) ^ (r & 7);
+        *reinterpret_cast<uint4*>(pt_row + u0 * 16) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        *reinterpret_cast<uint4*>(pt_row + u1 * 16) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      }
+      fence_proxy_async_smem();   // P^T stores visible to the MMA's reads
+      mbar_arrive(smem_u32(&sh->p_ready));
+      // dP^T(n): the warp reads all of it before any dS^T store lands over
+      // its upper half (a wait that times out leaves dS unusable; the next
+      // vote reports it)
+      dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim)) && dq_ok;
+      FA_BTRACE(0, 3, n);
+      tc_fence_after();
+      float gv[64];
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::DP_COL, reinterpret_cast<uint32_t*>(gv));
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::DP_COL + 32, reinterpret_cast<uint32_t*>(gv + 32));
+      tmem_wait_ld();
+      const float4* nd4 = reinterpret_cast<const float4*>(sh->ndelta[buf]) + half;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dw[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 v4 = nd4[2 * (8 * c + e4)];
+#pragma unroll
+          for (int x = 0; x < 4; x += 2) {
+            const int e = 32 * c + 4 * e4 + x;
+            float2 g = make_float2(gv[e], gv[e + 1]);
+            if constexpr (DROP) {
+              // dP of the dropped forward: Z / (1 - p) times dO V^T
+              const uint32_t kb = keep[c] >> ((4 * e4 + x) % 32);
+              g.x = (kb & 1u) ? g.x * p.drop_scale : 0.f;
+              g.y = (kb & 2u) ? g.y * p.drop_scale : 0.f;
+            }
+            const float2 nd = x == 0 ? make_float2(v4.x, v4.y) : make_float2(v4.z, v4.w);
+            const float2 d = __fmul2_rn(make_float2(pv[e], pv[e + 1]), __fadd2_rn(g, nd));
+            dw[(4 * e4 + x) / 2] = pack2<DT>(d.x, d.y);
+          }
+        }
+        // dS^T (16-bit) for the thread's queries 32c .. 32c + 31: columns
+        // DS_COL + 16c (+ 32 for the upper half-warp)
+        tmem_st_16x32bx2_x16<32>(tbase + lane_off + C::DS_COL + c * 16, dw);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sh->p_ready));
-      // dP^T(n) (committed after S^T(n); a wait that times out leaves dS
-      // unusable, which the next vote reports)
-      dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim)) && dq_ok;
-      // dS^T(n - 1) in shared memory has been read by dK(n - 1)
-      if (n > 0) dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->ds_free), (n - 1) & 1, lim)) && dq_ok;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        // dS^T for queries half * 64 + [16c, 16c + 16)
-        uint32_t dpv[16];
-        tmem_ld_16x32bx2_x16<64>(tbase + lane_off + C::DP_COL + c * 16, dpv);
-        tmem_wait_ld();
-        uint32_t dw[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const int ql = half * 64 + c * 16 + e;
-          float g0 = __uint_as_float(dpv[e]), g1 = __uint_as_float(dpv[e + 1]);
-          if constexpr (DROP) {
-            // dP of the dropped forward: Z / (1 - p) times dO V^T
-            const uint32_t kb = keep[(c * 16 + e) / 32] >> ((c * 16 + e) % 32);
-            g0 = (kb & 1u) ? g0 * p.drop_scale : 0.f;
-            g1 = (kb & 2u) ? g1 * p.drop_scale : 0.f;
-          }
-          const float d0 = pv[c * 16 + e] * (g0 - sh->delta[buf][ql]);
-          const float d1 = pv[c * 16 + e + 1] * (g1 - sh->delta[buf][ql + 1]);
-          dw[e / 2] = pack2<DT>(d0, d1);
-        }
-        // row r of dS^T, two 16-byte units of the 128-byte row, XOR-swizzled
-        // by (r mod 8) like a TMA 128B tile
-        const int u0 = (2 * c) ^ (r & 7), u1 = (2 * c + 1) ^ (r & 7);
-        *reinterpret_cast<uint4*>(ds_row + u0 * 16) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
-        *reinterpret_cast<uint4*>(ds_row + u1 * 16) = make_uint4(dw[4], dw[5], dw[6], dw[7]);
-      }
-      fence_proxy_async_smem();   // dS^T stores visible to the MMA's reads
-      tc_fence_before();
       mbar_arrive(smem_u32(&sh->ds_ready));
+      FA_BTRACE(0, 4, n);
     }
     if (!grad_bar_and(ok && dq_ok)) {
       ok = false;
@@ -480,19 +535,39 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 }
 
 // dQ kernel: one CTA per (batch, head, 128-query block i), head-major, the
-// query blocks with the most keys first.  Warp 0 loads Q_i and dO_i once and
-// K_j, V_j of every key block the queries see through two stages; warp 1
-// issues S = Q_i K_j^T and dP = dO_i V_j^T (queries on the lanes), then on
-// dS(j): dQ += dS K_j (A = dS from TMEM), then the next block's S and dP at
-// once; warps 4-11 form dS = P * (dP - D) with P = exp(S - LSE).
+// query blocks with the most keys first.  Warp 0 loads Q_i and dO_i once,
+// then K_j through three stages and V_j through two; warp 1 issues
+// S = Q_i K_j^T and dP = dO_i V_j^T (queries on the lanes) and, on dS(j),
+// dQ += dS K_j with A = dS from TMEM; warps 4-11 form dS = P * (dP - D) with
+// P = exp(S - LSE).  S is double-buffered in TMEM, so the gradient warps
+// form P(j+1) while the tensor pipe runs dP(j+1), dQ(j) and S(j+2): per key
+// block the MMA thread issues, after dS(j), dP(j+1) (over dP(j), read by
+// then), dQ(j), and S(j+2) into the buffer of S(j) (whose dS(j) dQ(j) has
+// read, in pipe order).  K_j stays until dQ(j), hence the third K stage.
+// TMEM: S(even) [0,128), dP [128,256), dQ [256,256+D), S(odd) [384,512);
+// dS (16-bit) over the upper half of its S buffer.
 struct DqHeader {
   uint64_t q_full;
-  uint64_t kv_full[2], kv_empty[2];
-  uint64_t dp_full;          // S(j) and dP(j) computed
+  uint64_t k_full[3], k_empty[3];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2];        // S(j) in buffer j mod 2 computed
+  uint64_t dp_full;          // dP(j) computed
   uint64_t ds_ready;         // dS(j) in TMEM
   uint64_t dq_done;          // every MMA done
   uint32_t tmem_base;
   int abort_flag;
+};
+static_assert(sizeof(DqHeader) <= 1024, "dQ header");
+
+template <int D>
+struct DqCfg {
+  static constexpr int TILE = BwdCfg<D>::TILE;
+  static constexpr int OFF_Q = 1024, OFF_DO = OFF_Q + TILE;
+  static constexpr int OFF_K = OFF_DO + TILE;           // 3 stages
+  static constexpr int OFF_V = OFF_K + 3 * TILE;        // 2 stages
+  static constexpr int SMEM_USED = OFF_V + 2 * TILE;
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 384, DP_COL = 128, DQ_COL = 256;
+  static_assert(SMEM_USED <= 232448, "shared memory budget");
 };
 
 template <int D, int DT, bool DROP>
@@ -501,7 +576,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const BwdParams p) {
   using C = BwdCfg<D>;
-  constexpr int OFF_Q = 1024, OFF_DO = OFF_Q + C::TILE, OFF_KV = OFF_DO + C::TILE;   // then 2 x (K, V)
+  using Q = DqCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) atomicOr(p.status, ST_SMEM_MISALIGNED);
@@ -523,9 +598,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sh->q_full), 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(smem_u32(&sh->k_full[s]), 1);
+      mbar_init(smem_u32(&sh->k_empty[s]), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&sh->kv_full[s]), 1);
-      mbar_init(smem_u32(&sh->kv_empty[s]), 1);
+      mbar_init(smem_u32(&sh->v_full[s]), 1);
+      mbar_init(smem_u32(&sh->v_empty[s]), 1);
+      mbar_init(smem_u32(&sh->s_full[s]), 1);
     }
     mbar_init(smem_u32(&sh->dp_full), 1);
     mbar_init(smem_u32(&sh->ds_ready), 256);
@@ -555,79 +635,96 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_arrive_expect_tx(smem_u32(&sh->q_full), 2 * C::TILE);
 #pragma unroll
       for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d_hint(sbase + OFF_Q + c * C::CHUNK, &tm_q, smem_u32(&sh->q_full), c * 64, h, q0, b, pol_q);
-        tma_load_4d_hint(sbase + OFF_DO + c * C::CHUNK, &tm_do, smem_u32(&sh->q_full), c * 64, h, q0, b, pol_q);
+        tma_load_4d_hint(sbase + Q::OFF_Q + c * C::CHUNK, &tm_q, smem_u32(&sh->q_full), c * 64, h, q0, b, pol_q);
+        tma_load_4d_hint(sbase + Q::OFF_DO + c * C::CHUNK, &tm_do, smem_u32(&sh->q_full), c * 64, h, q0, b, pol_q);
       }
-      int n = 0;
-      for (; n < cnt; ++n) {
-        const int j = j_lo + n, s = n & 1;
-        if (!mbar_wait(smem_u32(&sh->kv_empty[s]), ((n >> 1) & 1) ^ 1, lim)) {
-          atomicOr(p.status, ST_TIMEOUT_LOAD);
-          ok = false;
-          break;
-        }
-        const uint32_t bar = smem_u32(&sh->kv_full[s]);
-        const uint32_t kdst = sbase + OFF_KV + s * 2 * C::TILE;
-        mbar_arrive_expect_tx(bar, 2 * C::TILE);
+      int nk = 0, nv = 0;   // K and V loads issued
+      for (int n = 0; n < cnt && ok; ++n) {
+        const int j = j_lo + n;
+        const int sk = n % 3, sv = n & 1;
+        if (!mbar_wait(smem_u32(&sh->k_empty[sk]), ((n / 3) & 1) ^ 1, lim)) { ok = false; break; }
+        mbar_arrive_expect_tx(smem_u32(&sh->k_full[sk]), C::TILE);
 #pragma unroll
-        for (int c = 0; c < C::NCHUNK; ++c) {
-          tma_load_4d_hint(kdst + c * C::CHUNK, &tm_k, bar, c * 64, hk, j * 128, b, pol_kv);
-          tma_load_4d_hint(kdst + C::TILE + c * C::CHUNK, &tm_v, bar, c * 64, hk, j * 128, b, pol_kv);
-        }
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d_hint(sbase + Q::OFF_K + sk * C::TILE + c * C::CHUNK, &tm_k, smem_u32(&sh->k_full[sk]), c * 64,
+                           hk, j * 128, b, pol_kv);
+        ++nk;
+        if (!mbar_wait(smem_u32(&sh->v_empty[sv]), ((n >> 1) & 1) ^ 1, lim)) { ok = false; break; }
+        mbar_arrive_expect_tx(smem_u32(&sh->v_full[sv]), C::TILE);
+#pragma unroll
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d_hint(sbase + Q::OFF_V + sv * C::TILE + c * C::CHUNK, &tm_v, smem_u32(&sh->v_full[sv]), c * 64,
+                           hk, j * 128, b, pol_kv);
+        ++nv;
       }
       if (!ok) {
+        // drain: the copies already issued land before the CTA exits
+        atomicOr(p.status, ST_TIMEOUT_LOAD);
         mbar_wait(smem_u32(&sh->q_full), 0, lim);
-        for (int m = max(0, n - 2); m < n; ++m) mbar_wait(smem_u32(&sh->kv_full[m & 1]), (m >> 1) & 1, lim);
+        for (int m = max(0, nk - 3); m < nk; ++m) mbar_wait(smem_u32(&sh->k_full[m % 3]), (m / 3) & 1, lim);
+        for (int m = max(0, nv - 2); m < nv; ++m) mbar_wait(smem_u32(&sh->v_full[m & 1]), (m >> 1) & 1, lim);
       }
     }
   } else if (warp == 1) {
     if (lane_id() == 0 && cnt > 0) {
+      FA_BTRACE_DECL;
       constexpr uint32_t FMT = DT == DT_BF16 ? 1u : 0u;
       constexpr uint32_t ID_S = make_idesc(FMT, false, 128, 128);   // S, dP: both K-major
       constexpr uint32_t ID_Q = make_idesc(FMT, true, 128, D);      // dQ: A in TMEM, B head-dim-major
       constexpr uint32_t HI = sdesc_sw128_hi(1024);
-      const uint32_t q_kmaj = sdesc_sw128_lo(sbase + OFF_Q, 16);
-      const uint32_t do_kmaj = sdesc_sw128_lo(sbase + OFF_DO, 16);
-      // S(n) and dP(n) for the n-th key block
-      auto issue_s_dp = [&](int n) {
-        const uint32_t kt = sbase + OFF_KV + (n & 1) * 2 * C::TILE;
-        const uint32_t k_kmaj = sdesc_sw128_lo(kt, 16), v_kmaj = sdesc_sw128_lo(kt + C::TILE, 16);
+      const uint32_t q_kmaj = sdesc_sw128_lo(sbase + Q::OFF_Q, 16);
+      const uint32_t do_kmaj = sdesc_sw128_lo(sbase + Q::OFF_DO, 16);
+      // S(n) = Q K_n^T into buffer n mod 2, on K_n landed
+      auto issue_s = [&](int n) -> bool {
+        if (!mbar_wait(smem_u32(&sh->k_full[n % 3]), (n / 3) & 1, lim)) return false;
+        tc_fence_after();
+        const uint32_t k_kmaj = sdesc_sw128_lo(sbase + Q::OFF_K + (n % 3) * C::TILE, 16);
+        const uint32_t col = (n & 1) ? Q::S_COL1 : Q::S_COL0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int byte = kk * 32;
           const uint32_t off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
-          mma_f16_ss_lo(tbase + C::S_COL, q_kmaj + off, k_kmaj + off, HI, ID_S, kk > 0);
+          mma_f16_ss_lo(tbase + col, q_kmaj + off, k_kmaj + off, HI, ID_S, kk > 0);
         }
+        mma_commit(smem_u32(&sh->s_full[n & 1]));
+        return true;
+      };
+      // dP(n) = dO V_n^T, on V_n landed; V_n's stage is free after it
+      auto issue_dp = [&](int n) -> bool {
+        if (!mbar_wait(smem_u32(&sh->v_full[n & 1]), (n >> 1) & 1, lim)) return false;
+        tc_fence_after();
+        const uint32_t v_kmaj = sdesc_sw128_lo(sbase + Q::OFF_V + (n & 1) * C::TILE, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int byte = kk * 32;
           const uint32_t off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
-          mma_f16_ss_lo(tbase + C::DP_COL, do_kmaj + off, v_kmaj + off, HI, ID_S, kk > 0);
+          mma_f16_ss_lo(tbase + Q::DP_COL, do_kmaj + off, v_kmaj + off, HI, ID_S, kk > 0);
         }
         mma_commit(smem_u32(&sh->dp_full));
+        mma_commit(smem_u32(&sh->v_empty[n & 1]));
+        return true;
       };
-      bool ok = mbar_wait(smem_u32(&sh->q_full), 0, lim) && mbar_wait(smem_u32(&sh->kv_full[0]), 0, lim);
-      if (ok) {
-        tc_fence_after();
-        issue_s_dp(0);
-      }
+      bool ok = mbar_wait(smem_u32(&sh->q_full), 0, lim) && issue_s(0) && issue_dp(0) && (cnt < 2 || issue_s(1));
       for (int n = 0; n < cnt && ok; ++n) {
+        FA_BTRACE(4, 0, n);
         if (!mbar_wait(smem_u32(&sh->ds_ready), n & 1, lim)) { ok = false; break; }
+        FA_BTRACE(4, 1, n);
         tc_fence_after();
-        // dQ += dS K_n: A = dS (16-bit, over S's upper half), 16 keys = 8 columns per step
-        const uint32_t k_mn = sdesc_sw128_lo(sbase + OFF_KV + (n & 1) * 2 * C::TILE, C::CHUNK);
+        // dP(n+1) over dP(n): the gradient warps read dP(n) before dS(n)
+        if (n + 1 < cnt && !issue_dp(n + 1)) { ok = false; break; }
+        // dQ += dS K_n: A = dS (16-bit, upper half of S(n)'s buffer), 16 keys = 8 columns per step
+        const uint32_t k_mn = sdesc_sw128_lo(sbase + Q::OFF_K + (n % 3) * C::TILE, C::CHUNK);
+        const uint32_t ds_col = ((n & 1) ? Q::S_COL1 : Q::S_COL0) + 64;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
-          mma_f16_ts_lo(tbase + C::DQ_COL, tbase + C::P_COL + kk * 8, k_mn + off, HI, ID_Q, n > 0 || kk > 0);
+          mma_f16_ts_lo(tbase + Q::DQ_COL, tbase + ds_col + kk * 8, k_mn + off, HI, ID_Q, n > 0 || kk > 0);
         }
-        mma_commit(smem_u32(&sh->kv_empty[n & 1]));   // last readers of K_n, V_n
-        if (n + 1 < cnt) {
-          // S(n+1) overwrites dS(n) after dQ(n) has read it (same pipe, in order)
-          if (!mbar_wait(smem_u32(&sh->kv_full[(n + 1) & 1]), ((n + 1) >> 1) & 1, lim)) { ok = false; break; }
-          tc_fence_after();
-          issue_s_dp(n + 1);
-        }
+        mma_commit(smem_u32(&sh->k_empty[n % 3]));   // last reader of K_n
+        FA_BTRACE(4, 2, n);
+        // S(n+2) over S(n) and dS(n), after dQ(n) (same pipe, in order)
+        if (n + 2 < cnt && !issue_s(n + 2)) { ok = false; break; }
+        FA_BTRACE(4, 3, n);
       }
       if (!ok) atomicOr(p.status, ST_TIMEOUT_MMA);
       mma_commit(smem_u32(&sh->dq_done));
@@ -642,23 +739,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32 + sub * 16) << 16;
     const int q = q0 + r;
     const long long bhq = static_cast<long long>(bh) * p.Nq;
-    // this row's statistics: LSE * log2(e) (+inf: the row contributes nothing) and D
-    float lse2 = INFINITY, dlt = 0.f;
+    // this row's statistics: -LSE * log2(e) (-inf: the row contributes nothing) and D
+    float nlse2 = -INFINITY, dlt = 0.f;
     if (q < p.Nq) {
       const float l = p.lse[bhq + q];
-      if (l != -INFINITY) lse2 = l * 1.4426950408889634f;
+      if (l != -INFINITY) nlse2 = l * -1.4426950408889634f;
       dlt = p.delta[bhq + q];
     }
     const float c2 = p.score_scale;
     bool ok = true;
+    FA_BTRACE_DECL;
     for (int n = 0; n < cnt; ++n) {
+      if (threadIdx.x == 128) FA_BTRACE(3, 0, n);
       const int k0 = (j_lo + n) * 128;
+      const uint32_t s_col = (n & 1) ? Q::S_COL1 : Q::S_COL0;
       const bool need_mask = (k0 + 128 > p.Nk) || (p.causal && k0 + 127 > q0) ||
                              (p.window_left >= 0 && k0 < q0 + 127 - p.window_left);
-      if (!grad_bar_and(mbar_wait(smem_u32(&sh->dp_full), n & 1, lim))) {
-        ok = false;
-        break;
-      }
       // dropout keep bits of this row's keys k0 + 64 * half + [0, 64)
       uint32_t keep[2] = {0u, 0u};
       if constexpr (DROP) {
@@ -670,46 +766,71 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                                     p.drop_threshold)
                          << (8 * (g % 4));
       }
+      // exit vote: this S landed, and every earlier wait of every warp held
+      if (!grad_bar_and(ok && mbar_wait(smem_u32(&sh->s_full[n & 1]), (n >> 1) & 1, lim))) {
+        ok = false;
+        break;
+      }
+      if (threadIdx.x == 128) FA_BTRACE(3, 1, n);
       tc_fence_after();
       // the whole half row of S (keys half * 64 + [0, 64)) before any dS store
       float pv[64];
-      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::S_COL, reinterpret_cast<uint32_t*>(pv));
-      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + C::S_COL + 32, reinterpret_cast<uint32_t*>(pv + 32));
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + s_col, reinterpret_cast<uint32_t*>(pv));
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + s_col + 32, reinterpret_cast<uint32_t*>(pv + 32));
       tmem_wait_ld();
+      if (need_mask) {
+        // keys the row may not see: a score of -inf gives P = 0
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        float pe = ex2_approx(pv[e] * c2 - lse2);
-        if (need_mask) {
+        for (int e = 0; e < 64; ++e) {
           const int key = k0 + half * 64 + e;
           const bool vis = key < p.Nk && (!p.causal || key <= q) && (p.window_left < 0 || key >= q - p.window_left);
-          pe = vis ? pe : 0.f;
+          pv[e] = vis ? pv[e] : -INFINITY;
         }
-        pv[e] = pe;
       }
+      const float2 c2v = make_float2(c2, c2), nl2 = make_float2(nlse2, nlse2);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t dpv[16];
-        tmem_ld_16x32bx2_x16<64>(tbase + lane_off + C::DP_COL + c * 16, dpv);
-        tmem_wait_ld();
-        uint32_t dw[8];
+      for (int e = 0; e < 64; e += 2) {
+        const float2 x = __ffma2_rn(make_float2(pv[e], pv[e + 1]), c2v, nl2);
+        pv[e] = ex2_approx(x.x);
+        pv[e + 1] = ex2_approx(x.y);
+      }
+      if (threadIdx.x == 128) FA_BTRACE(3, 2, n);
+      // dP(n) (a wait that times out leaves dS unusable; the next vote
+      // reports it)
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim)) && ok;
+      tc_fence_after();
+      float gv[64];
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + Q::DP_COL, reinterpret_cast<uint32_t*>(gv));
+      tmem_ld_16x32bx2_x32<64>(tbase + lane_off + Q::DP_COL + 32, reinterpret_cast<uint32_t*>(gv + 32));
+      tmem_wait_ld();
+      const float2 nd2 = make_float2(-dlt, -dlt);
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float g0 = __uint_as_float(dpv[e]), g1 = __uint_as_float(dpv[e + 1]);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dw[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float2 g = make_float2(gv[32 * c + e], gv[32 * c + e + 1]);
           if constexpr (DROP) {
             // dP of the dropped forward: Z / (1 - p) times dO V^T
-            const uint32_t kb = keep[(c * 16 + e) / 32] >> ((c * 16 + e) % 32);
-            g0 = (kb & 1u) ? g0 * p.drop_scale : 0.f;
-            g1 = (kb & 2u) ? g1 * p.drop_scale : 0.f;
+            const uint32_t kb = keep[c] >> e;
+            g.x = (kb & 1u) ? g.x * p.drop_scale : 0.f;
+            g.y = (kb & 2u) ? g.y * p.drop_scale : 0.f;
           }
-          dw[e / 2] = pack2<DT>(pv[c * 16 + e] * (g0 - dlt), pv[c * 16 + e + 1] * (g1 - dlt));
+          const float2 d = __fmul2_rn(make_float2(pv[32 * c + e], pv[32 * c + e + 1]), __fadd2_rn(g, nd2));
+          dw[e / 2] = pack2<DT>(d.x, d.y);
         }
-        tmem_st_16x32bx2_x8<32>(tbase + lane_off + C::P_COL + c * 8, dw);
+        // dS for the thread's keys 32c .. 32c + 31 over S(n)'s upper half
+        tmem_st_16x32bx2_x16<32>(tbase + lane_off + s_col + 64 + c * 16, dw);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&sh->ds_ready));
+      if (threadIdx.x == 128) FA_BTRACE(3, 3, n);
     }
-    if (!ok && threadIdx.x == 128) atomicOr(p.status, ST_TIMEOUT_SOFTMAX);
+    if (!grad_bar_and(ok)) {
+      ok = false;
+      if (threadIdx.x == 128) atomicOr(p.status, ST_TIMEOUT_SOFTMAX);
+    }
     // dQ = scale * (sum over key blocks of dS K), 16-bit
     bool have = ok && cnt > 0;
     if (have) {
@@ -719,14 +840,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     // (the TMEM loads are warp-collective: every lane takes them, whatever
     // its row; only rows inside N_q are stored)
-    if (have || cnt == 0) {
+    if (have || (ok && cnt == 0)) {
       uint8_t* dq_row = reinterpret_cast<uint8_t*>(p.dq) +
                         (((static_cast<long long>(b) * p.Nq + q) * p.H + h) * D + half * (D / 2)) * 2;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[16];
         if (cnt > 0) {
-          tmem_ld_16x32bx2_x16<D / 2>(tbase + lane_off + C::DQ_COL + c * 16, v);
+          tmem_ld_16x32bx2_x16<D / 2>(tbase + lane_off + Q::DQ_COL + c * 16, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -744,34 +865,42 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   }
 }
 
-// D_i = sum_d dO_id O_id (fp32) for every (b, h, i).  One warp per (b, i, h)
-// row.
+// D_i = sum_d dO_id O_id (fp32) for every (b, h, i).  Each thread reads 16
+// bytes of O and of dO (8 elements); the D / 8 threads of a row add theirs
+// with shuffles.  Whole warps step through the grid-stride loop together.
 template <int D>
 __global__ void fa_bwd_prologue_kernel(const void* __restrict__ out, const void* __restrict__ dout, int dt,
                                        float* __restrict__ delta, int B, int Nq, int H) {
-  constexpr int PER = D / 32;
-  const long long rows = static_cast<long long>(B) * Nq * H;
+  constexpr int TPR = D / 8;   // threads per row
+  const long long total = static_cast<long long>(B) * Nq * H * TPR;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const int lane = static_cast<int>(threadIdx.x & 31u);
-  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x / 32) + threadIdx.x / 32; i < rows; i += warps) {
+  const uint4* o4 = reinterpret_cast<const uint4*>(out);
+  const uint4* g4 = reinterpret_cast<const uint4*>(dout);
+  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g - lane < total; g += stride) {
     float acc = 0.f;
-    const long long base = i * D + lane * PER;
+    if (g < total) {
+      const uint4 ov = __ldg(o4 + g), gv = __ldg(g4 + g);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      float o, g;
-      if (dt == DT_BF16) {
-        o = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(out)[base + e]);
-        g = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(dout)[base + e]);
-      } else {
-        o = __half2float(reinterpret_cast<const __half*>(out)[base + e]);
-        g = __half2float(reinterpret_cast<const __half*>(dout)[base + e]);
+      for (int e = 0; e < 4; ++e) {
+        float2 of, gf;
+        if (dt == DT_BF16) {
+          of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[e]));
+          gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[e]));
+        } else {
+          of = __half22float2(*reinterpret_cast<const __half2*>(&ow[e]));
+          gf = __half22float2(*reinterpret_cast<const __half2*>(&gw[e]));
+        }
+        acc = fmaf(of.x, gf.x, acc);
+        acc = fmaf(of.y, gf.y, acc);
       }
-      acc = fmaf(o, g, acc);
     }
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-    if (lane == 0) {
-      // i enumerates (b, n, h); D_i is stored [B, H, N_q] like the LSE
+    for (int m = TPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (g < total && (lane % TPR) == 0) {
+      // row g / TPR enumerates (b, n, h); D_i is stored [B, H, N_q] like the LSE
+      const long long i = g / TPR;
       const long long h = i % H, bn = i / H, nq = bn % Nq, bb = bn / Nq;
       delta[(bb * H + h) * Nq + nq] = acc;
     }

@@ -544,7 +544,7 @@ int fa_wait_probe(unsigned long long limit_ns, fa_stream_t stream) {
 }
 
 int fa_exp2_check(const float* x, float* poly, float* mufu, int n, int degree, fa_stream_t stream) {
-  if (n < 0 || (degree != 2 && degree != 3)) return FA_ERR_ARG;
+  if (n < 0 || (degree != 2 && degree != 3 && degree != 5)) return FA_ERR_ARG;
   if (n == 0) return FA_OK;
   if (!x || !poly || !mufu) return FA_ERR_ARG;
   const int threads = 256;

@@ -40,13 +40,40 @@ namespace fa {
 
 // Timeline records of CTA 0 (see the forward's tracer); compiled out unless
 // FA_TRACE_BUILD is defined.
+// FA_BTRACE_W: lane 0 of every gradient warp w = 4..11 into slice base + w - 4.
 #ifdef FA_TRACE_BUILD
 #define FA_BTRACE_DECL FA_TRACE_DECL
 #define FA_BTRACE(who, ev, j) FA_TRACE(who, ev, j)
+#define FA_BTRACE_WDECL unsigned trace_w = 0
+#define FA_BTRACE_W(base, ev, j)                                                                     \
+  do {                                                                                               \
+    if (blockIdx.x == 0 && (threadIdx.x & 31u) == 0 && g_trace && trace_w < kTraceSlice)            \
+      g_trace[((base) + threadIdx.x / 32 - 4) * kTraceSlice + trace_w++] =                           \
+          (static_cast<unsigned long long>((ev) & 0xff) << 48) |                                    \
+          (static_cast<unsigned long long>((j) & 0xffff) << 32) |                                   \
+          (static_cast<unsigned long long>(clock64()) & 0xffffffffull);                             \
+  } while (0)
 #else
 #define FA_BTRACE_DECL do { } while (0)
 #define FA_BTRACE(who, ev, j) do { } while (0)
+#define FA_BTRACE_WDECL do { } while (0)
+#define FA_BTRACE_W(base, ev, j) do { } while (0)
 #endif
+
+// Exponentials of P taken on the FMA pipe: in blocks without masked keys,
+// pairs i with i mod 8 >= 8 - FA_BWD_EMU of a thread's 32 take the degree-5
+// polynomial (relative error 2.2e-7, like ex2.approx) instead of MUFU.  Off
+// by default: measured on B200, 2, 3 and 4 of 8 were 0.6-2.8 % slower (the
+// exponential unit does not bind the backward).
+#ifndef FA_BWD_EMU
+#define FA_BWD_EMU 0
+#endif
+
+// 2^x of pair i (i a compile-time constant after unrolling).
+__device__ __forceinline__ float2 bwd_exp2_pair(float2 x, int i, bool emulate) {
+  if (emulate && (i % 8) >= 8 - FA_BWD_EMU) return exp2_poly2<5>(x);
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
 
 struct BwdParams {
   void* dk;                 // [B, N_k, H, D], 16-bit like the inputs
@@ -95,6 +122,7 @@ struct BwdHeader {
   uint64_t pt_free;                   // dV has read P^T
   uint64_t ds_ready;                  // dS^T in TMEM
   uint64_t dkv_full;                  // every MMA of the CTA done
+  uint64_t stat_full[2], stat_empty[2];   // row statistics of a visit: loaded / read
   uint32_t tmem_base;
   int abort_flag;
   // -LSE * log2(e) (-inf: the row contributes nothing) and -D of the query
@@ -107,11 +135,15 @@ struct BwdHeader {
 __device__ __forceinline__ int stat_slot(int q) { return ((q & 63) >> 2) * 8 + (q >> 6) * 4 + (q & 3); }
 static_assert(sizeof(BwdHeader) <= 3072, "backward header");
 
-constexpr int BWD_THREADS = 384;      // warpgroup 0: load + MMA; warps 4-11: gradients
+constexpr int BWD_THREADS = 384;      // warpgroup 0: loads + MMA; warps 4-11: gradients
 
 __device__ __forceinline__ void bwd_error(BwdHeader* sh, const BwdParams& p, int code) {
   atomicOr(p.status, code);
   atomicExch(&sh->abort_flag, 1);
+}
+
+__device__ __forceinline__ bool bwd_aborted(const int* flag) {
+  return *reinterpret_cast<const volatile int*>(flag) != 0;
 }
 
 // Barrier 1 over the 256 gradient threads that also ANDs a flag across
@@ -187,6 +219,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(smem_u32(&sh->pt_free), 1);
     mbar_init(smem_u32(&sh->ds_ready), 256);
     mbar_init(smem_u32(&sh->dkv_full), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&sh->stat_full[s]), 64);
+      mbar_init(smem_u32(&sh->stat_empty[s]), 256);
+    }
     sh->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_map(&tm_q);
@@ -326,7 +362,39 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mma_commit(smem_u32(&sh->dkv_full));   // also: every MMA done before TMEM is released
       if (!ok) mbar_wait(smem_u32(&sh->dkv_full), 0, lim);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // ---------------------------------------------------- row statistics
+    // Warps 2-3 load, per visit, -LSE log2(e) and -D of the query block's
+    // 128 rows (two per thread) into stat buffer n mod 2, once the gradient
+    // warps have released it (rows past N_q: -inf and 0, so they contribute
+    // nothing)
+    const int u = static_cast<int>(threadIdx.x) - 64;   // 0..63
+    int qn = 0, ib = 0;   // visit n = qn * cnt + ib: query head hk * qpk + qn, block (ib + rot) mod cnt
+    for (int n = 0; n < visits; ++n) {
+      const int s = n & 1;
+      if (!mbar_wait(smem_u32(&sh->stat_empty[s]), ((n >> 1) & 1) ^ 1, lim)) {
+        if (u == 0) bwd_error(sh, p, ST_TIMEOUT_LOAD);
+        break;
+      }
+      const int hq = hk * p.qpk + qn;
+      const int i = i_lo + (ib + rot < cnt ? ib + rot : ib + rot - cnt);
+      const long long base = (static_cast<long long>(b) * p.H + hq) * p.Nq;
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int ql = 2 * u + x, q = i * 128 + ql;
+        float nl = -INFINITY, nd = 0.f;
+        if (q < p.Nq) {
+          const float l = p.lse[base + q];
+          if (l != -INFINITY) nl = l * -1.4426950408889634f;
+          nd = -p.delta[base + q];
+        }
+        sh->nlse2[s][stat_slot(ql)] = nl;
+        sh->ndelta[s][stat_slot(ql)] = nd;
+      }
+      mbar_arrive(smem_u32(&sh->stat_full[s]));   // release: the stores above are seen after the wait
+      if (++ib == cnt) { ib = 0; ++qn; }
+    }
+  } else {
     // ---------------------------------------------------------- gradients
     const int quad = warp & 3;
     const int sub = (warp - 4) >> 2;
@@ -334,35 +402,25 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int half = lane >> 4;
     const int r = quad * 32 + sub * 16 + (lane & 15);           // TMEM lane: key
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32 + sub * 16) << 16;
-    const int t = static_cast<int>(threadIdx.x) - 128;          // 0..255
     const int key = jk * 128 + r;
     const float c2 = p.score_scale;
     uint8_t* pt_row = smem + C::OFF_PT + half * C::CHUNK + r * 128;
+    // Each warp takes its own exit decision: a wait that runs out records
+    // the error and raises the CTA's abort flag, which every warp checks
+    // once per visit (all waits are bounded, so no warp is left behind for
+    // long); the vote after the loop then agrees on the outcome.
     bool ok = true;
-    bool dq_ok = true;   // this block's later waits (reported at the next vote)
-    // one row statistic per thread (threads 0-127: LSE, 128-255: D) of
-    // visit m, loaded a visit ahead
-    auto load_stat = [&](int m) -> float {
-      const int hq = hk * p.qpk + m / cnt;
-      const int q = (i_lo + (m % cnt + rot) % cnt) * 128 + (t & 127);
-      if (q >= p.Nq) return t < 128 ? -INFINITY : 0.f;   // rows past N_q contribute nothing
-      const long long at = (static_cast<long long>(b) * p.H + hq) * p.Nq + q;
-      if (t >= 128) return -p.delta[at];
-      const float l = p.lse[at];
-      return l != -INFINITY ? l * -1.4426950408889634f : -INFINITY;
-    };
-    float stat = visits > 0 ? load_stat(0) : 0.f;
     FA_BTRACE_DECL;
+    FA_BTRACE_WDECL;
+    int qn = 0, ib = 0;   // visit n = qn * cnt + ib
     for (int n = 0; n < visits; ++n) {
       FA_BTRACE(0, 0, n);
-      const int hq = hk * p.qpk + n / cnt;
-      const int i = i_lo + (n % cnt + rot) % cnt;
+      FA_BTRACE_W(4, 0, n);
+      if (__any_sync(0xffffffffu, bwd_aborted(&sh->abort_flag))) { ok = false; break; }
+      const int hq = hk * p.qpk + qn;
+      const int i = i_lo + (ib + rot < cnt ? ib + rot : ib + rot - cnt);
+      if (++ib == cnt) { ib = 0; ++qn; }
       const int buf = n & 1;
-      // row statistics of query block i; the vote below is also the
-      // barrier that publishes them (buffer buf was last read in visit
-      // n - 2, before every thread's vote of visit n - 1)
-      (t < 128 ? sh->nlse2[buf] : sh->ndelta[buf])[stat_slot(t & 127)] = stat;
-      if (n + 1 < visits) stat = load_stat(n + 1);
       const int q0 = i * 128;
       const bool need_mask = (jk * 128 + 128 > p.Nk) || (p.causal && jk * 128 + 127 > q0) ||
                              (p.window_left >= 0 && jk * 128 < q0 + 127 - p.window_left);
@@ -388,12 +446,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           keep[m / 4] |= got8 << (8 * (m % 4));
         }
       }
-      const bool got = mbar_wait(smem_u32(&sh->s_full), n & 1, lim);
-      if (!grad_bar_and(got && dq_ok)) {
+      FA_BTRACE_W(4, 1, n);
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->s_full), n & 1, lim) &&
+                                       mbar_wait(smem_u32(&sh->stat_full[buf]), (n >> 1) & 1, lim))) {
+        if (lane == 0) bwd_error(sh, p, ST_TIMEOUT_SOFTMAX);
         ok = false;
         break;
       }
+      FA_BTRACE_W(4, 2, n);
       FA_BTRACE(0, 1, n);
+      FA_BTRACE_W(4, 3, n);
       tc_fence_after();
       // the thread's half row of S^T (queries half * 64 + [0, 64)); the MMA
       // may overwrite S^T with the next block's once every thread has it
@@ -413,22 +475,29 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
       }
       // P = 2^(S c2 - LSE log2 e), the statistic held negated; queries
-      // e..e+3 at [2 (e / 4)]
+      // e..e+3 at [2 (e / 4)].  Two copies of the loop, so that no branch
+      // sits between its exponentials
       const float4* nl4 = reinterpret_cast<const float4*>(sh->nlse2[buf]) + half;
       const float2 c2v = make_float2(c2, c2);
+      auto p_block = [&](bool emulate) {
 #pragma unroll
-      for (int e4 = 0; e4 < 16; ++e4) {
-        const float4 l4 = nl4[2 * e4];
-        const float2 x0 = __ffma2_rn(make_float2(pv[4 * e4], pv[4 * e4 + 1]), c2v, make_float2(l4.x, l4.y));
-        const float2 x1 = __ffma2_rn(make_float2(pv[4 * e4 + 2], pv[4 * e4 + 3]), c2v, make_float2(l4.z, l4.w));
-        pv[4 * e4] = ex2_approx(x0.x);
-        pv[4 * e4 + 1] = ex2_approx(x0.y);
-        pv[4 * e4 + 2] = ex2_approx(x1.x);
-        pv[4 * e4 + 3] = ex2_approx(x1.y);
-      }
+        for (int e4 = 0; e4 < 16; ++e4) {
+          const float4 l4 = nl4[2 * e4];
+          const float2 x0 = __ffma2_rn(make_float2(pv[4 * e4], pv[4 * e4 + 1]), c2v, make_float2(l4.x, l4.y));
+          const float2 x1 = __ffma2_rn(make_float2(pv[4 * e4 + 2], pv[4 * e4 + 3]), c2v, make_float2(l4.z, l4.w));
+          const float2 y0 = bwd_exp2_pair(x0, 2 * e4, emulate), y1 = bwd_exp2_pair(x1, 2 * e4 + 1, emulate);
+          pv[4 * e4] = y0.x, pv[4 * e4 + 1] = y0.y, pv[4 * e4 + 2] = y1.x, pv[4 * e4 + 3] = y1.y;
+        }
+      };
+      if (need_mask) p_block(false);
+      else p_block(true);
       FA_BTRACE(0, 2, n);
       // P^T(n - 1) in shared memory has been read by dV(n - 1)
-      if (n > 0) dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->pt_free), (n - 1) & 1, lim)) && dq_ok;
+      if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->pt_free), (n - 1) & 1, lim))) {
+        if (lane == 0) bwd_error(sh, p, ST_TIMEOUT_SOFTMAX);
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         // P^T for queries half * 64 + [16c, 16c + 16) (dV takes the kept
@@ -452,9 +521,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       fence_proxy_async_smem();   // P^T stores visible to the MMA's reads
       mbar_arrive(smem_u32(&sh->p_ready));
       // dP^T(n): the warp reads all of it before any dS^T store lands over
-      // its upper half (a wait that times out leaves dS unusable; the next
-      // vote reports it)
-      dq_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim)) && dq_ok;
+      // its upper half
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim))) {
+        if (lane == 0) bwd_error(sh, p, ST_TIMEOUT_SOFTMAX);
+        ok = false;
+        break;
+      }
       FA_BTRACE(0, 3, n);
       tc_fence_after();
       float gv[64];
@@ -490,9 +562,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&sh->ds_ready));
+      mbar_arrive(smem_u32(&sh->stat_empty[buf]));   // this visit's statistics read
       FA_BTRACE(0, 4, n);
+      FA_BTRACE_W(4, 4, n);
     }
-    if (!grad_bar_and(ok && dq_ok)) {
+    if (!grad_bar_and(ok)) {
       ok = false;
       if (threadIdx.x == 128) bwd_error(sh, p, ST_TIMEOUT_SOFTMAX);
     }
@@ -558,6 +632,11 @@ struct DqHeader {
   int abort_flag;
 };
 static_assert(sizeof(DqHeader) <= 1024, "dQ header");
+
+__device__ __forceinline__ void dq_error(DqHeader* sh, const BwdParams& p, int code) {
+  atomicOr(p.status, code);
+  atomicExch(&sh->abort_flag, 1);
+}
 
 template <int D>
 struct DqCfg {
@@ -659,7 +738,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       if (!ok) {
         // drain: the copies already issued land before the CTA exits
-        atomicOr(p.status, ST_TIMEOUT_LOAD);
+        dq_error(sh, p, ST_TIMEOUT_LOAD);
         mbar_wait(smem_u32(&sh->q_full), 0, lim);
         for (int m = max(0, nk - 3); m < nk; ++m) mbar_wait(smem_u32(&sh->k_full[m % 3]), (m / 3) & 1, lim);
         for (int m = max(0, nv - 2); m < nv; ++m) mbar_wait(smem_u32(&sh->v_full[m & 1]), (m >> 1) & 1, lim);
@@ -706,9 +785,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       };
       bool ok = mbar_wait(smem_u32(&sh->q_full), 0, lim) && issue_s(0) && issue_dp(0) && (cnt < 2 || issue_s(1));
       for (int n = 0; n < cnt && ok; ++n) {
-        FA_BTRACE(4, 0, n);
+        FA_BTRACE(12, 0, n);
         if (!mbar_wait(smem_u32(&sh->ds_ready), n & 1, lim)) { ok = false; break; }
-        FA_BTRACE(4, 1, n);
+        FA_BTRACE(12, 1, n);
         tc_fence_after();
         // dP(n+1) over dP(n): the gradient warps read dP(n) before dS(n)
         if (n + 1 < cnt && !issue_dp(n + 1)) { ok = false; break; }
@@ -721,12 +800,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_f16_ts_lo(tbase + Q::DQ_COL, tbase + ds_col + kk * 8, k_mn + off, HI, ID_Q, n > 0 || kk > 0);
         }
         mma_commit(smem_u32(&sh->k_empty[n % 3]));   // last reader of K_n
-        FA_BTRACE(4, 2, n);
+        FA_BTRACE(12, 2, n);
         // S(n+2) over S(n) and dS(n), after dQ(n) (same pipe, in order)
         if (n + 2 < cnt && !issue_s(n + 2)) { ok = false; break; }
-        FA_BTRACE(4, 3, n);
+        FA_BTRACE(12, 3, n);
       }
-      if (!ok) atomicOr(p.status, ST_TIMEOUT_MMA);
+      if (!ok) dq_error(sh, p, ST_TIMEOUT_MMA);
       mma_commit(smem_u32(&sh->dq_done));
       if (!ok) mbar_wait(smem_u32(&sh->dq_done), 0, lim);
     }
@@ -747,10 +826,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       dlt = p.delta[bhq + q];
     }
     const float c2 = p.score_scale;
+    // Each warp takes its own exit decision (see the dK/dV kernel); the
+    // vote after the loop agrees on the outcome
     bool ok = true;
     FA_BTRACE_DECL;
+    FA_BTRACE_WDECL;
     for (int n = 0; n < cnt; ++n) {
       if (threadIdx.x == 128) FA_BTRACE(3, 0, n);
+      FA_BTRACE_W(16, 0, n);
+      if (__any_sync(0xffffffffu, bwd_aborted(&sh->abort_flag))) { ok = false; break; }
       const int k0 = (j_lo + n) * 128;
       const uint32_t s_col = (n & 1) ? Q::S_COL1 : Q::S_COL0;
       const bool need_mask = (k0 + 128 > p.Nk) || (p.causal && k0 + 127 > q0) ||
@@ -766,12 +850,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                                     p.drop_threshold)
                          << (8 * (g % 4));
       }
-      // exit vote: this S landed, and every earlier wait of every warp held
-      if (!grad_bar_and(ok && mbar_wait(smem_u32(&sh->s_full[n & 1]), (n >> 1) & 1, lim))) {
+      FA_BTRACE_W(16, 1, n);
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->s_full[n & 1]), (n >> 1) & 1, lim))) {
+        if (lane == 0) dq_error(sh, p, ST_TIMEOUT_SOFTMAX);
         ok = false;
         break;
       }
+      FA_BTRACE_W(16, 2, n);
       if (threadIdx.x == 128) FA_BTRACE(3, 1, n);
+      FA_BTRACE_W(16, 3, n);
       tc_fence_after();
       // the whole half row of S (keys half * 64 + [0, 64)) before any dS store
       float pv[64];
@@ -787,17 +874,25 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           pv[e] = vis ? pv[e] : -INFINITY;
         }
       }
+      // P = 2^(S c2 - LSE log2 e); two copies of the loop, so that no
+      // branch sits between its exponentials
       const float2 c2v = make_float2(c2, c2), nl2 = make_float2(nlse2, nlse2);
+      auto p_block = [&](bool emulate) {
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        const float2 x = __ffma2_rn(make_float2(pv[e], pv[e + 1]), c2v, nl2);
-        pv[e] = ex2_approx(x.x);
-        pv[e + 1] = ex2_approx(x.y);
-      }
+        for (int e = 0; e < 64; e += 2) {
+          const float2 y = bwd_exp2_pair(__ffma2_rn(make_float2(pv[e], pv[e + 1]), c2v, nl2), e / 2, emulate);
+          pv[e] = y.x, pv[e + 1] = y.y;
+        }
+      };
+      if (need_mask) p_block(false);
+      else p_block(true);
       if (threadIdx.x == 128) FA_BTRACE(3, 2, n);
-      // dP(n) (a wait that times out leaves dS unusable; the next vote
-      // reports it)
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim)) && ok;
+      // dP(n)
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->dp_full), n & 1, lim))) {
+        if (lane == 0) dq_error(sh, p, ST_TIMEOUT_SOFTMAX);
+        ok = false;
+        break;
+      }
       tc_fence_after();
       float gv[64];
       tmem_ld_16x32bx2_x32<64>(tbase + lane_off + Q::DP_COL, reinterpret_cast<uint32_t*>(gv));
@@ -826,6 +921,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_before();
       mbar_arrive(smem_u32(&sh->ds_ready));
       if (threadIdx.x == 128) FA_BTRACE(3, 3, n);
+      FA_BTRACE_W(16, 4, n);
     }
     if (!grad_bar_and(ok)) {
       ok = false;

@@ -822,7 +822,9 @@ __device__ __forceinline__ void store_part_row16(float* dst, const float* o, flo
 
 // Coefficients of 2^f on f in [-1/2, 1/2], fitted by the Remez exchange on
 // relative error (csrc/gen_exp2_poly.py): degree 3, max relative error
-// 7.5e-5 (below the 16-bit P rounding); degree 2, 1.7e-3 (far below e4m3's).
+// 7.5e-5 (below the 16-bit P rounding); degree 2, 1.7e-3 (far below e4m3's);
+// degree 5, 2.2e-7 (as close as ex2.approx itself, for the backward, whose
+// P also enters dS in fp32).
 
 // 2^x on the FMA pipe for a pair of finite x (unmasked blocks only).
 // Range reduction for base 2 is exact: x = j + f with j = round(x) and
@@ -838,7 +840,14 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
   const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
   float2 q;
-  if constexpr (DEG == 3) {
+  if constexpr (DEG == 5) {
+    q = __ffma2_rn(make_float2(0.0013276472454890609f, 0.0013276472454890609f), f,
+                   make_float2(0.009675540961325169f, 0.009675540961325169f));
+    q = __ffma2_rn(q, f, make_float2(0.05550713092088699f, 0.05550713092088699f));
+    q = __ffma2_rn(q, f, make_float2(0.24022120237350464f, 0.24022120237350464f));
+    q = __ffma2_rn(q, f, make_float2(0.6931469440460205f, 0.6931469440460205f));
+    q = __ffma2_rn(q, f, make_float2(1.0000001192092896f, 1.0000001192092896f));
+  } else if constexpr (DEG == 3) {
     q = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
                    make_float2(0.2426111251115799f, 0.2426111251115799f));
     q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
@@ -1355,7 +1364,7 @@ __global__ void fa_exp2_check_kernel(const float* __restrict__ x, float* __restr
                                      float* __restrict__ mufu, int n, int degree) {
   for (int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * gridDim.x * blockDim.x) {
     const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
-    const float2 r = degree == 2 ? exp2_poly2<2>(v) : exp2_poly2<3>(v);
+    const float2 r = degree == 2 ? exp2_poly2<2>(v) : degree == 5 ? exp2_poly2<5>(v) : exp2_poly2<3>(v);
     poly[i] = r.x;
     mufu[i] = ex2_approx(v.x);
     if (i + 1 < n) {

@@ -327,9 +327,10 @@ int fa_wait_probe(unsigned long long limit_ns, fa_stream_t stream);
 
 /*
  * fa_exp2_check -- diagnostic: for the n device floats x, writes 2^x as the
- * forward's FMA-pipe polynomial of the given degree (2 or 3) takes it into
- * poly, and as the exponential unit's approximation (ex2.approx.ftz) takes
- * it into mufu, both device arrays of n floats.  The polynomial clamps x at
+ * FMA-pipe polynomial of the given degree (2 or 3: the forward's; 5: the
+ * backward's) takes it into poly, and as the exponential unit's
+ * approximation (ex2.approx.ftz) takes it into mufu, both device arrays of
+ * n floats.  The polynomial clamps x at
  * -125 (2^x below 2^-124 comes out as about 2^-125).  Runs on `stream`;
  * FA_ERR_ARG for n < 0, another degree or a NULL pointer with n > 0.
  */

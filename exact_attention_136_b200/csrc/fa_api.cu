@@ -122,7 +122,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 template <int D, int DT, bool SPLIT, int MASK = MASK_NONE>
 int launch(const void* q, const void* k, const void* v, const FwdParams& base, cudaStream_t stream,
            DeviceState* ds, int bit, unsigned* sched_override) {
-  using C = Cfg<D, DT>;
+  using C = Cfg<D, DT, MASK>;
   FwdParams p = base;
   const CUtensorMapDataType tdt = DT == DT_FP16   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                   : DT == DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -135,6 +135,13 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
       encode_bnhd(&mk, k, tdt, C::ES, mb, mnk, p.Hkv, D, C::BOX_INNER, BLOCK_N) ||
       encode_bnhd(&mv, v, tdt, C::ES, mb, mnk, p.Hkv, D, C::BOX_INNER, BLOCK_N))
     return FA_ERR_CUDA;
+  // the attention mask's map (other variants get an unused copy of Q's)
+  CUtensorMap mm = mq;
+  if constexpr (C::TMA_MASK) {
+    const CUtensorMapDataType mdt = MASK == MASK_BOOL ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+    if (encode_mask(&mm, p.mask, mdt, C::MES, p.B, p.H, p.Nq, p.Nk, p.mask_sb, p.mask_sh, p.mask_sq, 128 / C::MES))
+      return FA_ERR_CUDA;
+  }
   if (!(ds->attr_set.load(std::memory_order_acquire) & (1u << bit))) {
     // The per-role register split (setmaxnreg) redistributes the registers
     // the CTA was launched with; it is only valid for the launch count it
@@ -152,7 +159,7 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     int rc = sched_counters(ds, stream, &p.sched);
     if (rc != FA_OK) return rc;
   }
-  fa_fwd_kernel<D, DT, SPLIT, MASK><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  fa_fwd_kernel<D, DT, SPLIT, MASK><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mm, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

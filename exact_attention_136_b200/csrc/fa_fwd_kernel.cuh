@@ -129,23 +129,31 @@ constexpr int NUM_THREADS = 640;   // warpgroup 0: load + MMA; 2 warpgroups per 
 constexpr int HEADER_BYTES = 1024;  // mbarriers and flags
 constexpr int XCH_BYTES = 0;        // (no shared-memory exchange)
 
-template <int D, int DT>
+template <int D, int DT, int MASK = 0>
 struct Cfg {
   static constexpr int ES = DT == DT_E4M3 ? 1 : 2;           // input element bytes
   static constexpr int TILE_BYTES = 128 * D * ES;            // one 128-row tile
   static constexpr int BOX_INNER = 128 / ES;                 // elements per 128-byte row
   static constexpr int NCHUNK = D * ES / 128;                // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = 128 * 128;              // one chunk of 128 rows
+  // Attention-mask tiles (boolean: 1 byte, additive: 2 bytes per element)
+  // staged by TMA: per Q tile, M_SLOTS slots of 128 rows x 128 keys
+  static constexpr bool TMA_MASK = MASK == MASK_BOOL || MASK == MASK_ADD;
+  static constexpr int MES = MASK == MASK_BOOL ? 1 : 2;
+  static constexpr int M_TILE = 128 * 128 * MES;
+  static constexpr int M_SLOTS = MASK == MASK_BOOL ? 2 : (MASK == MASK_ADD ? 1 : 0);
+  static constexpr int M_BYTES = 2 * M_SLOTS * M_TILE;
   // K/V ring slots: whatever shared memory is left after the header, the
-  // exchange buffer and Q0, Q1
-  static constexpr int STAGES_FIT = (232448 - HEADER_BYTES - XCH_BYTES - 2 * TILE_BYTES) / TILE_BYTES;
+  // exchange buffer, Q0, Q1 and the mask slots
+  static constexpr int STAGES_FIT = (232448 - HEADER_BYTES - XCH_BYTES - 2 * TILE_BYTES - M_BYTES) / TILE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+  static constexpr int OFF_MASK = (2 + STAGES) * TILE_BYTES;   // from the first Q tile
   static constexpr int KSTEP = DT == DT_E4M3 ? 32 : 16;      // K per MMA instruction
   static constexpr int P_COLS = 128 * ES / 4;                // TMEM columns of one P row
   static constexpr int P_OFF = 64;                           // P column offset inside S_t
   static constexpr int O_COL0 = 256;
   // the dynamic shared memory base is 1024-byte aligned (checked at entry)
-  static constexpr int SMEM_BYTES = HEADER_BYTES + XCH_BYTES + (2 + STAGES) * TILE_BYTES;
+  static constexpr int SMEM_BYTES = HEADER_BYTES + XCH_BYTES + (2 + STAGES) * TILE_BYTES + M_BYTES;
   static constexpr uint32_t FMT = DT == DT_BF16 ? 1u : 0u;
   static constexpr uint32_t IDESC_S = make_idesc(FMT, false, 128, 128);
   static constexpr uint32_t IDESC_O = make_idesc(FMT, true, 128, D);
@@ -165,6 +173,7 @@ struct Cfg {
   static constexpr int EMU_FROM = DT == DT_E4M3 ? FA_EMU_FROM_E4M3 : (D == 64 ? FA_EMU_FROM_D64 : FA_EMU_FROM_D128);
   static constexpr int EMU_DEG = DT == DT_E4M3 ? 2 : 3;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(STAGES >= 3, "K/V ring");
   static_assert(D == 64 || D == 128, "head dim");
 };
 
@@ -173,6 +182,7 @@ struct SharedHeader {
   uint64_t kv_full[12], kv_empty[12];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t p_half[2];   // first half of P_t stored (keys k of the block with k mod 64 < 32)
+  uint64_t m_full[2][2], m_empty[2][2];   // attention-mask slots per Q tile: loaded / read
   uint64_t mma_done;
   uint64_t uq_full[4], uq_empty[4];   // unit queue: producer -> MMA + softmax warps
   int uq[4];                          // claimed unit ids, -1 = no more work
@@ -356,13 +366,17 @@ template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N)); }
 
 // ------------------------------------------------------------------ producer
-template <int D, int DT, bool SPLIT>
+template <int D, int DT, bool SPLIT, int MASK>
 __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMap* mq,
-                              const CUtensorMap* mk, const CUtensorMap* mv, const FwdParams& p) {
-  using C = Cfg<D, DT>;
+                              const CUtensorMap* mk, const CUtensorMap* mv, const CUtensorMap* mm,
+                              const FwdParams& p) {
+  using C = Cfg<D, DT, MASK>;
   uint8_t* sq = tiles;
   uint8_t* ring = tiles + 2 * C::TILE_BYTES;
   uint32_t kv_it = 0;
+  uint32_t m_it[2] = {0u, 0u};   // mask tiles loaded per Q tile
+  uint32_t m_issued = 0;         // bit 2t + s: mask slot s of tile t has had a load
+  uint32_t m_phase = 0;          // ... and the parity of its latest
   uint32_t q_uses = 0;
   uint32_t issued_mask = 0;   // bit s: slot s has had a load
   uint32_t phase_mask = 0;    // bit s: parity of slot s's latest load
@@ -436,6 +450,29 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
         phase_mask = (phase_mask & ~(1u << slot)) | ((round & 1u) << slot);
         ++kv_it;
       }
+      if constexpr (C::TMA_MASK) {
+        // this block's mask tile of each Q tile that computes the block
+        // (rows past N_q and keys past N_k read as zero)
+        const int mh = p.mask_sh != 0 ? w.h : 0, mb = p.mask_sb != 0 ? w.b : 0;
+#pragma unroll
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!w.valid[t] || j < w.lo[t] || j > w.hi[t]) continue;
+          const uint32_t ms = m_it[t] % C::M_SLOTS, mr = m_it[t] / C::M_SLOTS;
+          if (!mbar_wait(smem_u32(&sh->m_empty[t][ms]), (mr & 1u) ^ 1u, p.wait_limit_ns)) {
+            record_error(sh, p, ST_TIMEOUT_LOAD); ok = false; break;
+          }
+          const uint32_t bar = smem_u32(&sh->m_full[t][ms]);
+          mbar_arrive_expect_tx(bar, C::M_TILE);
+          uint8_t* dst = tiles + C::OFF_MASK + (t * C::M_SLOTS + ms) * C::M_TILE;
+#pragma unroll
+          for (int c = 0; c < C::MES; ++c)   // 128-byte column chunks of 128 rows
+            tma_load_4d(smem_u32(dst + c * C::CHUNK_BYTES), mm, bar, j * BLOCK_N + c * (128 / C::MES),
+                        w.q0 + t * BLOCK_M, mh, mb);
+          m_issued |= 1u << (2 * t + ms);
+          m_phase = (m_phase & ~(1u << (2 * t + ms))) | ((mr & 1u) << (2 * t + ms));
+          ++m_it[t];
+        }
+      }
       if (nxt == -2) {
         // claim the next unit while these loads are in flight, and warm L2
         // with its Q tiles
@@ -465,6 +502,13 @@ __device__ void producer_role(SharedHeader* sh, uint8_t* tiles, const CUtensorMa
     for (int t = 0; t < 2; ++t)
       if (((q_loaded >> t) & 1u) && !mbar_wait(smem_u32(&sh->q_full[t]), (q_phase >> t) & 1u, p.wait_limit_ns))
         record_error(sh, p, ST_TIMEOUT_DRAIN);
+    if constexpr (C::TMA_MASK) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (((m_issued >> i) & 1u) &&
+            !mbar_wait(smem_u32(&sh->m_full[i / 2][i % 2]), (m_phase >> i) & 1u, p.wait_limit_ns))
+          record_error(sh, p, ST_TIMEOUT_DRAIN);
+    }
   }
   FA_TRACE(3, 15, 0);
 }
@@ -558,9 +602,9 @@ __device__ __forceinline__ bool issue_pv_handover(uint32_t p_half_bar, uint32_t 
 // MMA groups delays the tensor pipe: per key block the steady state below
 // issues its 32 MMAs with nothing but the four waits, four commits and the
 // ring advance between them; every decision is taken once per unit.
-template <int D, int DT, bool SPLIT>
+template <int D, int DT, bool SPLIT, int MASK>
 __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const FwdParams& p) {
-  using C = Cfg<D, DT>;
+  using C = Cfg<D, DT, MASK>;
   constexpr uint32_t SLOT_DESC = C::TILE_BYTES >> 4;   // descriptor start-address step per ring slot
   const uint32_t ring = smem_u32(tiles + 2 * C::TILE_BYTES);
   const uint32_t q_desc0 = sdesc_sw128_lo(smem_u32(tiles), 16);
@@ -934,8 +978,10 @@ __device__ __forceinline__ float2 exp_half(const float* s, float cc, float neg_m
 // (the tcgen05 16x32bx2 access shape), so the two halves of a row meet with
 // one shuffle and apply identical references and rescale factors.
 template <int D, int DT, bool SPLIT, int MASK>
-__device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, const int sub, const FwdParams& p) {
-  using C = Cfg<D, DT>;
+__device__ void softmax_role(SharedHeader* sh, const uint8_t* tiles, uint32_t tbase, const int t, const int sub,
+                             const FwdParams& p) {
+  using C = Cfg<D, DT, MASK>;
+  uint32_t m_cnt = 0;   // mask tiles of this Q tile consumed (the producer's sequence)
   constexpr int HALF_N = BLOCK_N / 2;
   constexpr int HALF_D = D / 2;
   const int quad = (threadIdx.x / 32) & 3;
@@ -998,37 +1044,14 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
     float m_used = -INFINITY;   // reference max (log2 units) that P and l are taken against
     float l = 0.f;              // this thread's share of the row sum (exact)
     float lq = 0.f;             // ... of the stored P values (differs for e4m3)
-    // this thread's mask row (its 64 keys of each block start at key
-    // k0 + 64 * half); rows past N_q read nothing
-    constexpr bool ATTN_MASK = MASK == MASK_BOOL || MASK == MASK_ADD;
+    constexpr bool ATTN_MASK = C::TMA_MASK;
     constexpr bool DROP = MASK == MASK_DROPOUT;
-    constexpr int MES = MASK == MASK_BOOL ? 1 : 2;   // mask element bytes
-    const uint8_t* mask_row = nullptr;
-    if constexpr (ATTN_MASK) {
-      if (row_ok)
-        mask_row = static_cast<const uint8_t*>(p.mask) +
-                   (static_cast<int64_t>(w.b) * p.mask_sb + static_cast<int64_t>(w.h) * p.mask_sh +
-                    static_cast<int64_t>(row) * p.mask_sq + half * HALF_N) * MES;
-    }
     for (int j = w.lo; j <= w.hi; ++j) {
       // boundary blocks (causal diagonal, window edge, key tail), decided
       // before S arrives
       const int k0 = j * BLOCK_N;
       const bool need_mask = (k0 + BLOCK_N > w.nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
                              (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
-      // the mask values of this block, loaded while S is computed (16-byte
-      // chunks that start at or past N_k are not read)
-      constexpr int MCHUNKS = ATTN_MASK ? HALF_N * MES / 16 : 1;
-      uint4 mk[MCHUNKS];
-      if constexpr (ATTN_MASK) {
-#pragma unroll
-        for (int c = 0; c < MCHUNKS; ++c) {
-          const int key = k0 + half * HALF_N + c * (16 / MES);
-          mk[c] = (mask_row && key < w.nk)
-                      ? __ldg(reinterpret_cast<const uint4*>(mask_row + static_cast<int64_t>(k0) * MES) + c)
-                      : make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
       // dropout keep bits of this thread's keys (bit c: key k0 + 64 * half + c),
       // generated while S is computed
       uint32_t keep[2] = {0u, 0u};
@@ -1052,27 +1075,48 @@ __device__ void softmax_role(SharedHeader* sh, uint32_t tbase, const int t, cons
       tmem_ld_16x32bx2_x32<64>(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
       tmem_wait_ld();
       FA_TRACE(t, 2, j);
-      if constexpr (MASK == MASK_BOOL) {
-        // byte c of the thread's 64: key k0 + 64 * half + c; 0 = masked out
+      // this block's mask values for the thread's 64 keys, from the tile's
+      // slot (staged by the producer's TMA, 128-byte swizzled: 16-byte unit
+      // u of row r at u ^ (r mod 8)), applied one 16-byte unit at a time;
+      // the slot is released once read
+      if constexpr (ATTN_MASK) {
+        const uint32_t ms = C::M_SLOTS == 1 ? 0u : (m_cnt & 1u);
+        const uint32_t mpar = (C::M_SLOTS == 1 ? m_cnt : (m_cnt >> 1)) & 1u;
+        ++m_cnt;
+        bool got_m = mbar_wait(smem_u32(&sh->m_full[t][ms]), mpar, p.wait_limit_ns);
+        got_m = __all_sync(0xffffffffu, got_m);
+        if (!got_m) { record_error(sh, p, ST_TIMEOUT_SOFTMAX); ok = false; break; }
+        // boolean: the row's 128 bytes, keys 64 * half on in units 4 * half ..;
+        // additive: column chunk `half` (64 keys of 2 bytes), units 0-7
+        const uint8_t* mrow = tiles + C::OFF_MASK + (t * C::M_SLOTS + ms) * C::M_TILE +
+                              (C::MES == 2 ? half * C::CHUNK_BYTES : 0) + r * 128;
+        constexpr int KEYS_PER_UNIT = 16 / C::MES;
 #pragma unroll
-        for (int c = 0; c < HALF_N; ++c) {
-          const uint32_t word = reinterpret_cast<const uint32_t*>(mk)[c / 4];
-          if (((word >> (8 * (c % 4))) & 0xffu) == 0u) s[c] = -INFINITY;
-        }
-      } else if constexpr (MASK == MASK_ADD) {
-        // the additive mask goes into the raw score: s + m / (scale * descales)
+        for (int c0 = 0; c0 < HALF_N; c0 += KEYS_PER_UNIT) {
+          const int u = (C::MES == 2 ? 0 : 4 * half) + c0 / KEYS_PER_UNIT;
+          const uint4 v4 = *reinterpret_cast<const uint4*>(mrow + ((u ^ (r & 7)) << 4));
+          const uint32_t wd[4] = {v4.x, v4.y, v4.z, v4.w};
+          if constexpr (MASK == MASK_BOOL) {
+            // byte i: key k0 + 64 * half + c0 + i; 0 = masked out
 #pragma unroll
-        for (int c = 0; c < HALF_N; c += 2) {
-          const uint32_t word = reinterpret_cast<const uint32_t*>(mk)[c / 2];
-          float2 m2;
-          if constexpr (DT == DT_FP16) {
-            m2 = __half22float2(*reinterpret_cast<const __half2*>(&word));
+            for (int i = 0; i < 16; ++i)
+              if (((wd[i / 4] >> (8 * (i % 4))) & 0xffu) == 0u) s[c0 + i] = -INFINITY;
           } else {
-            m2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&word));
+            // the additive mask goes into the raw score: s + m / (scale * descales)
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              float2 m2;
+              if constexpr (DT == DT_FP16) {
+                m2 = __half22float2(*reinterpret_cast<const __half2*>(&wd[i / 2]));
+              } else {
+                m2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[i / 2]));
+              }
+              s[c0 + i] = fmaf(m2.x, p.mask_scale, s[c0 + i]);
+              s[c0 + i + 1] = fmaf(m2.y, p.mask_scale, s[c0 + i + 1]);
+            }
           }
-          s[c] = fmaf(m2.x, p.mask_scale, s[c]);
-          s[c + 1] = fmaf(m2.y, p.mask_scale, s[c + 1]);
         }
+        mbar_arrive(smem_u32(&sh->m_empty[t][ms]));
       }
       if (need_mask) {
         const int kh = k0 + half * HALF_N;
@@ -1207,8 +1251,9 @@ __device__ __forceinline__ void cta_finished(const FwdParams& p) {
 template <int D, int DT, bool SPLIT, int MASK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = Cfg<D, DT>;
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
+                  const FwdParams p) {
+  using C = Cfg<D, DT, MASK>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {
     // 128-byte swizzled tiles need 1024-byte alignment; never expected.  The
@@ -1240,6 +1285,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&sh->o_empty[t]), 256);
     }
     mbar_init(smem_u32(&sh->mma_done), 1);
+    for (int t = 0; t < 2; ++t)
+      for (int ms = 0; ms < 2; ++ms) {
+        mbar_init(smem_u32(&sh->m_full[t][ms]), 1);
+        mbar_init(smem_u32(&sh->m_empty[t][ms]), 256);   // every thread of the tile's softmax warps
+      }
     for (int i = 0; i < 4; ++i) {
       mbar_init(smem_u32(&sh->uq_full[i]), 1);
       mbar_init(smem_u32(&sh->uq_empty[i]), UQ_CONSUMERS);
@@ -1252,6 +1302,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
+    if constexpr (C::TMA_MASK) tma_prefetch_map(&tm_m);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&sh->tmem_base), 512);
@@ -1264,15 +1315,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp < 4) {
     setmaxnreg_dec<REGS_LOAD_MMA>();
-    if (warp == 0 && lane_id() == 0) producer_role<D, DT, SPLIT>(sh, tiles, &tm_q, &tm_k, &tm_v, p);
-    else if (warp == 1 && lane_id() == 0) mma_role<D, DT, SPLIT>(sh, tiles, tbase, p);
+    if (warp == 0 && lane_id() == 0) producer_role<D, DT, SPLIT, MASK>(sh, tiles, &tm_q, &tm_k, &tm_v, &tm_m, p);
+    else if (warp == 1 && lane_id() == 0) mma_role<D, DT, SPLIT, MASK>(sh, tiles, tbase, p);
   } else {
     setmaxnreg_inc<REGS_SOFTMAX>();
     // warps 4-11: tile 0, warps 12-19: tile 1; within a tile the first four
     // warps take the upper 16 rows of each lane quadrant, the next four the lower
     const int t = warp < 12 ? 0 : 1;
     const int sub = ((warp - 4) >> 2) & 1;
-    softmax_role<D, DT, SPLIT, MASK>(sh, tbase, t, sub, p);
+    softmax_role<D, DT, SPLIT, MASK>(sh, tiles, tbase, t, sub, p);
   }
   tc_fence_before();
   __syncthreads();

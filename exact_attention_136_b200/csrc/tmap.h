@@ -45,4 +45,26 @@ inline int encode_bnhd(CUtensorMap* map, const void* base, CUtensorMapDataType d
   return r == CUDA_SUCCESS ? 0 : -2;
 }
 
+// Map over an attention mask [Bm, Hm, N_q, N_k] (keys innermost; row stride
+// sq, head stride sh, batch stride sb in elements, a stride of 0 making that
+// dimension one deep) whose box is `box_inner` keys by 128 rows, 128-byte
+// swizzle.  Rows past N_q and keys past N_k read as zero.  Returns 0 on
+// success.
+inline int encode_mask(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, int B, int H,
+                       int Nq, int Nk, long long sb, long long sh, long long sq, int box_inner) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return -1;
+  const cuuint64_t row = (cuuint64_t)sq * elem_bytes;
+  cuuint64_t dims[4] = {(cuuint64_t)Nk, (cuuint64_t)Nq, (cuuint64_t)(sh != 0 ? H : 1), (cuuint64_t)(sb != 0 ? B : 1)};
+  // a one-deep dimension still needs a valid stride: the row stride
+  cuuint64_t strides[3] = {row, sh != 0 ? (cuuint64_t)sh * elem_bytes : row,
+                           sb != 0 ? (cuuint64_t)sb * elem_bytes : row};
+  cuuint32_t box[4] = {(cuuint32_t)box_inner, 128u, 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -2;
+}
+
 }  // namespace fa

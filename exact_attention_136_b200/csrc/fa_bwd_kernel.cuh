@@ -44,11 +44,13 @@ namespace fa {
 #ifdef FA_TRACE_BUILD
 #define FA_BTRACE_DECL FA_TRACE_DECL
 #define FA_BTRACE(who, ev, j) FA_TRACE(who, ev, j)
-#define FA_BTRACE_WDECL unsigned trace_w = 0
+#define FA_BTRACE_WDECL                                                                              \
+  unsigned trace_w = 0;                                                                              \
+  unsigned long long* const trace_wp = blockIdx.x == 0 ? g_trace : nullptr
 #define FA_BTRACE_W(base, ev, j)                                                                     \
   do {                                                                                               \
-    if (blockIdx.x == 0 && (threadIdx.x & 31u) == 0 && g_trace && trace_w < kTraceSlice)            \
-      g_trace[((base) + threadIdx.x / 32 - 4) * kTraceSlice + trace_w++] =                           \
+    if (trace_wp && (threadIdx.x & 31u) == 0 && trace_w < kTraceSlice)                               \
+      trace_wp[((base) + threadIdx.x / 32 - 4) * kTraceSlice + trace_w++] =                          \
           (static_cast<unsigned long long>((ev) & 0xff) << 48) |                                    \
           (static_cast<unsigned long long>((j) & 0xffff) << 32) |                                   \
           (static_cast<unsigned long long>(clock64()) & 0xffffffffull);                             \
@@ -104,8 +106,12 @@ struct BwdCfg {
   static constexpr int HDR = 3072;                // barriers and the per-stage row statistics
   static constexpr int OFF_K = HDR;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_STAGE = OFF_V + TILE;  // 2 stages of (Q_i, dO_i)
-  static constexpr int OFF_PT = OFF_STAGE + 2 * 2 * TILE;   // P^T, 128 keys x 128 queries
+  // Q_i through three stages: S^T(n+1) wants Q_{n+1} early in visit n,
+  // while Q_{n-1} is read until dK(n-1) at the end of visit n-1.  dO_i
+  // through one: its first reader, dP^T(n+1), comes after its last, dV(n).
+  static constexpr int OFF_Q = OFF_V + TILE;       // 3 stages of Q_i
+  static constexpr int OFF_DO = OFF_Q + 3 * TILE;  // dO_i
+  static constexpr int OFF_PT = OFF_DO + TILE;     // P^T, 128 keys x 128 queries
   static constexpr int SMEM = OFF_PT + 128 * 128 * 2;
   static constexpr int S_COL = 0, DP_COL = 128, DS_COL = 192;   // dS^T (16-bit) over dP^T's upper half
   static constexpr int DV_COL = 256, DK_COL = 256 + D;
@@ -115,7 +121,8 @@ struct BwdCfg {
 
 struct BwdHeader {
   uint64_t kv_full;
-  uint64_t st_full[2], st_empty[2];   // (Q_i, dO_i) stages
+  uint64_t q_full[3], q_empty[3];     // Q_i stages
+  uint64_t do_full, do_empty;         // dO_i
   uint64_t s_full, dp_full;           // S^T, dP^T computed
   uint64_t s_free;                    // every gradient thread holds S^T in registers
   uint64_t p_ready;                   // P^T in shared memory
@@ -208,10 +215,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sh->kv_full), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&sh->st_full[s]), 1);
-      mbar_init(smem_u32(&sh->st_empty[s]), 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(smem_u32(&sh->q_full[s]), 1);
+      mbar_init(smem_u32(&sh->q_empty[s]), 1);
     }
+    mbar_init(smem_u32(&sh->do_full), 1);
+    mbar_init(smem_u32(&sh->do_empty), 1);
     mbar_init(smem_u32(&sh->s_full), 1);
     mbar_init(smem_u32(&sh->s_free), 256);
     mbar_init(smem_u32(&sh->dp_full), 1);
@@ -254,29 +263,39 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tma_load_4d_hint(sbase + C::OFF_V + c * C::CHUNK, &tm_v, smem_u32(&sh->kv_full), c * 64, hk, jk * 128, b,
                          pol_kv);
       }
-      int n = 0;
-      for (; n < visits; ++n) {
+      int nq = 0, nd = 0;   // Q and dO loads issued
+      for (int n = 0; n < visits; ++n) {
         const int hq = hk * p.qpk + n / cnt;
         const int i = i_lo + (n % cnt + rot) % cnt;
-        const int s = n & 1;
-        if (!mbar_wait(smem_u32(&sh->st_empty[s]), ((n >> 1) & 1) ^ 1, lim)) {
+        const int s = n % 3;
+        if (!mbar_wait(smem_u32(&sh->q_empty[s]), ((n / 3) & 1) ^ 1, lim)) {
           bwd_error(sh, p, ST_TIMEOUT_LOAD);
           ok = false;
           break;
         }
-        const uint32_t bar = smem_u32(&sh->st_full[s]);
-        const uint32_t qdst = sbase + C::OFF_STAGE + s * 2 * C::TILE;
-        mbar_arrive_expect_tx(bar, 2 * C::TILE);
+        const uint32_t qbar = smem_u32(&sh->q_full[s]);
+        mbar_arrive_expect_tx(qbar, C::TILE);
 #pragma unroll
-        for (int c = 0; c < C::NCHUNK; ++c) {
-          tma_load_4d_hint(qdst + c * C::CHUNK, &tm_q, bar, c * 64, hq, i * 128, b, pol_q);
-          tma_load_4d_hint(qdst + C::TILE + c * C::CHUNK, &tm_do, bar, c * 64, hq, i * 128, b, pol_q);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d_hint(sbase + C::OFF_Q + s * C::TILE + c * C::CHUNK, &tm_q, qbar, c * 64, hq, i * 128, b, pol_q);
+        ++nq;
+        if (!mbar_wait(smem_u32(&sh->do_empty), (n & 1) ^ 1, lim)) {
+          bwd_error(sh, p, ST_TIMEOUT_LOAD);
+          ok = false;
+          break;
         }
+        const uint32_t dbar = smem_u32(&sh->do_full);
+        mbar_arrive_expect_tx(dbar, C::TILE);
+#pragma unroll
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d_hint(sbase + C::OFF_DO + c * C::CHUNK, &tm_do, dbar, c * 64, hq, i * 128, b, pol_q);
+        ++nd;
       }
       if (!ok) {
         // drain: the copies already issued land before the CTA exits
         mbar_wait(smem_u32(&sh->kv_full), 0, lim);
-        for (int m = max(0, n - 2); m < n; ++m) mbar_wait(smem_u32(&sh->st_full[m & 1]), (m >> 1) & 1, lim);
+        for (int m = max(0, nq - 3); m < nq; ++m) mbar_wait(smem_u32(&sh->q_full[m % 3]), (m / 3) & 1, lim);
+        if (nd > 0) mbar_wait(smem_u32(&sh->do_full), (nd - 1) & 1, lim);
       }
     }
   } else if (warp == 1) {
@@ -290,7 +309,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const uint32_t k_kmaj = sdesc_sw128_lo(sbase + C::OFF_K, 16);
       const uint32_t v_kmaj = sdesc_sw128_lo(sbase + C::OFF_V, 16);
       const uint32_t pt_kmaj = sdesc_sw128_lo(sbase + C::OFF_PT, 16);
-      const uint32_t q_tile0 = sbase + C::OFF_STAGE;
+      const uint32_t q_tile0 = sbase + C::OFF_Q, do_tile = sbase + C::OFF_DO;
       // S^T = K Q_n^T and dP^T = V dO_n^T for the n-th query block (keys on
       // the lanes); both K-major
       auto issue_kmaj = [&](uint32_t col, uint32_t a_kmaj, uint32_t b_tile) {
@@ -306,33 +325,33 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       // warps hold S^T(n) in registers), dV(n) on P^T(n), dK(n) on dS^T(n),
       // then dP^T(n+1) over dP^T(n) and dS^T(n).  The gradient warps form
       // P(n+1) while dV(n), dK(n) and dP^T(n+1) run.
-      bool ok = mbar_wait(smem_u32(&sh->kv_full), 0, lim) && mbar_wait(smem_u32(&sh->st_full[0]), 0, lim);
+      bool ok = mbar_wait(smem_u32(&sh->kv_full), 0, lim) && mbar_wait(smem_u32(&sh->q_full[0]), 0, lim) &&
+                mbar_wait(smem_u32(&sh->do_full), 0, lim);
       if (ok && visits > 0) {
         tc_fence_after();
         issue_kmaj(C::S_COL, k_kmaj, q_tile0);
         mma_commit(smem_u32(&sh->s_full));
-        issue_kmaj(C::DP_COL, v_kmaj, q_tile0 + C::TILE);
+        issue_kmaj(C::DP_COL, v_kmaj, do_tile);
         mma_commit(smem_u32(&sh->dp_full));
       }
       for (int n = 0; n < visits && ok; ++n) {
-        const uint32_t q_tile = q_tile0 + (n & 1) * 2 * C::TILE;
-        const uint32_t q_next = q_tile0 + ((n + 1) & 1) * 2 * C::TILE;
+        const uint32_t q_tile = q_tile0 + (n % 3) * C::TILE;
         if (n + 1 < visits) {
           FA_BTRACE(2, 0, n);
           if (!mbar_wait(smem_u32(&sh->s_free), n & 1, lim) ||
-              !mbar_wait(smem_u32(&sh->st_full[(n + 1) & 1]), ((n + 1) >> 1) & 1, lim)) {
+              !mbar_wait(smem_u32(&sh->q_full[(n + 1) % 3]), ((n + 1) / 3) & 1, lim)) {
             ok = false;
             break;
           }
           FA_BTRACE(2, 1, n);
           tc_fence_after();
-          issue_kmaj(C::S_COL, k_kmaj, q_next);
+          issue_kmaj(C::S_COL, k_kmaj, q_tile0 + ((n + 1) % 3) * C::TILE);
           mma_commit(smem_u32(&sh->s_full));
         }
         if (!mbar_wait(smem_u32(&sh->p_ready), n & 1, lim)) { ok = false; break; }
         FA_BTRACE(2, 2, n);
         tc_fence_after();
-        const uint32_t q_mn = sdesc_sw128_lo(q_tile, C::CHUNK), do_mn = sdesc_sw128_lo(q_tile + C::TILE, C::CHUNK);
+        const uint32_t q_mn = sdesc_sw128_lo(q_tile, C::CHUNK), do_mn = sdesc_sw128_lo(do_tile, C::CHUNK);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // dV += P^T dO_n: A = P^T in shared memory, K-major (16 queries = 32 bytes of a row)
@@ -342,6 +361,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_f16_ss_lo(tbase + C::DV_COL, pt_kmaj + a_off, do_mn + b_off, HI, ID_KV, n > 0 || kk > 0);
         }
         mma_commit(smem_u32(&sh->pt_free));
+        mma_commit(smem_u32(&sh->do_empty));   // dV(n) is dO_n's last reader
         if (!mbar_wait(smem_u32(&sh->ds_ready), n & 1, lim)) { ok = false; break; }
         FA_BTRACE(2, 3, n);
         tc_fence_after();
@@ -351,9 +371,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const uint32_t off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
           mma_f16_ts_lo(tbase + C::DK_COL, tbase + C::DS_COL + kk * 8, q_mn + off, HI, ID_KV, n > 0 || kk > 0);
         }
-        mma_commit(smem_u32(&sh->st_empty[n & 1]));   // last readers of Q_n and dO_n
+        mma_commit(smem_u32(&sh->q_empty[n % 3]));   // dK(n) is Q_n's last reader
         if (n + 1 < visits) {
-          issue_kmaj(C::DP_COL, v_kmaj, q_next + C::TILE);
+          if (!mbar_wait(smem_u32(&sh->do_full), (n + 1) & 1, lim)) { ok = false; break; }
+          tc_fence_after();
+          issue_kmaj(C::DP_COL, v_kmaj, do_tile);
           mma_commit(smem_u32(&sh->dp_full));
         }
         FA_BTRACE(2, 4, n);
@@ -610,19 +632,26 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
 // dQ kernel: one CTA per (batch, head, 128-query block i), head-major, the
 // query blocks with the most keys first.  Warp 0 loads Q_i and dO_i once,
-// then K_j through three stages and V_j through two; warp 1 issues
+// then K_j and V_j through their stages (below); warp 1 issues
 // S = Q_i K_j^T and dP = dO_i V_j^T (queries on the lanes) and, on dS(j),
 // dQ += dS K_j with A = dS from TMEM; warps 4-11 form dS = P * (dP - D) with
 // P = exp(S - LSE).  S is double-buffered in TMEM, so the gradient warps
 // form P(j+1) while the tensor pipe runs dP(j+1), dQ(j) and S(j+2): per key
 // block the MMA thread issues, after dS(j), dP(j+1) (over dP(j), read by
 // then), dQ(j), and S(j+2) into the buffer of S(j) (whose dS(j) dQ(j) has
-// read, in pipe order).  K_j stays until dQ(j), hence the third K stage.
+// read, in pipe order).
 // TMEM: S(even) [0,128), dP [128,256), dQ [256,256+D), S(odd) [384,512);
 // dS (16-bit) over the upper half of its S buffer.
+// K and V stages: K_j is read until dQ(j), V_j only by dP(j), and the two
+// share five tile slots; four K stages and one V stage measured 0.3 % ahead
+// of three and two (S(j+2) no longer waits for K_{j+2} to land).
+#ifndef FA_DQ_KSTAGES
+#define FA_DQ_KSTAGES 4
+#endif
+
 struct DqHeader {
   uint64_t q_full;
-  uint64_t k_full[3], k_empty[3];
+  uint64_t k_full[4], k_empty[4];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2];        // S(j) in buffer j mod 2 computed
   uint64_t dp_full;          // dP(j) computed
@@ -642,9 +671,10 @@ template <int D>
 struct DqCfg {
   static constexpr int TILE = BwdCfg<D>::TILE;
   static constexpr int OFF_Q = 1024, OFF_DO = OFF_Q + TILE;
-  static constexpr int OFF_K = OFF_DO + TILE;           // 3 stages
-  static constexpr int OFF_V = OFF_K + 3 * TILE;        // 2 stages
-  static constexpr int SMEM_USED = OFF_V + 2 * TILE;
+  static constexpr int KS = FA_DQ_KSTAGES, VS = 5 - FA_DQ_KSTAGES;   // K and V stages
+  static constexpr int OFF_K = OFF_DO + TILE;
+  static constexpr int OFF_V = OFF_K + KS * TILE;
+  static constexpr int SMEM_USED = OFF_V + VS * TILE;
   static constexpr uint32_t S_COL0 = 0, S_COL1 = 384, DP_COL = 128, DQ_COL = 256;
   static_assert(SMEM_USED <= 232448, "shared memory budget");
 };
@@ -677,15 +707,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sh->q_full), 1);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < Q::KS; ++s) {
       mbar_init(smem_u32(&sh->k_full[s]), 1);
       mbar_init(smem_u32(&sh->k_empty[s]), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < Q::VS; ++s) {
       mbar_init(smem_u32(&sh->v_full[s]), 1);
       mbar_init(smem_u32(&sh->v_empty[s]), 1);
-      mbar_init(smem_u32(&sh->s_full[s]), 1);
     }
+    for (int s = 0; s < 2; ++s) mbar_init(smem_u32(&sh->s_full[s]), 1);
     mbar_init(smem_u32(&sh->dp_full), 1);
     mbar_init(smem_u32(&sh->ds_ready), 256);
     mbar_init(smem_u32(&sh->dq_done), 1);
@@ -720,15 +750,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       int nk = 0, nv = 0;   // K and V loads issued
       for (int n = 0; n < cnt && ok; ++n) {
         const int j = j_lo + n;
-        const int sk = n % 3, sv = n & 1;
-        if (!mbar_wait(smem_u32(&sh->k_empty[sk]), ((n / 3) & 1) ^ 1, lim)) { ok = false; break; }
+        const int sk = n % Q::KS, sv = n % Q::VS;
+        if (!mbar_wait(smem_u32(&sh->k_empty[sk]), ((n / Q::KS) & 1) ^ 1, lim)) { ok = false; break; }
         mbar_arrive_expect_tx(smem_u32(&sh->k_full[sk]), C::TILE);
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d_hint(sbase + Q::OFF_K + sk * C::TILE + c * C::CHUNK, &tm_k, smem_u32(&sh->k_full[sk]), c * 64,
                            hk, j * 128, b, pol_kv);
         ++nk;
-        if (!mbar_wait(smem_u32(&sh->v_empty[sv]), ((n >> 1) & 1) ^ 1, lim)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&sh->v_empty[sv]), ((n / Q::VS) & 1) ^ 1, lim)) { ok = false; break; }
         mbar_arrive_expect_tx(smem_u32(&sh->v_full[sv]), C::TILE);
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
@@ -740,8 +770,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         // drain: the copies already issued land before the CTA exits
         dq_error(sh, p, ST_TIMEOUT_LOAD);
         mbar_wait(smem_u32(&sh->q_full), 0, lim);
-        for (int m = max(0, nk - 3); m < nk; ++m) mbar_wait(smem_u32(&sh->k_full[m % 3]), (m / 3) & 1, lim);
-        for (int m = max(0, nv - 2); m < nv; ++m) mbar_wait(smem_u32(&sh->v_full[m & 1]), (m >> 1) & 1, lim);
+        for (int m = max(0, nk - Q::KS); m < nk; ++m) mbar_wait(smem_u32(&sh->k_full[m % Q::KS]), (m / Q::KS) & 1, lim);
+        for (int m = max(0, nv - Q::VS); m < nv; ++m) mbar_wait(smem_u32(&sh->v_full[m % Q::VS]), (m / Q::VS) & 1, lim);
       }
     }
   } else if (warp == 1) {
@@ -755,9 +785,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const uint32_t do_kmaj = sdesc_sw128_lo(sbase + Q::OFF_DO, 16);
       // S(n) = Q K_n^T into buffer n mod 2, on K_n landed
       auto issue_s = [&](int n) -> bool {
-        if (!mbar_wait(smem_u32(&sh->k_full[n % 3]), (n / 3) & 1, lim)) return false;
+        if (!mbar_wait(smem_u32(&sh->k_full[n % Q::KS]), (n / Q::KS) & 1, lim)) return false;
+        FA_BTRACE(12, 6, n);
         tc_fence_after();
-        const uint32_t k_kmaj = sdesc_sw128_lo(sbase + Q::OFF_K + (n % 3) * C::TILE, 16);
+        const uint32_t k_kmaj = sdesc_sw128_lo(sbase + Q::OFF_K + (n % Q::KS) * C::TILE, 16);
         const uint32_t col = (n & 1) ? Q::S_COL1 : Q::S_COL0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -765,22 +796,25 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const uint32_t off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
           mma_f16_ss_lo(tbase + col, q_kmaj + off, k_kmaj + off, HI, ID_S, kk > 0);
         }
+        FA_BTRACE(12, 7, n);
         mma_commit(smem_u32(&sh->s_full[n & 1]));
         return true;
       };
       // dP(n) = dO V_n^T, on V_n landed; V_n's stage is free after it
       auto issue_dp = [&](int n) -> bool {
-        if (!mbar_wait(smem_u32(&sh->v_full[n & 1]), (n >> 1) & 1, lim)) return false;
+        if (!mbar_wait(smem_u32(&sh->v_full[n % Q::VS]), (n / Q::VS) & 1, lim)) return false;
+        FA_BTRACE(12, 4, n);
         tc_fence_after();
-        const uint32_t v_kmaj = sdesc_sw128_lo(sbase + Q::OFF_V + (n & 1) * C::TILE, 16);
+        const uint32_t v_kmaj = sdesc_sw128_lo(sbase + Q::OFF_V + (n % Q::VS) * C::TILE, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int byte = kk * 32;
           const uint32_t off = static_cast<uint32_t>(((byte / 128) * C::CHUNK + (byte % 128)) >> 4);
           mma_f16_ss_lo(tbase + Q::DP_COL, do_kmaj + off, v_kmaj + off, HI, ID_S, kk > 0);
         }
+        FA_BTRACE(12, 5, n);
         mma_commit(smem_u32(&sh->dp_full));
-        mma_commit(smem_u32(&sh->v_empty[n & 1]));
+        mma_commit(smem_u32(&sh->v_empty[n % Q::VS]));
         return true;
       };
       bool ok = mbar_wait(smem_u32(&sh->q_full), 0, lim) && issue_s(0) && issue_dp(0) && (cnt < 2 || issue_s(1));
@@ -792,14 +826,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         // dP(n+1) over dP(n): the gradient warps read dP(n) before dS(n)
         if (n + 1 < cnt && !issue_dp(n + 1)) { ok = false; break; }
         // dQ += dS K_n: A = dS (16-bit, upper half of S(n)'s buffer), 16 keys = 8 columns per step
-        const uint32_t k_mn = sdesc_sw128_lo(sbase + Q::OFF_K + (n % 3) * C::TILE, C::CHUNK);
+        const uint32_t k_mn = sdesc_sw128_lo(sbase + Q::OFF_K + (n % Q::KS) * C::TILE, C::CHUNK);
         const uint32_t ds_col = ((n & 1) ? Q::S_COL1 : Q::S_COL0) + 64;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk * 16 * 128) >> 4);
           mma_f16_ts_lo(tbase + Q::DQ_COL, tbase + ds_col + kk * 8, k_mn + off, HI, ID_Q, n > 0 || kk > 0);
         }
-        mma_commit(smem_u32(&sh->k_empty[n % 3]));   // last reader of K_n
+        mma_commit(smem_u32(&sh->k_empty[n % Q::KS]));   // last reader of K_n
         FA_BTRACE(12, 2, n);
         // S(n+2) over S(n) and dS(n), after dQ(n) (same pipe, in order)
         if (n + 2 < cnt && !issue_s(n + 2)) { ok = false; break; }

@@ -299,11 +299,13 @@ __device__ __forceinline__ Unit get_unit(int u, int split, const FwdParams& p) {
 #ifdef FA_TRACE_BUILD
 __device__ unsigned long long* g_trace;
 constexpr int kTraceSlice = 16384;
-#define FA_TRACE_DECL unsigned trace_n = 0
+#define FA_TRACE_DECL                                                                                 \
+  unsigned trace_n = 0;                                                                               \
+  unsigned long long* const trace_p = blockIdx.x == 0 ? g_trace : nullptr
 #define FA_TRACE(who, ev, j)                                                                          \
   do {                                                                                                \
-    if (blockIdx.x == 0 && ((who) >= 2 || threadIdx.x == 128u + 256u * (who)) && g_trace && trace_n < kTraceSlice) \
-      g_trace[(who) * kTraceSlice + trace_n++] =                                                      \
+    if (trace_p && ((who) >= 2 || threadIdx.x == 128u + 256u * (who)) && trace_n < kTraceSlice)       \
+      trace_p[(who) * kTraceSlice + trace_n++] =                                                      \
           (static_cast<unsigned long long>((ev) & 0xff) << 48) |                                     \
           (static_cast<unsigned long long>((j) & 0xffff) << 32) |                                    \
           (static_cast<unsigned long long>(clock64()) & 0xffffffffull);                              \

@@ -301,6 +301,7 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
     p.drop_threshold = static_cast<unsigned>(std::nearbyint(static_cast<double>(dropout_p) * 65536.0));
     p.seed_lo = static_cast<unsigned>(seed & 0xffffffffull);
     p.seed_hi = static_cast<unsigned>(seed >> 32);
+    p.drop_keys = philox_round_keys(p.seed_lo, p.seed_hi);
     p.drop_offset = offset;
     p.out_scale = static_cast<float>(static_cast<double>(vd) / (1.0 - static_cast<double>(dropout_p)));
     switch (dtype * 2 + (D == 128 ? 1 : 0)) {

@@ -113,6 +113,7 @@ int backward(const void* q, const void* k, const void* v, const void* out, const
       p.drop_threshold = static_cast<unsigned>(std::nearbyint(static_cast<double>(dropout_p) * 65536.0));
       p.seed_lo = static_cast<unsigned>(seed & 0xffffffffull);
       p.seed_hi = static_cast<unsigned>(seed >> 32);
+      p.drop_keys = philox_round_keys(p.seed_lo, p.seed_hi);
       p.drop_offset = offset;
       p.drop_scale = static_cast<float>(1.0 / (1.0 - static_cast<double>(dropout_p)));
     }

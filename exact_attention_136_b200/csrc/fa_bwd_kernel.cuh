@@ -95,6 +95,7 @@ struct BwdParams {
   // dropout (DROP kernels): the forward's keep bits (keep_bits8 with these
   // values) and 1 / (1 - p)
   unsigned drop_threshold, seed_lo, seed_hi, drop_offset;
+  PhiloxKeys drop_keys;     // the round keys of (seed_lo, seed_hi)
   float drop_scale;
 };
 
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
           const uint32_t qq = static_cast<uint32_t>(q0 + half * 64 + 8 * m + lane8);
-          const uint32_t mine8 = keep_bits8(grp, qq, bh, p.drop_offset, p.seed_lo, p.seed_hi, p.drop_threshold);
+          const uint32_t mine8 = keep_bits8(grp, qq, bh, p.drop_offset, p.drop_keys, p.drop_threshold);
           uint32_t got8 = 0;
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
@@ -880,7 +881,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const uint32_t bhq = static_cast<uint32_t>(b * p.H + h);
 #pragma unroll
         for (int g = 0; g < 8; ++g)
-          keep[g / 4] |= keep_bits8(g0 + g, static_cast<uint32_t>(q), bhq, p.drop_offset, p.seed_lo, p.seed_hi,
+          keep[g / 4] |= keep_bits8(g0 + g, static_cast<uint32_t>(q), bhq, p.drop_offset, p.drop_keys,
                                     p.drop_threshold)
                          << (8 * (g % 4));
       }

@@ -63,6 +63,23 @@ enum : int {
   ST_SMEM_MISALIGNED = 16,
 };
 
+// Philox4x32-10 round keys: round r uses (seed_lo + r * 0x9E3779B9,
+// seed_hi + r * 0xBB67AE85) mod 2^32.  Computed once on the host and read
+// from the kernel parameters, so a round costs two wide multiplies and two
+// three-input XORs.
+struct PhiloxKeys {
+  unsigned k0[10], k1[10];
+};
+
+inline PhiloxKeys philox_round_keys(unsigned seed_lo, unsigned seed_hi) {
+  PhiloxKeys k;
+  for (int r = 0; r < 10; ++r) {
+    k.k0[r] = seed_lo + static_cast<unsigned>(r) * 0x9E3779B9u;
+    k.k1[r] = seed_hi + static_cast<unsigned>(r) * 0xBB67AE85u;
+  }
+  return k;
+}
+
 struct FwdParams {
   void* out;           // [B, N_q, H, D] fp16 (fp16 inputs) or bf16
   float* lse;          // [B, H, N_q] fp32, may be null
@@ -102,6 +119,7 @@ struct FwdParams {
   // least drop_threshold; out_scale already holds the 1 / (1 - p)
   unsigned drop_threshold;
   unsigned seed_lo, seed_hi, drop_offset;
+  PhiloxKeys drop_keys;   // the round keys of (seed_lo, seed_hi)
   // packed variable-length batches (cu_q non-null): sequence b holds query
   // rows [cu_q[b], cu_q[b+1]) of q / out ([total_q, H, D]) and keys
   // [cu_k[b], cu_k[b+1]) of k / v ([total_k, H_kv, D]); LSE is [H, total_q];
@@ -789,16 +807,12 @@ __device__ void mma_role(SharedHeader* sh, uint8_t* tiles, uint32_t tbase, const
 // words 0 and 2 by two fixed odd constants and mixes the high and low
 // halves of the products with words 1 and 3 and the key; the key is bumped
 // by two Weyl constants between rounds.
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& key) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += 0x9E3779B9u;
-      k1 += 0xBB67AE85u;
-    }
     const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
     const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    c = make_uint4(hi1 ^ c.y ^ key.k0[r], lo1, hi0 ^ c.w ^ key.k1[r], lo0);
   }
   return c;
 }
@@ -806,8 +820,8 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 // Keep bits of 8 consecutive keys 8g .. 8g+7 of one row: bit e for key
 // 8g + e, from the 16-bit halves of the four output words (low half first).
 __device__ __forceinline__ uint32_t keep_bits8(uint32_t g, uint32_t row, uint32_t bh, uint32_t offset,
-                                               uint32_t seed_lo, uint32_t seed_hi, uint32_t t) {
-  const uint4 w = philox4x32_10(make_uint4(g, row, bh, offset), seed_lo, seed_hi);
+                                               const PhiloxKeys& key, uint32_t t) {
+  const uint4 w = philox4x32_10(make_uint4(g, row, bh, offset), key);
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};
   uint32_t bits = 0;
 #pragma unroll
@@ -1062,7 +1076,7 @@ __device__ void softmax_role(SharedHeader* sh, const uint8_t* tiles, uint32_t tb
         const uint32_t bh = static_cast<uint32_t>(w.b * p.H + w.h);
 #pragma unroll
         for (int g = 0; g < HALF_N / 8; ++g)
-          keep[g / 4] |= keep_bits8(g0 + g, static_cast<uint32_t>(row), bh, p.drop_offset, p.seed_lo, p.seed_hi,
+          keep[g / 4] |= keep_bits8(g0 + g, static_cast<uint32_t>(row), bh, p.drop_offset, p.drop_keys,
                                     p.drop_threshold)
                          << (8 * (g % 4));
       }

@@ -32,6 +32,12 @@
  * Calls are asynchronous on `stream` (NULL = the legacy default stream);
  * outputs are ready when the stream's work completes.
  *
+ * CUDA graphs: after one call on a stream (which sets kernel attributes and
+ * takes the stream's counters), calls on that stream can be captured; a
+ * captured forward keeps that stream's counters, so a graph must not be
+ * replayed while another forward runs on the stream it was captured on
+ * (fa_fwd_noalloc's one fixed array is shared by all its calls likewise).
+ *
  * Errors: every entry point returns FA_OK (0) or a negative fa_status and
  * never aborts.  Argument errors are detected before any GPU work is queued.
  * Wait timeouts inside a running kernel are recorded on the device and

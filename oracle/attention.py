@@ -29,9 +29,15 @@ Rows that see no key at all get O_i = 0 and LSE_i = -inf.
 
 Visibility (the "mask" of the pages' ``causal=True`` and ``window_size``
 arguments; Flash Attention | Hermes Skill, Workflow 2, Steps 2-3):
-    causal:               key j visible to query i only if j <= i
-    window_left = w >= 0: key j visible to query i only if j >= i - w
-    window_left = -1:     no window (the pages' ``(-1, -1)``)
+    causal:                key j visible to query i only if j <= i
+    window_left = w >= 0:  key j visible to query i only if j >= i - w
+    window_right = w >= 0: key j visible to query i only if j <= i + w
+    -1:                    no bound on that side (the pages' ``(-1, -1)``)
+The pages' sliding-window example passes ``window_size=(256, 256)``, i.e. up
+to 256 keys on each side of the query; with ``causal=True`` beside it
+the keys after the query stay hidden (causal wins, as in the flash-attn
+call the pages show), and without ``causal`` the right window admits keys up
+to ``w`` positions after the query.
 Indices are absolute (top-left aligned) also when N_q != N_k; this is the
 plainest reading, since the pages only show N_q == N_k.
 
@@ -91,13 +97,14 @@ __all__ = [
 ]
 
 
-def visibility(rows: Iterable[int], n_k: int, causal: bool, window_left: int) -> np.ndarray:
+def visibility(rows: Iterable[int], n_k: int, causal: bool, window_left: int, window_right: int = -1) -> np.ndarray:
     """Boolean [len(rows), n_k] table: True where key j is visible to query i.
 
     Follows the pages' flash_attn_func arguments (Flash Attention | Hermes
     Skill, Workflow 2, Step 2 ``causal=True`` and Step 3 ``window_size=(left,
     right)``): causal hides keys after the query, a left window of ``w`` hides
-    keys more than ``w`` positions before it, ``-1`` means unlimited.
+    keys more than ``w`` positions before it, a right window of ``w`` keys
+    more than ``w`` positions after it, ``-1`` means unlimited.
     """
     i = np.asarray(list(rows) if not isinstance(rows, np.ndarray) else rows, dtype=np.int64)[:, None]
     j = np.arange(n_k, dtype=np.int64)[None, :]
@@ -106,12 +113,14 @@ def visibility(rows: Iterable[int], n_k: int, causal: bool, window_left: int) ->
         vis &= j <= i
     if window_left >= 0:
         vis &= j >= i - window_left
+    if window_right >= 0:
+        vis &= j <= i + window_right
     return vis
 
 
 def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
                   rows=None, return_probs: bool = False, mask=None, dropout_p: float = 0.0,
-                  seed: int = 0, offset: int = 0):
+                  seed: int = 0, offset: int = 0, window_right: int = -1):
     """Exact attention forward in float64 (definition in the module docstring).
 
     q: [B, N_q, H, D]; k, v: [B, N_k, H_kv, D] with H a multiple of H_kv
@@ -140,7 +149,7 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
     group = H // h_kv
     rows = np.arange(n_q, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     R = rows.shape[0]
-    vis0 = visibility(rows, n_k, causal, window_left)
+    vis0 = visibility(rows, n_k, causal, window_left, window_right)
     if mask is not None:
         mask = np.asarray(mask)
         if mask.ndim != 4 or mask.shape[2] != n_q or mask.shape[3] != n_k or mask.shape[0] not in (1, B) \
@@ -187,7 +196,7 @@ def attention_ref(q, k, v, scale: float, causal: bool = False, window_left: int 
 
 
 def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_left: int = -1, mask=None,
-                         dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+                         dropout_p: float = 0.0, seed: int = 0, offset: int = 0, window_right: int = -1):
     """Pure-Python triple loop over (query, key, dim), for tiny shapes only.
 
     Written independently of ``attention_ref``: nested lists, ``math.exp``, no
@@ -217,6 +226,8 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
                     if causal and j > i:
                         continue
                     if window_left != -1 and i - j > window_left:
+                        continue
+                    if window_right != -1 and j - i > window_right:
                         continue
                     bias = 0.0
                     if mask is not None:
@@ -249,7 +260,7 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool = False, window_lef
 
 
 def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, window_left: int = -1,
-                           dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+                           dropout_p: float = 0.0, seed: int = 0, offset: int = 0, window_right: int = -1):
     """Gradients of the exact attention forward, in float64.
 
     The pages name the backward pass only by its method: the speed and memory
@@ -286,7 +297,7 @@ def attention_backward_ref(q, k, v, do, scale: float, causal: bool = False, wind
     n_k, h_kv = k.shape[1], k.shape[2]
     if do.shape != q.shape:
         raise ValueError("do must be shaped like q")
-    _, _, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True)
+    _, _, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True, window_right=window_right)
     rows = np.arange(n_q, dtype=np.int64)
     group = H // h_kv
     dq = np.zeros_like(q)

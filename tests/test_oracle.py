@@ -288,7 +288,7 @@ def test_planted_mistake_is_caught(mut):
 
 @pytest.mark.parametrize("bad", ["strict_causal", "window_off_by_one", "window_ignored", "causal_ignored"])
 def test_planted_mask_mistake_is_caught(monkeypatch, bad):
-    def mutated(rows, n_k, causal, window_left):
+    def mutated(rows, n_k, causal, window_left, window_right=-1):
         i = np.asarray(rows, dtype=np.int64)[:, None]
         j = np.arange(n_k)[None, :]
         vis = np.ones((i.shape[0], n_k), bool)
@@ -296,6 +296,8 @@ def test_planted_mask_mistake_is_caught(monkeypatch, bad):
             vis &= (j < i) if bad == "strict_causal" else (j <= i)
         if window_left >= 0 and bad != "window_ignored":
             vis &= (j > i - window_left) if bad == "window_off_by_one" else (j >= i - window_left)
+        if window_right >= 0:
+            vis &= j <= i + window_right
         return vis
 
     monkeypatch.setattr(oa, "visibility", mutated)

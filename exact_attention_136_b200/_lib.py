@@ -31,6 +31,8 @@ SIGNATURES = {
                             _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
     "fa_fwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                             _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
+    "fa_fwd_window": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                               _c_int, _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
     "fa_fwd_splitkv_workspace_bytes": (ctypes.c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "fa_fwd_splitkv": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                                 _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _c_int, _vp, ctypes.c_size_t,
@@ -52,6 +54,8 @@ SIGNATURES = {
                         _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
     "fa_bwd_gqa": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                             _c_int, _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
+    "fa_bwd_window": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
+                               _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
     "fa_bwd_dropout": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                                 _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, ctypes.c_ulonglong,
                                 ctypes.c_uint, _vp, ctypes.c_size_t, _vp]),

@@ -139,11 +139,14 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
             lse: Optional[torch.Tensor] = None, return_lse: bool = True,
             stream: Optional[torch.cuda.Stream] = None, num_splits: int = 1,
             attn_mask: Optional[torch.Tensor] = None, dropout_p: float = 0.0, seed: Optional[int] = None,
-            offset: int = 0) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            offset: int = 0, window_right: int = -1) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Exact attention forward; returns (out, lse).
 
     scale=None means 1/sqrt(headdim), the pages' auto scale (Workflow 2,
-    Step 2).  window_left=-1 means no window.  For float8_e4m3fn inputs all
+    Step 2).  window_left=-1 means no window.  window_right >= 0 keeps only
+    keys at most that many positions after the query (the right entry of the
+    pages' window_size, Workflow 2, Step 3; fa_fwd_window), not combined with
+    attn_mask, num_splits or dropout.  For float8_e4m3fn inputs all
     descales are 1; use forward_fp8 to pass per-tensor scales.  k and v may
     have fewer heads than q (multi-query / grouped-query attention, Workflow
     2, Step 3): query head h then reads head h // (H / H_kv).  num_splits > 1
@@ -158,6 +161,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
     backward needs the same seed and offset.
     """
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
+    _check_right_window(window_right, attn_mask, num_splits, dropout_p)
     if dropout_p:
         return _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, stream, num_splits,
                                 attn_mask, dropout_p, seed, offset)
@@ -165,7 +169,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
         num_splits = auto_splits(B, n_q, n_k, H, q.device)
     if q.dtype == torch.float8_e4m3fn:
         return forward_fp8(q, k, v, 1.0, 1.0, 1.0, scale, causal, window_left, out, lse, return_lse, stream,
-                           num_splits, attn_mask)
+                           num_splits, attn_mask, window_right)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     out, lse = _outputs(q, B, n_q, H, D, out, lse, return_lse)
     with torch.cuda.device(q.device):
@@ -181,6 +185,12 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
             _splitkv(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _DT[q.dtype],
                      (1.0, 1.0, 1.0), num_splits, s)
             return out, lse
+        if window_right != -1:
+            rc = _lib.lib().fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_p, B, n_q,
+                                          n_k, H, h_kv, D, scale, int(bool(causal)), int(window_left),
+                                          int(window_right), _DT[q.dtype], 1.0, 1.0, 1.0, s.cuda_stream)
+            _lib.check(rc, "fa_fwd_window")
+            return out, lse
         if h_kv == H:
             rc = _lib.lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_p, B, n_q, n_k, H,
                                    D, scale, int(bool(causal)), int(window_left), _DT[q.dtype], s.cuda_stream)
@@ -190,6 +200,16 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
                                        1.0, 1.0, 1.0, s.cuda_stream)
     _lib.check(rc, "fa_fwd" if h_kv == H else "fa_fwd_gqa")
     return out, lse
+
+
+def _check_right_window(window_right, attn_mask=None, num_splits=1, dropout_p=0.0):
+    if window_right == -1:
+        return
+    if window_right < -1:
+        raise ValueError("window_right must be -1 (no bound) or >= 0")
+    if attn_mask is not None or num_splits not in (0, 1) or dropout_p:
+        raise ValueError("window_right is not combined with attn_mask, num_splits or dropout "
+                         "(a boolean attn_mask expresses any window)")
 
 
 def _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, stream, num_splits, attn_mask,
@@ -257,9 +277,10 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
                 v_descale: float, scale: Optional[float] = None, causal: bool = False,
                 window_left: int = -1, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                 return_lse: bool = True, stream: Optional[torch.cuda.Stream] = None, num_splits: int = 1,
-                attn_mask: Optional[torch.Tensor] = None):
+                attn_mask: Optional[torch.Tensor] = None, window_right: int = -1):
     """FP8 e4m3 forward with per-tensor descales; out is bfloat16."""
     B, n_q, n_k, H, h_kv, D = _check_inputs(q8, k8, v8)
+    _check_right_window(window_right, attn_mask, num_splits)
     if num_splits == 0:
         num_splits = auto_splits(B, n_q, n_k, H, q8.device)
     if q8.dtype != torch.float8_e4m3fn:
@@ -279,6 +300,13 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
             _splitkv(q8, k8, v8, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, _lib.FA_E4M3,
                      (q_descale, k_descale, v_descale), num_splits, s)
             return out, lse
+        if window_right != -1:
+            rc = _lib.lib().fa_fwd_window(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(), lse_p, B, n_q,
+                                          n_k, H, h_kv, D, scale, int(bool(causal)), int(window_left),
+                                          int(window_right), _lib.FA_E4M3, float(q_descale), float(k_descale),
+                                          float(v_descale), s.cuda_stream)
+            _lib.check(rc, "fa_fwd_window")
+            return out, lse
         if h_kv == H:
             rc = _lib.lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(), lse_p, B, n_q,
                                        n_k, H, D, scale, int(bool(causal)), int(window_left), float(q_descale),
@@ -294,10 +322,10 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
 def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
              dout: torch.Tensor, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,
              stream: Optional[torch.cuda.Stream] = None, dropout_p: float = 0.0, seed: Optional[int] = None,
-             offset: int = 0) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Gradients (dq, dk, dv) of forward(q, k, v, scale, causal, window_left)
-    for the upstream gradient dout, from the forward's out and lse (fp16 /
-    bf16).  k and v may have fewer heads than q (grouped-query attention):
+             offset: int = 0, window_right: int = -1) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients (dq, dk, dv) of forward(q, k, v, scale, causal, window_left,
+    window_right=...) for the upstream gradient dout, from the forward's out
+    and lse (fp16 / bf16).  k and v may have fewer heads than q (grouped-query attention):
     dk and dv of a K/V head then sum over the query heads that read it.
     dropout_p, seed, offset: those of a dropout forward (fa_bwd_dropout redraws
     its keep bits).  The fp32 workspace the library needs is taken from
@@ -305,6 +333,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
     if q.dtype not in (torch.float16, torch.bfloat16):
         raise ValueError("backward takes fp16 or bf16 inputs")
+    _check_right_window(window_right, dropout_p=dropout_p)
     for name, t in (("out", out), ("dout", dout)):
         if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous tensor like q")
@@ -325,6 +354,11 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
                                            h_kv, D, scale, int(bool(causal)), int(window_left), _DT[q.dtype],
                                            float(dropout_p), int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF,
                                            ws.data_ptr(), nbytes, s.cuda_stream)
+        elif window_right != -1:
+            rc = _lib.lib().fa_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H,
+                                          h_kv, D, scale, int(bool(causal)), int(window_left), int(window_right),
+                                          _DT[q.dtype], ws.data_ptr(), nbytes, s.cuda_stream)
         elif h_kv == H:
             rc = _lib.lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
                                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, n_q, n_k, H, D,
@@ -340,7 +374,8 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
         if s != torch.cuda.current_stream(q.device):
             for t in (dq, dk, dv):
                 t.record_stream(s)
-    _lib.check(rc, "fa_bwd_dropout" if dropout_p else ("fa_bwd" if h_kv == H else "fa_bwd_gqa"))
+    _lib.check(rc, "fa_bwd_dropout" if dropout_p else "fa_bwd_window" if window_right != -1
+               else ("fa_bwd" if h_kv == H else "fa_bwd_gqa"))
     return dq, dk, dv
 
 

@@ -183,6 +183,17 @@ int validate(const void* q, const void* k, const void* v, void* out, int B, int 
   return FA_OK;
 }
 
+// The keys' upper bound j <= i + R the kernels apply (R = -1: none).  causal
+// is R = 0 (a right window beside it cannot widen it); a right window that
+// reaches past the last key bounds nothing.  With a bound, i + R stays in int
+// range: N_q + N_k below 2^31 - 256 (else FA_ERR_ARG).
+int right_bound(int causal, int window_right, int Nq, int Nk, int* R) {
+  if (window_right < -1) return FA_ERR_ARG;
+  *R = causal ? 0 : (window_right >= Nk ? -1 : window_right);
+  if (*R > 0 && static_cast<int64_t>(Nq) + Nk >= (int64_t(1) << 31) - 256) return FA_ERR_ARG;
+  return FA_OK;
+}
+
 // Workspace of a split forward: fp32 O of every slice [splits, B, N_q, H, D]
 // followed by its LSE [splits, B, H, N_q].
 size_t splitkv_workspace_bytes(int B, int Nq, int H, int D, int splits) {
@@ -195,11 +206,14 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
             void* workspace = nullptr, size_t workspace_bytes = 0, const void* mask = nullptr,
             int mask_type = 0, long long mask_sb = 0, long long mask_sh = 0, long long mask_sq = 0,
             float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0, const int* cu_q = nullptr,
-            const int* cu_k = nullptr, int total_q = 0, int total_k = 0) {
+            const int* cu_k = nullptr, int total_q = 0, int total_k = 0, int window_right = -1) {
   // (packed batches are validated by fa_fwd_varlen, with N_q and N_k the
   // longest sequences; here only their totals address the tensors)
   int rc = cu_q ? validate(q, k, v, out, 1, total_q, total_k, H, D, scale, causal, window_left, dtype, Hkv)
                 : validate(q, k, v, out, B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
+  if (rc != FA_OK) return rc;
+  int R = -1;
+  rc = right_bound(causal, window_right, Nq, Nk, &R);
   if (rc != FA_OK) return rc;
   if (splits < 1) return FA_ERR_ARG;
   // dropout: 0 <= p < 1, 16-bit inputs, not combined with a mask or a split key range
@@ -256,6 +270,7 @@ int forward(const void* q, const void* k, const void* v, void* out, float* lse, 
   p.qpk = H / Hkv;
   p.causal = causal;
   p.window_left = window_left;
+  p.window_right = R;
   p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
                                      static_cast<double>(qd) * static_cast<double>(kd));
   p.out_scale = vd;
@@ -391,6 +406,14 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* ls
                      k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int fa_fwd_window(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q, int N_k,
+                  int H, int H_kv, int D, float scale, int causal, int window_left, int window_right, int dtype,
+                  float q_descale, float k_descale, float v_descale, fa_stream_t stream) {
+  return fa::forward(q, k, v, out, lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype, q_descale,
+                     k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream), nullptr, 1, nullptr, 0, nullptr, 0,
+                     0, 0, 0, 0.f, 0, 0, nullptr, nullptr, 0, 0, window_right);
+}
+
 size_t fa_fwd_splitkv_workspace_bytes(int B, int N_q, int N_k, int H, int D, int num_splits) {
   if (B < 1 || N_q < 0 || N_k < 0 || H < 1 || D < 1 || num_splits < 1) return 0;
   // the slices the forward will actually use
@@ -513,6 +536,15 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* out, con
                fa_stream_t stream) {
   return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, H_kv, D, scale, causal, window_left,
                       dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_window(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int H_kv, int D, float scale,
+                  int causal, int window_left, int window_right, int dtype, void* workspace, size_t workspace_bytes,
+                  fa_stream_t stream) {
+  return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, N_q, N_k, H, H_kv, D, scale, causal, window_left,
+                      dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), 0.f, 0, 0,
+                      window_right);
 }
 
 int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out, const void* dout,

@@ -49,8 +49,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dout, co
 int backward(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
              void* dq, void* dk, void* dv, int B, int Nq, int Nk, int H, int Hkv, int D, float scale, int causal,
              int window_left, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-             float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0) {
+             float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0, int window_right = -1) {
   int rc = validate(q, k, v, const_cast<void*>(out), B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
+  if (rc != FA_OK) return rc;
+  int R = -1;
+  rc = right_bound(causal, window_right, Nq, Nk, &R);
   if (rc != FA_OK) return rc;
   if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
   if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_ARG;
@@ -102,6 +105,7 @@ int backward(const void* q, const void* k, const void* v, const void* out, const
     p.qpk = H / Hkv;
     p.causal = causal;
     p.window_left = window_left;
+    p.window_right = R;
     p.scale = scale;
     p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.nkb = (Nk + 127) / 128;

@@ -85,7 +85,10 @@ struct BwdParams {
   const float* delta;       // [B, H, N_q] rowsum(dO * O)
   int B, Nq, Nk, H;
   int Hkv, qpk;             // key/value heads; query head h reads K/V head h / qpk
-  int causal, window_left;  // window_left -1 = unlimited
+  int causal;               // scheduling order only; the key bounds carry the mask
+  int window_left;          // keys at most this many before the query; -1 = unlimited
+  int window_right;         // keys at most this many after it; -1 = unlimited, 0 under
+                            // causal (set by the host, below N_k + N_q < 2^31)
   float scale;              // softmax scale
   float score_scale;        // scale * log2(e)
   int nkb;                  // key blocks per (batch, head)
@@ -169,12 +172,12 @@ __device__ __forceinline__ bool grad_bar_and(bool v) {
   return r != 0u;
 }
 
-// Query blocks that see key block jk: causal keeps queries at or after the
-// key (absolute indices), a left window keeps queries at most window_left
-// after it.
+// Query blocks that see key block jk: a right window (causal: 0) keeps
+// queries at least window_right before the key (absolute indices), a left
+// window keeps queries at most window_left after it.
 __device__ __forceinline__ void bwd_query_range(int jk, const BwdParams& p, int& i_lo, int& i_hi) {
   const int nqb = (p.Nq + 127) / 128;
-  i_lo = p.causal ? jk : 0;
+  i_lo = p.window_right >= 0 ? max(0, jk * 128 - p.window_right) / 128 : 0;
   i_hi = nqb - 1;
   if (p.window_left >= 0) {
     const long long last = static_cast<long long>(jk) * 128 + 127 + p.window_left;
@@ -445,7 +448,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (++ib == cnt) { ib = 0; ++qn; }
       const int buf = n & 1;
       const int q0 = i * 128;
-      const bool need_mask = (jk * 128 + 128 > p.Nk) || (p.causal && jk * 128 + 127 > q0) ||
+      const bool need_mask = (jk * 128 + 128 > p.Nk) || (p.window_right >= 0 && jk * 128 + 127 > q0 + p.window_right) ||
                              (p.window_left >= 0 && jk * 128 < q0 + 127 - p.window_left);
       // dropout keep bits of this thread's key for its 64 queries (bit e:
       // query q0 + 64 * half + e).  The generator gives 8 keys of one query
@@ -493,7 +496,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const int q = q0 + half * 64 + e;
-          const bool vis = key < p.Nk && (!p.causal || key <= q) && (p.window_left < 0 || key >= q - p.window_left);
+          const bool vis = key < p.Nk && (p.window_right < 0 || key <= q + p.window_right) &&
+                           (p.window_left < 0 || key >= q - p.window_left);
           pv[e] = vis ? pv[e] : -INFINITY;
         }
       }
@@ -702,7 +706,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   // key blocks the rows of this query block see (as in the forward)
   const int qe = min(q0 + 127, p.Nq - 1);
   const int j_lo = p.window_left >= 0 ? max(0, q0 - p.window_left) / 128 : 0;
-  const int j_hi = p.causal ? min(qe, p.Nk - 1) / 128 : p.nkb - 1;
+  const int j_hi = p.window_right >= 0 ? min(qe + p.window_right, p.Nk - 1) / 128 : p.nkb - 1;
   const int cnt = (q0 < p.Nq && p.Nk > 0) ? max(0, j_hi - j_lo + 1) : 0;
   const uint64_t lim = p.wait_limit_ns;
 
@@ -872,7 +876,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (__any_sync(0xffffffffu, bwd_aborted(&sh->abort_flag))) { ok = false; break; }
       const int k0 = (j_lo + n) * 128;
       const uint32_t s_col = (n & 1) ? Q::S_COL1 : Q::S_COL0;
-      const bool need_mask = (k0 + 128 > p.Nk) || (p.causal && k0 + 127 > q0) ||
+      const bool need_mask = (k0 + 128 > p.Nk) || (p.window_right >= 0 && k0 + 127 > q0 + p.window_right) ||
                              (p.window_left >= 0 && k0 < q0 + 127 - p.window_left);
       // dropout keep bits of this row's keys k0 + 64 * half + [0, 64)
       uint32_t keep[2] = {0u, 0u};
@@ -905,7 +909,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const int key = k0 + half * 64 + e;
-          const bool vis = key < p.Nk && (!p.causal || key <= q) && (p.window_left < 0 || key >= q - p.window_left);
+          const bool vis = key < p.Nk && (p.window_right < 0 || key <= q + p.window_right) &&
+                           (p.window_left < 0 || key >= q - p.window_left);
           pv[e] = vis ? pv[e] : -INFINITY;
         }
       }

@@ -86,8 +86,10 @@ struct FwdParams {
   int B, Nq, Nk, H;
   int Hkv;             // key/value heads (H a multiple of Hkv)
   int qpk;             // H / Hkv: query head h reads K/V head h / qpk
-  int causal;
-  int window_left;     // -1 = unlimited
+  int causal;          // scheduling order only; the key bounds below carry the mask
+  int window_left;     // keys at most this many before the query; -1 = unlimited
+  int window_right;    // keys at most this many after the query; -1 = unlimited,
+                       // 0 under causal (set by the host, below N_k + N_q < 2^31)
   float score_scale;   // scale * log2(e) * q_descale * k_descale
   float out_scale;     // v_descale (1 for 16-bit inputs)
   int num_units;
@@ -271,7 +273,7 @@ __device__ __forceinline__ Tile get_tile(int u, int split, int t, const FwdParam
   w.rows = w.qs < w.nq;
   const int qe = min(w.qs + BLOCK_M - 1, w.nq - 1);
   w.lo = p.window_left >= 0 ? max(0, w.qs - p.window_left) / BLOCK_N : 0;
-  w.hi = p.causal ? min(qe, w.nk - 1) / BLOCK_N : (w.nk - 1) / BLOCK_N;
+  w.hi = p.window_right >= 0 ? min(qe + p.window_right, w.nk - 1) / BLOCK_N : (w.nk - 1) / BLOCK_N;
   if (SPLIT) {
     w.lo = max(w.lo, w.split * p.split_blocks);
     w.hi = min(w.hi, (w.split + 1) * p.split_blocks - 1);
@@ -1063,10 +1065,11 @@ __device__ void softmax_role(SharedHeader* sh, const uint8_t* tiles, uint32_t tb
     constexpr bool ATTN_MASK = C::TMA_MASK;
     constexpr bool DROP = MASK == MASK_DROPOUT;
     for (int j = w.lo; j <= w.hi; ++j) {
-      // boundary blocks (causal diagonal, window edge, key tail), decided
-      // before S arrives
+      // boundary blocks (causal diagonal or right window edge, left window
+      // edge, key tail), decided before S arrives
       const int k0 = j * BLOCK_N;
-      const bool need_mask = (k0 + BLOCK_N > w.nk) || (p.causal && k0 + BLOCK_N - 1 > w.qs) ||
+      const bool need_mask = (k0 + BLOCK_N > w.nk) ||
+                             (p.window_right >= 0 && k0 + BLOCK_N - 1 > w.qs + p.window_right) ||
                              (p.window_left >= 0 && k0 < w.qs + BLOCK_M - 1 - p.window_left);
       // dropout keep bits of this thread's keys (bit c: key k0 + 64 * half + c),
       // generated while S is computed
@@ -1136,7 +1139,7 @@ __device__ void softmax_role(SharedHeader* sh, const uint8_t* tiles, uint32_t tb
       }
       if (need_mask) {
         const int kh = k0 + half * HALF_N;
-        const int hi_c = min(w.nk - kh, p.causal ? row - kh + 1 : HALF_N);
+        const int hi_c = min(w.nk - kh, p.window_right >= 0 ? row + p.window_right - kh + 1 : HALF_N);
         const int lo_c = p.window_left >= 0 ? row - p.window_left - kh : 0;
 #pragma unroll
         for (int c = 0; c < HALF_N; ++c)

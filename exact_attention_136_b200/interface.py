@@ -10,11 +10,12 @@ computation is libfa_b200.so's), so code written against the pages' call can
 switch to this library and train through it.
 
 Readings (the pages leave these open):
-- ``window_size=(left, right)``: ``left`` is the window before the query
-  (-1 = unlimited); with ``causal=True`` the right window is zero whatever
+- ``window_size=(left, right)``: key j is visible to query i only if
+  i - left <= j <= i + right, -1 meaning no bound on that side
+  (fa_fwd_window).  With ``causal=True`` the right window is zero whatever
   ``right`` says (the page pairs causal=True with a two-sided window, which
-  contradict each other; causal wins).  Without causal only ``right = -1``
-  (no right bound) is available.
+  contradict each other; causal wins).  A right window without causal is
+  not combined with dropout.
 - ``dropout_p``: the usual attention dropout, each softmax probability kept
   with probability 1 - p and scaled by 1 / (1 - p) (fa_fwd_dropout).  The
   pages name no random generator; each call draws a 64-bit seed from
@@ -32,26 +33,29 @@ import torch
 from .api import backward, forward
 
 
-def _window_left(causal: bool, window_size: Tuple[int, int]) -> int:
+def _window(causal: bool, window_size: Tuple[int, int], dropout_p: float) -> Tuple[int, int]:
+    """(left, right) as forward / backward take them; right -1 under causal."""
     left, right = (int(window_size[0]), int(window_size[1]))
     if left < -1 or right < -1:
         raise ValueError("window_size entries are -1 (unlimited) or >= 0")
-    if not causal and right != -1:
-        raise NotImplementedError("a right window without causal=True is not supported (only left windows)")
-    return left
+    if causal:
+        return left, -1
+    if right != -1 and dropout_p:
+        raise NotImplementedError("a right window without causal=True is not combined with dropout")
+    return left, right
 
 
 class _FlashAttn(torch.autograd.Function):
     """O = attention(q, k, v); the backward recomputes from O and the LSE."""
 
     @staticmethod
-    def forward(ctx, q, k, v, scale, causal, window_left, dropout_p, seed):
+    def forward(ctx, q, k, v, scale, causal, window_left, window_right, dropout_p, seed):
         if dropout_p:
             out, lse = forward(q, k, v, scale, causal, window_left, dropout_p=dropout_p, seed=seed)
         else:
-            out, lse = forward(q, k, v, scale, causal, window_left)
+            out, lse = forward(q, k, v, scale, causal, window_left, window_right=window_right)
         ctx.save_for_backward(q, k, v, out, lse)
-        ctx.scale, ctx.causal, ctx.window_left = scale, causal, window_left
+        ctx.scale, ctx.causal, ctx.window_left, ctx.window_right = scale, causal, window_left, window_right
         ctx.dropout_p, ctx.seed = dropout_p, seed
         ctx.mark_non_differentiable(lse)
         return out, lse
@@ -65,8 +69,9 @@ class _FlashAttn(torch.autograd.Function):
             dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left,
                                   dropout_p=ctx.dropout_p, seed=ctx.seed)
         else:
-            dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left)
-        return dq, dk, dv, None, None, None, None, None
+            dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left,
+                                  window_right=ctx.window_right)
+        return dq, dk, dv, None, None, None, None, None, None
 
 
 def flash_attn_func(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dropout_p: float = 0.0,
@@ -82,14 +87,14 @@ def flash_attn_func(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dropout_p
     dropout_p = float(dropout_p)
     if not (0.0 <= dropout_p < 1.0):
         raise ValueError("dropout_p must be in [0, 1)")
-    wl = _window_left(bool(causal), window_size)
+    wl, wr = _window(bool(causal), window_size, dropout_p)
     scale = float(softmax_scale) if softmax_scale is not None else q.shape[-1] ** -0.5
     seed = int(torch.randint(0, 2 ** 62, (1,)).item()) if dropout_p > 0.0 else 0
     needs_grad = torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v))
     if needs_grad:
-        out, lse = _FlashAttn.apply(q, k, v, scale, bool(causal), wl, dropout_p, seed)
+        out, lse = _FlashAttn.apply(q, k, v, scale, bool(causal), wl, wr, dropout_p, seed)
     elif dropout_p > 0.0:
         out, lse = forward(q, k, v, scale, bool(causal), wl, dropout_p=dropout_p, seed=seed)
     else:
-        out, lse = forward(q, k, v, scale, bool(causal), wl)
+        out, lse = forward(q, k, v, scale, bool(causal), wl, window_right=wr)
     return (out, lse) if return_lse else out

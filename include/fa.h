@@ -14,7 +14,9 @@
  * "Technical insight").  Visibility follows the flash_attn_func arguments
  * shown on the pages (Workflow 2, Steps 2-3): with `causal`, key j is visible
  * to query i only if j <= i; with window_left = w >= 0, only if j >= i - w;
- * window_left = -1 means no window (the pages' window_size=(-1,-1)).  Query
+ * window_left = -1 means no window (the pages' window_size=(-1,-1)); the
+ * right entry of window_size, taken by fa_fwd_window / fa_bwd_window, keeps
+ * only j <= i + window_right (local attention on both sides).  Query
  * and key indices are absolute (top-left aligned) also when N_q != N_k.  A
  * row that sees no key gets O = 0 and LSE = -inf.
  *
@@ -109,6 +111,22 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* ls
                int B, int N_q, int N_k, int H, int H_kv, int D, float scale, int causal,
                int window_left, int dtype, float q_descale, float k_descale, float v_descale,
                fa_stream_t stream);
+
+/*
+ * fa_fwd_window -- fa_fwd_gqa with both entries of the pages' window_size
+ * (Flash Attention | Hermes Skill, Workflow 2, Step 3: the sliding-window
+ * example passes (256, 256), keys on both sides of the query).  Key j is
+ * visible to query i only if i - window_left <= j <= i + window_right, -1
+ * meaning no bound on that side; causal = 1 still hides every j > i, so a
+ * right window beside it changes nothing.  window_right = 0 is causal,
+ * window_right >= N_k no right bound.  Every other argument and the return
+ * values as fa_fwd_gqa; FA_ERR_ARG also for window_right < -1, or for a right
+ * bound with N_q + N_k >= 2^31 - 256.
+ */
+int fa_fwd_window(const void* q, const void* k, const void* v, void* out, float* lse,
+                  int B, int N_q, int N_k, int H, int H_kv, int D, float scale, int causal,
+                  int window_left, int window_right, int dtype, float q_descale, float k_descale,
+                  float v_descale, fa_stream_t stream);
 
 /*
  * fa_fwd_splitkv -- the forward of fa_fwd_gqa with the key range split into
@@ -297,6 +315,16 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* out, con
                const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H,
                int H_kv, int D, float scale, int causal, int window_left, int dtype,
                void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fa_bwd_window -- fa_bwd_gqa for the forward of fa_fwd_window: the same
+ * causal, window_left and window_right.  Workspace, ownership, kernels and
+ * return values as fa_bwd_gqa; FA_ERR_ARG also as fa_fwd_window.
+ */
+int fa_bwd_window(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H,
+                  int H_kv, int D, float scale, int causal, int window_left, int window_right,
+                  int dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fa_bwd_dropout -- fa_bwd_gqa for the forward of fa_fwd_dropout: the same

@@ -17,7 +17,7 @@ def _f64(t: torch.Tensor, descale: float) -> np.ndarray:
     return (t.to(torch.float64) * descale).numpy()
 
 
-def oracle(qkv, scale, causal, window_left, rows=None, mask=None):
+def oracle(qkv, scale, causal, window_left, rows=None, mask=None, window_right=-1):
     """(O [B, R, H, D], LSE [B, H, R]) in float64 for the given QKV bundle (mask: numpy,
     [B or 1, H or 1, N_q, N_k], bool or real)."""
     B, n_q, H, D = qkv.q.shape
@@ -31,7 +31,7 @@ def oracle(qkv, scale, causal, window_left, rows=None, mask=None):
             mb = None if mask is None else mask[b:b + 1] if mask.shape[0] > 1 else mask
             o, l = attention_ref(_f64(qkv.q[b:b + 1], qkv.q_descale), _f64(qkv.k[b:b + 1], qkv.k_descale),
                                  _f64(qkv.v[b:b + 1], qkv.v_descale), scale, causal, window_left, rows=rows,
-                                 mask=mb)
+                                 mask=mb, window_right=window_right)
             O[b], L[b] = o[0], l[0]
         return O, L
     O = np.zeros((B, R, H, D))
@@ -41,7 +41,7 @@ def oracle(qkv, scale, causal, window_left, rows=None, mask=None):
             q = _f64(qkv.q[b:b + 1, :, h:h + 1], qkv.q_descale)
             k = _f64(qkv.k[b:b + 1, :, h:h + 1], qkv.k_descale)
             v = _f64(qkv.v[b:b + 1, :, h:h + 1], qkv.v_descale)
-            o, l = attention_ref(q, k, v, scale, causal, window_left, rows=rows)
+            o, l = attention_ref(q, k, v, scale, causal, window_left, rows=rows, window_right=window_right)
             O[b, :, h] = o[0, :, 0]
             L[b, h] = l[0, 0]
     return O, L
@@ -66,7 +66,7 @@ def compare(out, lse, ref_o, ref_l, rows=None):
 
 
 def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, unit_roundoff, dropout_p=0.0,
-                    seed=0, offset=0):
+                    seed=0, offset=0, window_right=-1):
     """Per-element bounds (dq, dk, dv; shaped like q, k, v) on how far a
     backward computed the way the CUDA path does can be from the exact
     gradients, all arrays float64 numpy.
@@ -95,7 +95,7 @@ def backward_bounds(q, k, v, do, o_used, lse_used, scale, causal, window_left, u
     group = H // h_kv
     bq, bk, bv = np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)
     o_ref, l_ref, probs = attention_ref(q, k, v, scale, causal, window_left, return_probs=True, dropout_p=dropout_p,
-                                        seed=seed, offset=offset)
+                                        seed=seed, offset=offset, window_right=window_right)
     for b in range(B):
         for h in range(H):
             hk = h // group

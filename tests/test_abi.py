@@ -287,3 +287,22 @@ def test_varlen_arguments_validated(kw, expect):
     assert f(a["q"], a["k"], a["v"], a["out"], a["lse"], a["cu_q"], a["cu_k"], a["B"], a["max_q"], a["max_k"],
              a["total_q"], a["total_k"], a["H"], a["H_kv"], a["D"], a["scale"], a["causal"], a["wl"], a["dt"], 1.0,
              1.0, 1.0, None) == expect
+
+
+@pytest.mark.parametrize("kw, expect", [
+    (dict(wr=-2), _lib.FA_ERR_ARG),
+    (dict(wr=-7, causal=1), _lib.FA_ERR_ARG),
+    (dict(wl=-2, wr=3), _lib.FA_ERR_ARG),
+    (dict(wr=5, D=96), _lib.FA_ERR_UNSUPPORTED),
+    (dict(nq=1 << 30, nk=1 << 30, wr=4), _lib.FA_ERR_ARG),   # i + window_right would leave int range
+])
+def test_window_arguments_validated(kw, expect):
+    """fa_fwd_window / fa_bwd_window check the right window on the host, before any GPU work."""
+    a = dict(nq=128, nk=128, H=1, H_kv=1, D=64, causal=0, wl=-1, wr=0)
+    a.update(kw)
+    f = _lib.lib().fa_fwd_window
+    assert f(A, A, A, A, None, 1, a["nq"], a["nk"], a["H"], a["H_kv"], a["D"], 0.125, a["causal"], a["wl"], a["wr"],
+             _lib.FA_FP16, 1.0, 1.0, 1.0, None) == expect
+    g = _lib.lib().fa_bwd_window
+    assert g(A, A, A, A, A, A, A, A, A, 1, a["nq"], a["nk"], a["H"], a["H_kv"], a["D"], 0.125, a["causal"], a["wl"],
+             a["wr"], _lib.FA_FP16, A, 1 << 40, None) == expect

@@ -16,16 +16,19 @@ from oracle import attention_backward_ref, attention_ref
 def oracle_backend(monkeypatch):
     calls = []
 
-    def fwd(q, k, v, scale, causal, window_left, dropout_p=0.0, seed=None, offset=0):
-        calls.append(("fwd", scale, causal, window_left) + ((dropout_p, seed, offset) if dropout_p else ()))
+    def fwd(q, k, v, scale, causal, window_left, dropout_p=0.0, seed=None, offset=0, window_right=-1):
+        calls.append(("fwd", scale, causal, window_left) + ((dropout_p, seed, offset) if dropout_p else ())
+                     + ((window_right,) if window_right != -1 else ()))
         o, l = attention_ref(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), scale, causal, window_left,
-                             dropout_p=dropout_p, seed=seed or 0, offset=offset)
+                             dropout_p=dropout_p, seed=seed or 0, offset=offset, window_right=window_right)
         return torch.from_numpy(o), torch.from_numpy(l)
 
-    def bwd(q, k, v, out, lse, dout, scale, causal, window_left, dropout_p=0.0, seed=None, offset=0):
-        calls.append(("bwd", scale, causal, window_left) + ((dropout_p, seed, offset) if dropout_p else ()))
+    def bwd(q, k, v, out, lse, dout, scale, causal, window_left, dropout_p=0.0, seed=None, offset=0, window_right=-1):
+        calls.append(("bwd", scale, causal, window_left) + ((dropout_p, seed, offset) if dropout_p else ())
+                     + ((window_right,) if window_right != -1 else ()))
         g = attention_backward_ref(q.detach().numpy(), k.detach().numpy(), v.detach().numpy(), dout.numpy(), scale,
-                                   causal, window_left, dropout_p=dropout_p, seed=seed or 0, offset=offset)
+                                   causal, window_left, dropout_p=dropout_p, seed=seed or 0, offset=offset,
+                                   window_right=window_right)
         return tuple(torch.from_numpy(x) for x in g)
 
     monkeypatch.setattr(itf, "forward", fwd)
@@ -33,7 +36,7 @@ def oracle_backend(monkeypatch):
     return calls
 
 
-def _plain_attention(q, k, v, scale, causal, wl):
+def _plain_attention(q, k, v, scale, causal, wl, wr=-1):
     """Softmax attention with torch ops, [B, N, H, D] (torch autograd differentiates it)."""
     s = torch.einsum("bihd,bjhd->bhij", q, k) * scale
     n_q, n_k = q.shape[1], k.shape[1]
@@ -44,26 +47,30 @@ def _plain_attention(q, k, v, scale, causal, wl):
         vis &= j <= i
     if wl >= 0:
         vis &= j >= i - wl
+    if wr >= 0:
+        vis &= j <= i + wr
     s = s.masked_fill(~vis, float("-inf"))
     return torch.einsum("bhij,bjhd->bihd", torch.softmax(s, dim=-1), v)
 
 
-@pytest.mark.parametrize("causal, window", [(False, (-1, -1)), (True, (-1, -1)), (True, (3, 3)), (False, (2, -1))])
+@pytest.mark.parametrize("causal, window", [(False, (-1, -1)), (True, (-1, -1)), (True, (3, 3)), (False, (2, -1)),
+                                           (False, (2, 3)), (False, (-1, 1))])
 def test_gradients_match_torch_autograd(oracle_backend, causal, window):
     g = torch.Generator().manual_seed(7)
     q, k, v = (torch.randn(1, 9, 2, 4, generator=g, dtype=torch.float64, requires_grad=True) for _ in range(3))
     do = torch.randn(1, 9, 2, 4, generator=g, dtype=torch.float64)
     out = itf.flash_attn_func(q, k, v, causal=causal, window_size=window)
     out.backward(do)
-    wl = window[0]
+    wl, wr = window[0], (-1 if causal else window[1])
     q2, k2, v2 = (t.detach().clone().requires_grad_() for t in (q, k, v))
-    ref = _plain_attention(q2, k2, v2, 0.5, causal, wl)   # default scale 1/sqrt(4)
+    ref = _plain_attention(q2, k2, v2, 0.5, causal, wl, wr)   # default scale 1/sqrt(4)
     ref.backward(do)
     assert torch.allclose(out, ref, atol=1e-12)
     for a, b in ((q.grad, q2.grad), (k.grad, k2.grad), (v.grad, v2.grad)):
         assert torch.allclose(a, b, atol=1e-12)
     # scale, causal and window reach the library unchanged, forward then backward
-    assert oracle_backend == [("fwd", 0.5, causal, wl), ("bwd", 0.5, causal, wl)]
+    extra = (wr,) if wr != -1 else ()
+    assert oracle_backend == [("fwd", 0.5, causal, wl) + extra, ("bwd", 0.5, causal, wl) + extra]
 
 
 def test_no_grad_path_and_lse(oracle_backend):
@@ -80,7 +87,7 @@ def test_rejected_arguments(oracle_backend):
         with pytest.raises(ValueError):
             itf.flash_attn_func(q, q, q, dropout_p=bad_p)
     with pytest.raises(NotImplementedError):
-        itf.flash_attn_func(q, q, q, causal=False, window_size=(2, 2))
+        itf.flash_attn_func(q, q, q, causal=False, window_size=(2, 2), dropout_p=0.1)
     with pytest.raises(ValueError):
         itf.flash_attn_func(q, q, q, window_size=(-2, -1))
     assert oracle_backend == []

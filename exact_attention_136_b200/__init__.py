@@ -9,10 +9,9 @@ The computation runs in libfa_b200.so (hand-written sm_100a CUDA, C ABI in
 include/fa.h); this package only marshals arguments.
 """
 
-from .api import (auto_splits, backward, device_status, forward, forward_fp8, forward_host, forward_varlen,
-                  set_wait_limit_ns,
-                  wait_probe)
+from .api import (auto_splits, backward, backward_varlen, device_status, forward, forward_fp8, forward_host,
+                  forward_varlen, set_wait_limit_ns, wait_probe)
 from .interface import flash_attn_func
 
-__all__ = ["forward", "forward_fp8", "forward_host", "forward_varlen", "backward", "flash_attn_func", "auto_splits", "device_status",
-           "set_wait_limit_ns", "wait_probe"]
+__all__ = ["forward", "forward_fp8", "forward_host", "forward_varlen", "backward", "backward_varlen",
+           "flash_attn_func", "auto_splits", "device_status", "set_wait_limit_ns", "wait_probe"]

@@ -56,6 +56,9 @@ SIGNATURES = {
                             _c_int, _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
     "fa_bwd_window": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                                _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t, _vp]),
+    "fa_bwd_varlen": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
+                               _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _vp, ctypes.c_size_t,
+                               _vp]),
     "fa_bwd_dropout": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                                 _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, ctypes.c_ulonglong,
                                 ctypes.c_uint, _vp, ctypes.c_size_t, _vp]),

@@ -273,6 +273,52 @@ def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
     return out, lse
 
 
+def backward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+                    dout: torch.Tensor, cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_q: int,
+                    max_seqlen_k: int, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,
+                    stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients (dq [total_q, H, D], dk, dv [total_k, H_kv, D]) of forward_varlen over the same packed
+    batch (fa_bwd_varlen), from its out and lse [H, total_q] (fp16 / bf16).  max_seqlen_q / max_seqlen_k
+    must bound every sequence's length."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor [total, heads, headdim]")
+    if q.dtype not in (torch.float16, torch.bfloat16) or not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("backward_varlen takes fp16 or bf16 q, k, v of one dtype")
+    for name, t in (("out", out), ("dout", dout)):
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError(f"{name} must be a tensor like q")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if not t.is_cuda or t.dtype != torch.int32 or t.dim() != 1 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 >= 2 entries")
+    total_q, H, D = q.shape
+    total_k, h_kv = k.shape[0], k.shape[1]
+    if v.shape != k.shape or k.shape[2] != D or h_kv < 1 or H % h_kv != 0:
+        raise ValueError("k and v must be [total_k, H_kv, D] with H a multiple of H_kv")
+    if lse.shape != (H, total_q) or lse.dtype != torch.float32 or lse.device != q.device or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [H, total_q] tensor on q's device")
+    B = cu_seqlens_q.numel() - 1
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    with torch.cuda.device(q.device):
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        nbytes = int(_lib.lib().fa_bwd_workspace_bytes(1, total_q, H, D))
+        with torch.cuda.stream(s):
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+        rc = _lib.lib().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                      cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+                                      int(max_seqlen_k), total_q, total_k, H, h_kv, D, scale, int(bool(causal)),
+                                      int(window_left), _DT[q.dtype], ws.data_ptr(), nbytes, s.cuda_stream)
+        if s != torch.cuda.current_stream(q.device):
+            for t in (dq, dk, dv):
+                t.record_stream(s)
+    _lib.check(rc, "fa_bwd_varlen")
+    return dq, dk, dv
+
+
 def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale: float, k_descale: float,
                 v_descale: float, scale: Optional[float] = None, causal: bool = False,
                 window_left: int = -1, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,

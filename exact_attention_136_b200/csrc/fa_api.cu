@@ -547,6 +547,27 @@ int fa_bwd_window(const void* q, const void* k, const void* v, const void* out, 
                       window_right);
 }
 
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                  int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int H, int H_kv, int D, float scale,
+                  int causal, int window_left, int dtype, void* workspace, size_t workspace_bytes,
+                  fa_stream_t stream) {
+  if (B < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return FA_ERR_ARG;
+  if (!cu_seqlens_q || !cu_seqlens_k || (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return FA_ERR_ARG;
+  // every row and key of a sequence lies in a launched block
+  if ((total_q > 0 && max_seqlen_q < 1) || (total_k > 0 && max_seqlen_k < 1) || max_seqlen_q > total_q ||
+      max_seqlen_k > total_k)
+    return FA_ERR_ARG;
+  const int64_t blocks_kv = static_cast<int64_t>((max_seqlen_k + 127) / 128) * B * (H_kv > 0 ? H_kv : 1);
+  const int64_t blocks_q = static_cast<int64_t>((max_seqlen_q + 127) / 128) * B * H;
+  if (blocks_kv > 0x7fffffff || blocks_q > 0x7fffffff) return FA_ERR_ARG;
+  return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, max_seqlen_q, max_seqlen_k, H, H_kv, D, scale, causal,
+                      window_left, dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), 0.f, 0,
+                      0, -1, cu_seqlens_q, cu_seqlens_k, total_q, total_k);
+}
+
 int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out, const void* dout,
                    const float* lse, void* dq, void* dk, void* dv, int B, int N_q, int N_k, int H, int H_kv, int D,
                    float scale, int causal, int window_left, int dtype, float dropout_p, unsigned long long seed,

@@ -25,10 +25,14 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dout, co
   constexpr int DQ_SMEM = DQ_SMEM_USED > 118 * 1024 ? DQ_SMEM_USED : 118 * 1024;
   const CUtensorMapDataType tdt = DT == DT_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap mq, mk, mv, mdo;
-  if (encode_bnhd(&mq, q, tdt, 2, p.B, p.Nq, p.H, D, 64, 128) ||
-      encode_bnhd(&mk, k, tdt, 2, p.B, p.Nk, p.Hkv, D, 64, 128) ||
-      encode_bnhd(&mv, v, tdt, 2, p.B, p.Nk, p.Hkv, D, 64, 128) ||
-      encode_bnhd(&mdo, dout, tdt, 2, p.B, p.Nq, p.H, D, 64, 128))
+  // packed sequences: one batch of total_q / total_k rows, each sequence
+  // addressed by its first row
+  const int tB = p.cu_q ? 1 : p.B;
+  const int tq = p.cu_q ? p.total_q : p.Nq, tk = p.cu_q ? p.total_k : p.Nk;
+  if (encode_bnhd(&mq, q, tdt, 2, tB, tq, p.H, D, 64, 128) ||
+      encode_bnhd(&mk, k, tdt, 2, tB, tk, p.Hkv, D, 64, 128) ||
+      encode_bnhd(&mv, v, tdt, 2, tB, tk, p.Hkv, D, 64, 128) ||
+      encode_bnhd(&mdo, dout, tdt, 2, tB, tq, p.H, D, 64, 128))
     return FA_ERR_CUDA;
   if (!(ds->attr_set.load(std::memory_order_acquire) & (1u << bit))) {
     if (cudaFuncSetAttribute(fa_bwd_dkdv_kernel<D, DT, DROP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
@@ -49,8 +53,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dout, co
 int backward(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
              void* dq, void* dk, void* dv, int B, int Nq, int Nk, int H, int Hkv, int D, float scale, int causal,
              int window_left, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream,
-             float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0, int window_right = -1) {
-  int rc = validate(q, k, v, const_cast<void*>(out), B, Nq, Nk, H, D, scale, causal, window_left, dtype, Hkv);
+             float dropout_p = 0.f, unsigned long long seed = 0, unsigned offset = 0, int window_right = -1,
+             const int* cu_q = nullptr, const int* cu_k = nullptr, int total_q = 0, int total_k = 0) {
+  // the tensors' rows: B x N_q / N_k, or one batch of total_q / total_k
+  // packed rows (N_q, N_k then the longest sequences, validated by the
+  // packed entry point)
+  const int rB = cu_q ? 1 : B, rNq = cu_q ? total_q : Nq, rNk = cu_q ? total_k : Nk;
+  int rc = validate(q, k, v, const_cast<void*>(out), rB, rNq, rNk, H, D, scale, causal, window_left, dtype, Hkv);
   if (rc != FA_OK) return rc;
   int R = -1;
   rc = right_bound(causal, window_right, Nq, Nk, &R);
@@ -58,34 +67,36 @@ int backward(const void* q, const void* k, const void* v, const void* out, const
   if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
   if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_ARG;
   const bool drop = dropout_p > 0.f;
-  if ((Nq > 0 && (!dout || !lse || !dq)) || (Nk > 0 && (!dk || !dv))) return FA_ERR_ARG;
+  if (cu_q && drop) return FA_ERR_ARG;
+  if ((rNq > 0 && (!dout || !lse || !dq)) || (rNk > 0 && (!dk || !dv))) return FA_ERR_ARG;
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return FA_ERR_ALIGN;
-  const size_t ws = bwd_workspace_bytes(B, Nq, H, D);
+  const size_t ws = bwd_workspace_bytes(rB, rNq, H, D);
   if (ws > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws))
     return FA_ERR_ARG;
-  if (Nq == 0 && Nk == 0) return FA_OK;
+  if (rNq == 0 && rNk == 0) return FA_OK;
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc != FA_OK) return rc;
-  if (Nq == 0) {
+  if (rNq == 0) {
     // no query sees any key: dK = dV = 0
-    const size_t kv_bytes = static_cast<size_t>(B) * Nk * Hkv * D * 2;
+    const size_t kv_bytes = static_cast<size_t>(rB) * rNk * Hkv * D * 2;
     if (cudaMemsetAsync(dk, 0, kv_bytes, stream) != cudaSuccess || cudaMemsetAsync(dv, 0, kv_bytes, stream) != cudaSuccess)
       return FA_ERR_CUDA;
     return FA_OK;
   }
   float* delta = static_cast<float*>(workspace);
-  const int64_t rows = static_cast<int64_t>(B) * Nq * H;
+  const int64_t rows = static_cast<int64_t>(rB) * rNq * H;
   {
+    // ([B, H, N_q], or [H, total_q] like the packed forward's LSE)
     const int64_t want = (rows * (D / 8) + 255) / 256;   // D / 8 threads per row
     const int blocks = static_cast<int>(want < 8 * 148 ? want : 8 * 148);
-    if (D == 64) fa_bwd_prologue_kernel<64><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, B, Nq, H);
-    else fa_bwd_prologue_kernel<128><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, B, Nq, H);
+    if (D == 64) fa_bwd_prologue_kernel<64><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, rB, rNq, H);
+    else fa_bwd_prologue_kernel<128><<<blocks, 256, 0, stream>>>(out, dout, dtype, delta, rB, rNq, H);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  if (Nk == 0) {
+  if (rNk == 0) {
     // no key: dQ = 0
     if (cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * D * 2, stream) != cudaSuccess) return FA_ERR_CUDA;
     return FA_OK;
@@ -110,6 +121,10 @@ int backward(const void* q, const void* k, const void* v, const void* out, const
     p.score_scale = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.nkb = (Nk + 127) / 128;
     p.nqb = (Nq + 127) / 128;
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.total_q = total_q;
+    p.total_k = total_k;
     p.wait_limit_ns = g_wait_limit_ns;
     p.status = ds->status;
     if (drop) {

@@ -89,6 +89,13 @@ struct BwdParams {
   int window_left;          // keys at most this many before the query; -1 = unlimited
   int window_right;         // keys at most this many after it; -1 = unlimited, 0 under
                             // causal (set by the host, below N_k + N_q < 2^31)
+  // packed sequences (null cu_q: the padded batch [B, N_q / N_k, ...]):
+  // sequence b owns rows cu_q[b] .. cu_q[b+1] of [total_q, H, D] (and of the
+  // statistics [H, total_q]) and keys cu_k[b] .. cu_k[b+1] of [total_k, H_kv, D];
+  // N_q / N_k are then the longest sequences
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
   float scale;              // softmax scale
   float score_scale;        // scale * log2(e)
   int nkb;                  // key blocks per (batch, head)
@@ -172,18 +179,57 @@ __device__ __forceinline__ bool grad_bar_and(bool v) {
   return r != 0u;
 }
 
-// Query blocks that see key block jk: a right window (causal: 0) keeps
-// queries at least window_right before the key (absolute indices), a left
-// window keeps queries at most window_left after it.
-__device__ __forceinline__ void bwd_query_range(int jk, const BwdParams& p, int& i_lo, int& i_hi) {
-  const int nqb = (p.Nq + 127) / 128;
+// One sequence of the batch: its sizes and where its rows start.  Packed
+// sequences are clamped into the packed tensors (as in the forward), so bad
+// offsets give wrong results but no access outside them.
+struct BwdSeq {
+  int nq, nk;            // queries and keys of the sequence
+  int tq, tk, tb;        // TMA row of its first query / key, TMA batch coordinate
+  long long qrow, krow;  // its first query / key row in [rows, heads, D]
+  long long stat, stat_h;   // statistic of its first query for head 0, head stride
+};
+
+__device__ __forceinline__ BwdSeq bwd_seq(int b, const BwdParams& p) {
+  BwdSeq s;
+  if (p.cu_q) {
+    const int q_start = min(max(__ldg(p.cu_q + b), 0), p.total_q);
+    const int k_start = min(max(__ldg(p.cu_k + b), 0), p.total_k);
+    s.nq = min(max(__ldg(p.cu_q + b + 1), q_start), p.total_q) - q_start;
+    s.nk = min(max(__ldg(p.cu_k + b + 1), k_start), p.total_k) - k_start;
+    s.tq = q_start;
+    s.tk = k_start;
+    s.tb = 0;
+    s.qrow = q_start;
+    s.krow = k_start;
+    s.stat = q_start;
+    s.stat_h = p.total_q;
+  } else {
+    s.nq = p.Nq;
+    s.nk = p.Nk;
+    s.tq = 0;
+    s.tk = 0;
+    s.tb = b;
+    s.qrow = static_cast<long long>(b) * p.Nq;
+    s.krow = static_cast<long long>(b) * p.Nk;
+    s.stat = static_cast<long long>(b) * p.H * p.Nq;
+    s.stat_h = p.Nq;
+  }
+  return s;
+}
+
+// Query blocks of a sequence of nq queries and nk keys that see key block
+// jk: a right window (causal: 0) keeps queries at least window_right before
+// the key (absolute indices), a left window keeps queries at most
+// window_left after it.
+__device__ __forceinline__ void bwd_query_range(int jk, const BwdParams& p, int nq, int nk, int& i_lo, int& i_hi) {
+  const int nqb = (nq + 127) / 128;
   i_lo = p.window_right >= 0 ? max(0, jk * 128 - p.window_right) / 128 : 0;
   i_hi = nqb - 1;
   if (p.window_left >= 0) {
     const long long last = static_cast<long long>(jk) * 128 + 127 + p.window_left;
     i_hi = static_cast<int>(min(static_cast<long long>(i_hi), last / 128));
   }
-  if (jk * 128 >= p.Nk) i_hi = i_lo - 1;   // (not launched: the grid covers N_k)
+  if (jk * 128 >= nk) i_hi = i_lo - 1;   // past the sequence's keys (packed batches)
 }
 
 template <int D, int DT, bool DROP>
@@ -205,8 +251,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const int jk = static_cast<int>(blockIdx.x) % p.nkb;
   const int bhk = static_cast<int>(blockIdx.x) / p.nkb;   // (batch, K/V head)
   const int b = bhk / p.Hkv, hk = bhk - (bhk / p.Hkv) * p.Hkv;
+  const BwdSeq sq = bwd_seq(b, p);
   int i_lo, i_hi;
-  bwd_query_range(jk, p, i_lo, i_hi);
+  bwd_query_range(jk, p, sq.nq, sq.nk, i_lo, i_hi);
   // The n-th query block a CTA visits is i_lo + (n + rot) mod cnt: causal
   // CTAs already start at their own diagonal; the others start at a block
   // of their own, so CTAs running side by side read different Q blocks.
@@ -262,10 +309,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_arrive_expect_tx(smem_u32(&sh->kv_full), 2 * C::TILE);
 #pragma unroll
       for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d_hint(sbase + C::OFF_K + c * C::CHUNK, &tm_k, smem_u32(&sh->kv_full), c * 64, hk, jk * 128, b,
-                         pol_kv);
-        tma_load_4d_hint(sbase + C::OFF_V + c * C::CHUNK, &tm_v, smem_u32(&sh->kv_full), c * 64, hk, jk * 128, b,
-                         pol_kv);
+        tma_load_4d_hint(sbase + C::OFF_K + c * C::CHUNK, &tm_k, smem_u32(&sh->kv_full), c * 64, hk,
+                         sq.tk + jk * 128, sq.tb, pol_kv);
+        tma_load_4d_hint(sbase + C::OFF_V + c * C::CHUNK, &tm_v, smem_u32(&sh->kv_full), c * 64, hk,
+                         sq.tk + jk * 128, sq.tb, pol_kv);
       }
       int nq = 0, nd = 0;   // Q and dO loads issued
       for (int n = 0; n < visits; ++n) {
@@ -281,7 +328,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         mbar_arrive_expect_tx(qbar, C::TILE);
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d_hint(sbase + C::OFF_Q + s * C::TILE + c * C::CHUNK, &tm_q, qbar, c * 64, hq, i * 128, b, pol_q);
+          tma_load_4d_hint(sbase + C::OFF_Q + s * C::TILE + c * C::CHUNK, &tm_q, qbar, c * 64, hq, sq.tq + i * 128,
+                           sq.tb, pol_q);
         ++nq;
         if (!mbar_wait(smem_u32(&sh->do_empty), (n & 1) ^ 1, lim)) {
           bwd_error(sh, p, ST_TIMEOUT_LOAD);
@@ -292,7 +340,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         mbar_arrive_expect_tx(dbar, C::TILE);
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d_hint(sbase + C::OFF_DO + c * C::CHUNK, &tm_do, dbar, c * 64, hq, i * 128, b, pol_q);
+          tma_load_4d_hint(sbase + C::OFF_DO + c * C::CHUNK, &tm_do, dbar, c * 64, hq, sq.tq + i * 128, sq.tb,
+                           pol_q);
         ++nd;
       }
       if (!ok) {
@@ -404,12 +453,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       const int hq = hk * p.qpk + qn;
       const int i = i_lo + (ib + rot < cnt ? ib + rot : ib + rot - cnt);
-      const long long base = (static_cast<long long>(b) * p.H + hq) * p.Nq;
+      const long long base = sq.stat + hq * sq.stat_h;
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const int ql = 2 * u + x, q = i * 128 + ql;
         float nl = -INFINITY, nd = 0.f;
-        if (q < p.Nq) {
+        if (q < sq.nq) {
           const float l = p.lse[base + q];
           if (l != -INFINITY) nl = l * -1.4426950408889634f;
           nd = -p.delta[base + q];
@@ -448,7 +497,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (++ib == cnt) { ib = 0; ++qn; }
       const int buf = n & 1;
       const int q0 = i * 128;
-      const bool need_mask = (jk * 128 + 128 > p.Nk) || (p.window_right >= 0 && jk * 128 + 127 > q0 + p.window_right) ||
+      const bool need_mask = (jk * 128 + 128 > sq.nk) || (p.window_right >= 0 && jk * 128 + 127 > q0 + p.window_right) ||
                              (p.window_left >= 0 && jk * 128 < q0 + 127 - p.window_left);
       // dropout keep bits of this thread's key for its 64 queries (bit e:
       // query q0 + 64 * half + e).  The generator gives 8 keys of one query
@@ -496,7 +545,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const int q = q0 + half * 64 + e;
-          const bool vis = key < p.Nk && (p.window_right < 0 || key <= q + p.window_right) &&
+          const bool vis = key < sq.nk && (p.window_right < 0 || key <= q + p.window_right) &&
                            (p.window_left < 0 || key >= q - p.window_left);
           pv[e] = vis ? pv[e] : -INFINITY;
         }
@@ -606,7 +655,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_after();
     }
     if (ok) {
-      const long long row = (static_cast<long long>(b) * p.Nk + key) * p.Hkv + hk;
+      const long long row = (sq.krow + key) * p.Hkv + hk;
       uint8_t* dv_row = reinterpret_cast<uint8_t*>(p.dv) + (row * D + half * (D / 2)) * 2;
       uint8_t* dk_row = reinterpret_cast<uint8_t*>(p.dk) + (row * D + half * (D / 2)) * 2;
 #pragma unroll
@@ -620,7 +669,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] = k[e] = 0u;
         }
-        if (key < p.Nk) {
+        if (key < sq.nk) {
           store_out_row16<DT>(dv_row + c * 32, reinterpret_cast<const float*>(v), 1.f);
           store_out_row16<DT>(dk_row + c * 32, reinterpret_cast<const float*>(k), p.scale);
         }
@@ -702,12 +751,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const int bh = static_cast<int>(blockIdx.x) / p.nqb;
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int hk = h / p.qpk;   // this query head's K/V head
+  const BwdSeq sq = bwd_seq(b, p);
   const int q0 = iq * 128;
   // key blocks the rows of this query block see (as in the forward)
-  const int qe = min(q0 + 127, p.Nq - 1);
+  const int qe = min(q0 + 127, sq.nq - 1);
   const int j_lo = p.window_left >= 0 ? max(0, q0 - p.window_left) / 128 : 0;
-  const int j_hi = p.window_right >= 0 ? min(qe + p.window_right, p.Nk - 1) / 128 : p.nkb - 1;
-  const int cnt = (q0 < p.Nq && p.Nk > 0) ? max(0, j_hi - j_lo + 1) : 0;
+  const int j_hi = p.window_right >= 0 ? min(qe + p.window_right, sq.nk - 1) / 128 : (sq.nk - 1) / 128;
+  const int cnt = (q0 < sq.nq && sq.nk > 0) ? max(0, j_hi - j_lo + 1) : 0;
   const uint64_t lim = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -749,8 +799,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_arrive_expect_tx(smem_u32(&sh->q_full), 2 * C::TILE);
 #pragma unroll
       for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d_hint(sbase + Q::OFF_Q + c * C::CHUNK, &tm_q, smem_u32(&sh->q_full), c * 64, h, q0, b, pol_q);
-        tma_load_4d_hint(sbase + Q::OFF_DO + c * C::CHUNK, &tm_do, smem_u32(&sh->q_full), c * 64, h, q0, b, pol_q);
+        tma_load_4d_hint(sbase + Q::OFF_Q + c * C::CHUNK, &tm_q, smem_u32(&sh->q_full), c * 64, h, sq.tq + q0, sq.tb,
+                         pol_q);
+        tma_load_4d_hint(sbase + Q::OFF_DO + c * C::CHUNK, &tm_do, smem_u32(&sh->q_full), c * 64, h, sq.tq + q0,
+                         sq.tb, pol_q);
       }
       int nk = 0, nv = 0;   // K and V loads issued
       for (int n = 0; n < cnt && ok; ++n) {
@@ -761,14 +813,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d_hint(sbase + Q::OFF_K + sk * C::TILE + c * C::CHUNK, &tm_k, smem_u32(&sh->k_full[sk]), c * 64,
-                           hk, j * 128, b, pol_kv);
+                           hk, sq.tk + j * 128, sq.tb, pol_kv);
         ++nk;
         if (!mbar_wait(smem_u32(&sh->v_empty[sv]), ((n / Q::VS) & 1) ^ 1, lim)) { ok = false; break; }
         mbar_arrive_expect_tx(smem_u32(&sh->v_full[sv]), C::TILE);
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d_hint(sbase + Q::OFF_V + sv * C::TILE + c * C::CHUNK, &tm_v, smem_u32(&sh->v_full[sv]), c * 64,
-                           hk, j * 128, b, pol_kv);
+                           hk, sq.tk + j * 128, sq.tb, pol_kv);
         ++nv;
       }
       if (!ok) {
@@ -856,10 +908,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int r = quad * 32 + sub * 16 + (lane & 15);        // TMEM lane: query row
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32 + sub * 16) << 16;
     const int q = q0 + r;
-    const long long bhq = static_cast<long long>(bh) * p.Nq;
+    const long long bhq = sq.stat + h * sq.stat_h;
     // this row's statistics: -LSE * log2(e) (-inf: the row contributes nothing) and D
     float nlse2 = -INFINITY, dlt = 0.f;
-    if (q < p.Nq) {
+    if (q < sq.nq) {
       const float l = p.lse[bhq + q];
       if (l != -INFINITY) nlse2 = l * -1.4426950408889634f;
       dlt = p.delta[bhq + q];
@@ -876,7 +928,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (__any_sync(0xffffffffu, bwd_aborted(&sh->abort_flag))) { ok = false; break; }
       const int k0 = (j_lo + n) * 128;
       const uint32_t s_col = (n & 1) ? Q::S_COL1 : Q::S_COL0;
-      const bool need_mask = (k0 + 128 > p.Nk) || (p.window_right >= 0 && k0 + 127 > q0 + p.window_right) ||
+      const bool need_mask = (k0 + 128 > sq.nk) || (p.window_right >= 0 && k0 + 127 > q0 + p.window_right) ||
                              (p.window_left >= 0 && k0 < q0 + 127 - p.window_left);
       // dropout keep bits of this row's keys k0 + 64 * half + [0, 64)
       uint32_t keep[2] = {0u, 0u};
@@ -909,7 +961,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) {
           const int key = k0 + half * 64 + e;
-          const bool vis = key < p.Nk && (p.window_right < 0 || key <= q + p.window_right) &&
+          const bool vis = key < sq.nk && (p.window_right < 0 || key <= q + p.window_right) &&
                            (p.window_left < 0 || key >= q - p.window_left);
           pv[e] = vis ? pv[e] : -INFINITY;
         }
@@ -978,7 +1030,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     // its row; only rows inside N_q are stored)
     if (have || (ok && cnt == 0)) {
       uint8_t* dq_row = reinterpret_cast<uint8_t*>(p.dq) +
-                        (((static_cast<long long>(b) * p.Nq + q) * p.H + h) * D + half * (D / 2)) * 2;
+                        (((sq.qrow + q) * p.H + h) * D + half * (D / 2)) * 2;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[16];
@@ -989,7 +1041,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] = 0u;
         }
-        if (q < p.Nq) store_out_row16<DT>(dq_row + c * 32, reinterpret_cast<const float*>(v), p.scale);
+        if (q < sq.nq) store_out_row16<DT>(dq_row + c * 32, reinterpret_cast<const float*>(v), p.scale);
       }
     }
   }

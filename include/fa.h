@@ -327,6 +327,24 @@ int fa_bwd_window(const void* q, const void* k, const void* v, const void* out, 
                   int dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_bwd_varlen -- the backward of fa_fwd_varlen over the same packed batch:
+ * q, out, dout, dq [total_q, H, D]; k, v, dk, dv [total_k, H_kv, D]; lse
+ * [H, total_q] (the forward's); cu_seqlens_q / cu_seqlens_k, B, causal and
+ * window_left as given to the forward.  Gradients are taken within each
+ * sequence; keys no query of their sequence sees get dK = dV = 0.  Here
+ * max_seqlen_q and max_seqlen_k must bound every sequence's query and key
+ * count (the launch covers that many blocks per sequence; rows or keys past
+ * them are not computed).  workspace: fa_bwd_workspace_bytes(1, total_q, H,
+ * D) bytes, 256-byte aligned.  Returns FA_ERR_ARG for bad sizes or pointers
+ * (before any GPU work), else as fa_bwd_gqa.
+ */
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
+                  int total_k, int H, int H_kv, int D, float scale, int causal, int window_left,
+                  int dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fa_bwd_dropout -- fa_bwd_gqa for the forward of fa_fwd_dropout: the same
  * dropout_p, seed and offset redraw the forward's keep bits, and the
  * gradients are those of O = (Z / (1 - p) * P) V: dV = (Z P / (1 - p))^T dO,

@@ -306,3 +306,27 @@ def test_window_arguments_validated(kw, expect):
     g = _lib.lib().fa_bwd_window
     assert g(A, A, A, A, A, A, A, A, A, 1, a["nq"], a["nk"], a["H"], a["H_kv"], a["D"], 0.125, a["causal"], a["wl"],
              a["wr"], _lib.FA_FP16, A, 1 << 40, None) == expect
+
+
+@pytest.mark.parametrize("kw, expect", [
+    (dict(B=0), _lib.FA_ERR_ARG),
+    (dict(cu_q=None), _lib.FA_ERR_ARG),
+    (dict(cu_k=A + 2), _lib.FA_ERR_ARG),
+    (dict(max_q=0), _lib.FA_ERR_ARG),               # rows but no launched query block
+    (dict(max_k=0), _lib.FA_ERR_ARG),               # keys but no launched key block
+    (dict(max_q=5000), _lib.FA_ERR_ARG),
+    (dict(max_k=9000), _lib.FA_ERR_ARG),
+    (dict(D=96), _lib.FA_ERR_UNSUPPORTED),
+    (dict(dt=_lib.FA_E4M3, D=128), _lib.FA_ERR_UNSUPPORTED),
+    (dict(H=3, H_kv=2), _lib.FA_ERR_ARG),
+    (dict(ws_bytes=100), _lib.FA_ERR_ARG),           # workspace below H * total_q floats
+])
+def test_varlen_backward_arguments_validated(kw, expect):
+    """fa_bwd_varlen checks its sizes and pointers on the host, before any GPU work."""
+    a = dict(cu_q=A, cu_k=A, B=2, max_q=100, max_k=100, total_q=150, total_k=150, H=2, H_kv=2, D=64, causal=0,
+             wl=-1, dt=_lib.FA_FP16, ws_bytes=1 << 20)
+    a.update(kw)
+    f = _lib.lib().fa_bwd_varlen
+    assert f(A, A, A, A, A, A, A, A, A, a["cu_q"], a["cu_k"], a["B"], a["max_q"], a["max_k"], a["total_q"],
+             a["total_k"], a["H"], a["H_kv"], a["D"], 0.1, a["causal"], a["wl"], a["dt"], A, a["ws_bytes"],
+             None) == expect

@@ -92,3 +92,82 @@ def test_no_keys_at_all():
     out, lse = forward_varlen(q, k, k, cu_q, cu_k, max(lens), 0, 0.125, False)
     torch.cuda.synchronize()
     assert bool((out == 0).all()) and bool(torch.isinf(lse).all() and (lse < 0).all())
+
+
+U = {"fp16": 2.0 ** -11, "bf16": 2.0 ** -8}
+
+BWD_CASES = [
+    # lens_q, lens_k, H, H_kv, D, dtype, causal, window_left
+    ([1, 300, 128, 517, 64], [1, 300, 128, 517, 64], 2, 2, 128, "bf16", True, -1),
+    ([700, 5, 256, 1000], [700, 5, 256, 1000], 4, 2, 64, "fp16", False, -1),
+    ([129, 0, 333, 1], [200, 17, 0, 90], 2, 1, 128, "fp16", False, -1),
+    ([600, 255, 1024], [600, 255, 1024], 2, 2, 128, "bf16", True, 100),
+]
+
+
+@pytest.mark.parametrize("lens_q,lens_k,H,h_kv,D,dt,causal,wl", BWD_CASES)
+def test_varlen_backward_matches_oracle_per_sequence(lens_q, lens_k, H, h_kv, D, dt, causal, wl):
+    """fa_bwd_varlen: every sequence's dQ, dK, dV against the oracle's exact
+    gradients of that sequence alone, under the per-element bounds of the
+    padded backward's tests; a sequence without keys gets dQ = 0, keys
+    without queries dK = dV = 0."""
+    from exact_attention_136_b200 import backward_varlen
+    from oracle import attention_backward_ref
+    from tests.oracle_cmp import backward_bounds
+    qkv, q, k, v, cu_q, cu_k = _packed(lens_q, lens_k, H, h_kv, D, dt, 700 + sum(lens_q))
+    tq = int(sum(lens_q))
+    do = inputs.make_qkv(1, max(tq, 1), 1, H, D, dt, seeds=(901, 902, 903)).q[0, :tq]
+    scale = 1.0 / math.sqrt(D)
+    qd, kd, vd, dod, cq, ck = (t.contiguous().to(DEV) for t in (q, k, v, do, cu_q, cu_k))
+    out, lse = forward_varlen(qd, kd, vd, cq, ck, max(lens_q), max(lens_k), scale, causal, wl)
+    dq, dk, dv = backward_varlen(qd, kd, vd, out, lse, dod, cq, ck, max(lens_q), max(lens_k), scale, causal, wl)
+    torch.cuda.synchronize()
+    assert device_status()[0] == 0
+    f64 = lambda t: t.detach().double().cpu().numpy()
+    gq, gk, gv, o_all, l_all = f64(dq), f64(dk), f64(dv), f64(out), f64(lse)
+    for name, g in (("dq", gq), ("dk", gk), ("dv", gv)):
+        assert np.all(np.isfinite(g)), f"{name}: rows left unwritten"
+    for b in range(len(lens_q)):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        k0, k1 = int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0 or k1 == k0:
+            # nothing to attend: zero gradients
+            assert not gq[q0:q1].any() and not gk[k0:k1].any() and not gv[k0:k1].any(), f"sequence {b}"
+            continue
+        args = [f64(t)[None] for t in (q[q0:q1], k[k0:k1], v[k0:k1], do[q0:q1])]
+        ref = attention_backward_ref(*args, scale, causal, wl)
+        bounds = backward_bounds(*args, o_all[None, q0:q1], l_all[None, :, q0:q1], scale, causal, wl, U[dt])
+        for name, got, want, bnd in zip(("dq", "dk", "dv"), (gq[q0:q1], gk[k0:k1], gv[k0:k1]), ref, bounds):
+            err = np.abs(got - want[0])
+            worst = float(np.max(err / (bnd[0] + U[dt] * np.abs(want[0]) + 1e-6)))
+            assert worst <= 1.0, f"sequence {b} {name}: error exceeds its bound by x{worst:.3f}"
+
+
+def test_varlen_backward_equal_lengths_reproduce_the_padded_batch():
+    """Equal lengths: the packed backward takes the padded backward's steps in the same order (bit for bit)."""
+    from exact_attention_136_b200 import backward, backward_varlen
+    B, n, H, h_kv, D = 3, 513, 4, 2, 128
+    qkv = inputs.make_qkv(B, n, n, H, D, "bf16", seeds=(21, 22, 23), h_kv=h_kv)
+    q, k, v = qkv.q.to(DEV), qkv.k.to(DEV), qkv.v.to(DEV)
+    do = inputs.make_qkv(B, n, n, H, D, "bf16", seeds=(24, 25, 26)).q.to(DEV)
+    out, lse = forward(q, k, v, 0.09, True)
+    ref = backward(q, k, v, out, lse, do, 0.09, True)
+    cu = torch.arange(0, (B + 1) * n, n, dtype=torch.int32, device=DEV)
+    flat = lambda t: t.reshape(B * n, t.shape[2], D)
+    # the packed LSE is [H, total_q]: batch b's rows follow batch b-1's
+    lse_p = lse.permute(1, 0, 2).reshape(H, B * n).contiguous()
+    got = backward_varlen(flat(q), flat(k), flat(v), flat(out), lse_p, flat(do), cu, cu, n, n, 0.09, True)
+    torch.cuda.synchronize()
+    for g, r in zip(got, ref):
+        assert torch.equal(g, flat(r))
+
+
+def test_varlen_backward_rejects_bad_sizes():
+    from exact_attention_136_b200 import backward_varlen
+    t = torch.zeros((256, 2, 64), device=DEV, dtype=torch.float16)
+    lse = torch.zeros((2, 256), device=DEV)
+    cu = torch.tensor([0, 128, 256], dtype=torch.int32, device=DEV)
+    with pytest.raises(_lib.FAError):
+        backward_varlen(t, t, t, t, lse, t, cu, cu, 0, 128)       # rows but max_seqlen_q 0
+    with pytest.raises(_lib.FAError):
+        backward_varlen(t, t, t, t, lse, t, cu, cu, 128, 300)     # longer than the packed keys

@@ -414,42 +414,63 @@ def main():
         long_run = {"launches": n_long, "seconds": lms / 1e3, "ms_per_step": lms / n_long, "value": lval,
                     "clocks": lclocks, "value_clock_normalised": clock_normalised(lval, lclocks)}
 
-    # end to end through the host-buffer entry point: H2D inputs, kernel, D2H out + lse
-    ho = torch.empty((w.B, w.n_q, w.H, w.D), dtype=out_dtype, pin_memory=True)
-    hl = torch.empty((w.B, w.H, w.n_q), dtype=torch.float32, pin_memory=True)
-    staging = {"q": q, "k": k, "v": v, "out": out, "lse": lse}
+    # end to end through the host-buffer entry point: H2D inputs, kernel, D2H out + lse, every step.
+    # Three streams, each with its own device staging and pinned result buffers, take the steps in
+    # turn (fa_fwd_host_async), so a step's copies in overlap the previous steps' forward and copies
+    # out; grouped heads, split key ranges and masks go through pinned copies and the Python forward,
+    # one step at a time.
+    piped = w.h_kv == w.H and splits == 1 and mask is None
+    n_pipe = 3 if piped else 1
+    e2e_streams = [stream] + [torch.cuda.Stream(dev) for _ in range(n_pipe - 1)]
+    stagings = [{"q": q, "k": k, "v": v, "out": out, "lse": lse}] + [
+        {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+         "out": torch.empty_like(out), "lse": torch.empty_like(lse)} for _ in range(n_pipe - 1)]
+    hos = [torch.empty((w.B, w.n_q, w.H, w.D), dtype=out_dtype, pin_memory=True) for _ in range(n_pipe)]
+    hls = [torch.empty((w.B, w.H, w.n_q), dtype=torch.float32, pin_memory=True) for _ in range(n_pipe)]
     desc = (qkv.q_descale, qkv.k_descale, qkv.v_descale)
+    turn = [0]
 
     def e2e_step():
-        if w.h_kv == w.H and splits == 1 and mask is None:
-            forward_host(hq, hk, hv, staging, w.scale, w.causal, w.window_left, desc, ho, hl, stream)
+        i = turn[0] % n_pipe
+        turn[0] += 1
+        if piped:
+            forward_host(hq, hk, hv, stagings[i], w.scale, w.causal, w.window_left, desc, hos[i], hls[i],
+                         e2e_streams[i], synchronize=False)
         else:
-            # fa_fwd_host takes H K/V heads; grouped heads go through pinned
-            # copies on the same stream and the Python forward
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
             step()
-            ho.copy_(out, non_blocking=True)
-            hl.copy_(lse, non_blocking=True)
+            hos[0].copy_(out, non_blocking=True)
+            hls[0].copy_(lse, non_blocking=True)
             stream.synchronize()
 
-    for _ in range(2):
+    for _ in range(2 * n_pipe):
         e2e_step()
     barrier()
     torch.cuda.synchronize(dev)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
+    for s_ in e2e_streams[1:]:
+        s_.wait_event(t0)
     for _ in range(args.e2e_steps):
         e2e_step()
+    for s_ in e2e_streams[1:]:
+        stream.wait_stream(s_)
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     ems = max_over_ranks(t0.elapsed_time(t1), dev)
     e2e_value = world * flops * args.e2e_steps / (ems / 1e3) / 1e12
+    # every step computed the same forward: each stream's host result equals the device-timed run's
+    ref_out = stagings[0]["out"].cpu()
+    for i in range(n_pipe if piped else 0):
+        if not torch.equal(hos[i], ref_out):
+            raise RuntimeError(f"e2e: host result of stream {i} differs from the device forward")
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    d2h = hos[0].numel() * hos[0].element_size() + hls[0].numel() * hls[0].element_size()
+    del stagings, e2e_streams
 
     peak, peak_src, sustained = measured_peaks(w.dtype)
     bound, bpeak, bsrc = binding_roofline(w, sms, (clocks or {}).get("sm_max_mhz"))
@@ -463,7 +484,7 @@ def main():
                "sample": f"fp64 oracle on {args.cpu_rows} sampled query rows of each of the {w.B * w.H} "
                          f"(batch, head) pairs ({n_rows} rows, {dt:.1f} s); FLOP credited per row = "
                          f"the workload's average 4*N_k*D*block_fraction"}
-    del hq, hk, hv, ho, hl
+    del hq, hk, hv, hos, hls
 
     # the other configurations, one after another on this GPU (rank 0 of a single-GPU run)
     configs = None
@@ -500,8 +521,9 @@ def main():
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps,
-                "api": "fa_fwd_host (pinned host buffers)" if (w.h_kv == w.H and splits == 1 and mask is None)
-                       else "pinned host copies + forward"},
+                "api": "fa_fwd_host_async (pinned host buffers), 3 streams in turn: a step's copies in overlap "
+                       "the previous steps' forward and copies out" if piped
+                       else "pinned host copies + forward, one step at a time"},
         "roofline": {"bound": bound, "achieved": per_launch_tflops, "peak": bpeak, "unit": UNIT,
                      "frac": per_launch_tflops / bpeak, "traffic": traffic, "peak_source": bsrc,
                      "tensor_peak": peak, "tensor_peak_source": f"{peak_src} bf16 burst" +

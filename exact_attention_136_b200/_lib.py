@@ -47,6 +47,9 @@ SIGNATURES = {
     "fa_fwd_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                              _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, _c_float,
                              _c_float, _vp]),
+    "fa_fwd_host_async": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                   _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, _c_float,
+                                   _c_float, _vp]),
     "fa_fwd_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                                 _c_int, _c_int, _c_int, _c_float, _c_float, _c_float, _vp]),
     "fa_bwd_workspace_bytes": (ctypes.c_size_t, [_c_int, _c_int, _c_int, _c_int]),

@@ -427,12 +427,16 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
 
 def forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, staging, scale: float, causal: bool = False,
                  window_left: int = -1, descales=(1.0, 1.0, 1.0), out: Optional[torch.Tensor] = None,
-                 lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+                 lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                 synchronize: bool = True):
     """Forward on HOST tensors through fa_fwd_host.
 
     q, k, v are CPU tensors (pinned for asynchronous copies); `staging` is a
     dict of device tensors "q", "k", "v", "out", "lse" that the call copies
-    through.  Returns the host (out, lse).
+    through.  Returns the host (out, lse).  synchronize=False enqueues the
+    copies and the forward on the stream and returns at once
+    (fa_fwd_host_async): out and lse are valid after the stream completes,
+    and calls on other streams with their own staging run concurrently.
     """
     B, n_q, H, D = q.shape
     n_k = k.shape[1]
@@ -445,13 +449,13 @@ def forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, staging, sca
     dev = staging["q"].device
     with torch.cuda.device(dev):
         s = stream if stream is not None else torch.cuda.current_stream(dev)
-        rc = _lib.lib().fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                    staging["q"].data_ptr(), staging["k"].data_ptr(), staging["v"].data_ptr(),
-                                    staging["out"].data_ptr(), staging["lse"].data_ptr(), B, n_q, n_k, H, D,
-                                    float(scale), int(bool(causal)), int(window_left), dt,
-                                    float(descales[0]), float(descales[1]), float(descales[2]),
-                                    s.cuda_stream)
-    _lib.check(rc, "fa_fwd_host")
+        fn = _lib.lib().fa_fwd_host if synchronize else _lib.lib().fa_fwd_host_async
+        rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                staging["q"].data_ptr(), staging["k"].data_ptr(), staging["v"].data_ptr(),
+                staging["out"].data_ptr(), staging["lse"].data_ptr(), B, n_q, n_k, H, D,
+                float(scale), int(bool(causal)), int(window_left), dt,
+                float(descales[0]), float(descales[1]), float(descales[2]), s.cuda_stream)
+    _lib.check(rc, "fa_fwd_host" if synchronize else "fa_fwd_host_async")
     return out, lse
 
 

@@ -468,30 +468,59 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float*
                      nullptr, 0, 0, 0, 0, 0.f, 0, 0, cu_seqlens_q, cu_seqlens_k, total_q, total_k);
 }
 
-int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,
-                void* dv, void* dout, float* dlse, int B, int N_q, int N_k, int H, int D, float scale,
-                int causal, int window_left, int dtype, float q_descale, float k_descale,
-                float v_descale, fa_stream_t stream) {
+}  // extern "C"
+
+namespace fa {
+namespace {
+// Copies in, the forward, copies out, all enqueued on `s` (fa_fwd_host and
+// fa_fwd_host_async).
+int host_forward(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,
+                 void* dv, void* dout, float* dlse, int B, int N_q, int N_k, int H, int D, float scale,
+                 int causal, int window_left, int dtype, float q_descale, float k_descale,
+                 float v_descale, cudaStream_t s) {
   if (!q || !k || !v || !out) return FA_ERR_ARG;
-  int rc = fa::validate(dq, dk, dv, dout, B, N_q, N_k, H, D, scale, causal, window_left, dtype, H);
+  int rc = validate(dq, dk, dv, dout, B, N_q, N_k, H, D, scale, causal, window_left, dtype, H);
   if (rc != FA_OK) return rc;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const size_t es = fa::elem_bytes(dtype);
+  const size_t es = elem_bytes(dtype);
   const size_t nq = static_cast<size_t>(B) * N_q * H * D;
   const size_t nk = static_cast<size_t>(B) * N_k * H * D;
   if (cudaMemcpyAsync(dq, q, nq * es, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(dk, k, nk * es, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(dv, v, nk * es, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return FA_ERR_CUDA;
-  rc = fa::forward(dq, dk, dv, dout, dlse, B, N_q, N_k, H, H, D, scale, causal, window_left, dtype,
-                   q_descale, k_descale, v_descale, s);
+  rc = forward(dq, dk, dv, dout, dlse, B, N_q, N_k, H, H, D, scale, causal, window_left, dtype, q_descale,
+               k_descale, v_descale, s);
   if (rc != FA_OK) return rc;
   if (cudaMemcpyAsync(out, dout, nq * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_CUDA;
   if (lse && dlse &&
       cudaMemcpyAsync(lse, dlse, static_cast<size_t>(B) * H * N_q * sizeof(float), cudaMemcpyDeviceToHost,
                       s) != cudaSuccess)
     return FA_ERR_CUDA;
+  return FA_OK;
+}
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,
+                void* dv, void* dout, float* dlse, int B, int N_q, int N_k, int H, int D, float scale,
+                int causal, int window_left, int dtype, float q_descale, float k_descale,
+                float v_descale, fa_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int rc = fa::host_forward(q, k, v, out, lse, dq, dk, dv, dout, dlse, B, N_q, N_k, H, D, scale, causal,
+                                  window_left, dtype, q_descale, k_descale, v_descale, s);
+  if (rc != FA_OK) return rc;
   return cudaStreamSynchronize(s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_fwd_host_async(const void* q, const void* k, const void* v, void* out, float* lse, void* dq, void* dk,
+                      void* dv, void* dout, float* dlse, int B, int N_q, int N_k, int H, int D, float scale,
+                      int causal, int window_left, int dtype, float q_descale, float k_descale,
+                      float v_descale, fa_stream_t stream) {
+  return fa::host_forward(q, k, v, out, lse, dq, dk, dv, dout, dlse, B, N_q, N_k, H, D, scale, causal,
+                          window_left, dtype, q_descale, k_descale, v_descale,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N_q,

@@ -247,6 +247,23 @@ int fa_fwd_host(const void* q, const void* k, const void* v, void* out, float* l
                 float v_descale, fa_stream_t stream);
 
 /*
+ * fa_fwd_host_async -- fa_fwd_host without the final synchronisation: the
+ * copies in, the forward and the copies out are enqueued on `stream` and the
+ * call returns.  out and lse hold the result once `stream` has completed
+ * (synchronise it, or wait on an event recorded after the call); the host
+ * buffers must stay valid and unmodified until then, and must be pinned for
+ * the copies to overlap other work.  Calls on different streams with their
+ * own device buffers run concurrently, so one batch's copies in overlap
+ * another's forward and copies out.  Arguments and return values as
+ * fa_fwd_host.
+ */
+int fa_fwd_host_async(const void* q, const void* k, const void* v, void* out, float* lse,
+                      void* dq, void* dk, void* dv, void* dout, float* dlse,
+                      int B, int N_q, int N_k, int H, int D, float scale, int causal,
+                      int window_left, int dtype, float q_descale, float k_descale,
+                      float v_descale, fa_stream_t stream);
+
+/*
  * fa_fwd_noalloc -- the forward of fa_fwd / fa_fwd_fp8 (dtype FA_E4M3 uses
  * the three descales; other dtypes take 1.0) for callers that cannot
  * allocate device memory: code whose allocations must all come from its own

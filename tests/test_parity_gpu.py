@@ -430,6 +430,33 @@ def test_host_buffer_entry_point_matches_device_entry():
     assert torch.equal(ho, do.cpu()) and torch.equal(hl, dl.cpu())
 
 
+def test_async_host_entry_point_on_three_streams():
+    """fa_fwd_host_async: batches enqueued on three streams with their own
+    staging, nothing synchronised between calls; after the streams complete
+    every host result equals the device entry's for its batch."""
+    dev = torch.device("cuda", 0)
+    B, n, H, D = 1, 700, 4, 128
+    batches = [inputs.make_qkv(B, n, n, H, D, "bf16", seeds=(81 + 3 * i, 82 + 3 * i, 83 + 3 * i)) for i in range(6)]
+    streams = [torch.cuda.Stream(dev) for _ in range(3)]
+    stagings = [{"q": torch.empty((B, n, H, D), dtype=torch.bfloat16, device=dev),
+                 "k": torch.empty((B, n, H, D), dtype=torch.bfloat16, device=dev),
+                 "v": torch.empty((B, n, H, D), dtype=torch.bfloat16, device=dev),
+                 "out": torch.empty((B, n, H, D), dtype=torch.bfloat16, device=dev),
+                 "lse": torch.empty((B, H, n), dtype=torch.float32, device=dev)} for _ in range(3)]
+    pinned = [(b.q.pin_memory(), b.k.pin_memory(), b.v.pin_memory()) for b in batches]
+    results = []
+    for i, (hq, hk, hv) in enumerate(pinned):
+        ho = torch.empty((B, n, H, D), dtype=torch.bfloat16, pin_memory=True)
+        hl = torch.empty((B, H, n), dtype=torch.float32, pin_memory=True)
+        results.append(forward_host(hq, hk, hv, stagings[i % 3], 0.09, True, out=ho, lse=hl,
+                                    stream=streams[i % 3], synchronize=False))
+    torch.cuda.synchronize()
+    for b, (ho, hl) in zip(batches, results):
+        do, dl = forward(b.q.to(dev), b.k.to(dev), b.v.to(dev), 0.09, True)
+        torch.cuda.synchronize()
+        assert torch.equal(ho, do.cpu()) and torch.equal(hl, dl.cpu())
+
+
 def test_wait_timeout_reports_status_and_context_survives():
     """A wait that nothing completes ends after its limit with FA_ERR_TIMEOUT; later calls still work."""
     rc, _ = device_status()

@@ -153,6 +153,43 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def standard_attention_context(w: W.Workload, q, k, v, ms_ours: float, dev, stream):
+    """Informative only, for non-causal unmasked 16-bit workloads: the pages' "standard attention"
+    ((q @ k^T * scale).softmax(-1) @ v in the input type, torch eager on cuBLAS; Flash Attention |
+    Hermes Skill, Workflow 1, Step 3) and torch's scaled_dot_product_attention (the pages' flash
+    call, a library kernel) on the same inputs and GPU, each timed with CUDA events after warm-up.
+    Neither is a target or an oracle; `speedup` = their time / this library's."""
+    if w.causal or w.window_left >= 0 or w.mask or w.dtype not in ("fp16", "bf16") or w.h_kv != w.H:
+        return None
+    qt, kt, vt = (t.transpose(1, 2) for t in (q, k, v))   # [B, H, N, D] views, as the pages' snippet
+
+    def standard():
+        return (qt @ kt.transpose(-2, -1) * w.scale).softmax(dim=-1) @ vt
+
+    def sdpa():
+        return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=w.scale)
+
+    res = {}
+    with torch.cuda.stream(stream):
+        for name, fn in (("standard_attention", standard), ("sdpa", sdpa)):
+            try:
+                for _ in range(3):
+                    fn()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(20):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ms = e0.elapsed_time(e1) / 20
+                res[name] = {"ms": ms, "speedup": ms / ms_ours}
+            except (RuntimeError, torch.cuda.OutOfMemoryError) as exc:
+                res[name] = {"unavailable": str(exc).splitlines()[0][:200]}
+    res["what"] = ("informative: standard = the pages' eager (q @ k^T * scale).softmax(-1) @ v (torch, cuBLAS); "
+                   "sdpa = torch scaled_dot_product_attention (library kernel); speedup = their ms / ours")
+    return res
+
+
 def oracle_rows_tflops(w: W.Workload, qkv, rows_per_head: int, heads=None):
     """Time the fp64 oracle on `rows_per_head` sampled rows of each selected (b, h).
 
@@ -317,6 +354,9 @@ def measure_config(name, cpu_rows, dev, stream, local, sms, with_cpu):
              "roofline": {"bound": bound, "peak": peak, "frac": tf / peak, "peak_source": src},
              "pct_of_nominal_dense_peak": 100.0 * tf / NOMINAL_TFLOPS[w.dtype],
              "clocks": clocks, "tflops_clock_normalised": clock_normalised(tf, clocks)}
+    ctx = standard_attention_context(w, q, k, v, ms_launch, dev, stream)
+    if ctx is not None:
+        entry["vs_standard_attention"] = ctx
     if with_cpu:
         ctf, cdt, n_rows, threads = oracle_rows_tflops(w, qkv, cpu_rows)
         entry["cpu_oracle"] = {"tflops": ctf, "seconds": cdt, "rows": n_rows, "cores": threads,
@@ -489,7 +529,7 @@ def main():
     # the other configurations, one after another on this GPU (rank 0 of a single-GPU run)
     configs = None
     if rank == 0 and world == 1 and not args.no_extras and args.batch is None:
-        del q, k, v, out, lse, staging, step
+        del q, k, v, out, lse, step
         torch.cuda.empty_cache()
         configs = {w.name: {"desc": w.desc, "dtype": w.dtype, "ms_per_launch": ms_per_step,
                             "tflops": per_launch_tflops,

@@ -166,7 +166,8 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
         return _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, stream, num_splits,
                                 attn_mask, dropout_p, seed, offset)
     if num_splits == 0:
-        num_splits = auto_splits(B, n_q, n_k, H, q.device)
+        # (a right window takes the one-launch path: no key-range slices)
+        num_splits = 1 if window_right != -1 else auto_splits(B, n_q, n_k, H, q.device)
     if q.dtype == torch.float8_e4m3fn:
         return forward_fp8(q, k, v, 1.0, 1.0, 1.0, scale, causal, window_left, out, lse, return_lse, stream,
                            num_splits, attn_mask, window_right)
@@ -328,7 +329,7 @@ def forward_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_descale:
     B, n_q, n_k, H, h_kv, D = _check_inputs(q8, k8, v8)
     _check_right_window(window_right, attn_mask, num_splits)
     if num_splits == 0:
-        num_splits = auto_splits(B, n_q, n_k, H, q8.device)
+        num_splits = 1 if window_right != -1 else auto_splits(B, n_q, n_k, H, q8.device)
     if q8.dtype != torch.float8_e4m3fn:
         raise ValueError("forward_fp8 takes float8_e4m3fn tensors")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)

@@ -159,3 +159,17 @@ def test_window_rejected_combinations():
                                                                               device=DEV))
     with pytest.raises(ValueError):
         forward(q, q, q, 0.1, False, -1, window_right=4, dropout_p=0.1, seed=1)
+
+
+def test_right_window_with_automatic_slices_keeps_the_window():
+    """num_splits=0 (pick slices automatically) must not drop the right window: few queries against
+    many keys would otherwise take the key-range-slice path, which has no right bound."""
+    qkv = inputs.make_qkv(1, 128, 4096, 2, 128, "bf16", seeds=(660, 661, 662))
+    q, k, v = qkv.q.to(DEV), qkv.k.to(DEV), qkv.v.to(DEV)
+    o1, l1 = forward(q, k, v, 0.1, False, -1, window_right=300, num_splits=0)
+    o2, l2 = forward(q, k, v, 0.1, False, -1, window_right=300)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    ref_o, ref_l = oracle(qkv, 0.1, False, -1, window_right=300)
+    d_o, d_l = compare(o1, l1, ref_o, ref_l)
+    assert d_o <= TOL_O["bf16"] and d_l <= TOL_LSE, (d_o, d_l)

@@ -159,7 +159,21 @@ int launch(const void* q, const void* k, const void* v, const FwdParams& base, c
     int rc = sched_counters(ds, stream, &p.sched);
     if (rc != FA_OK) return rc;
   }
-  fa_fwd_kernel<D, DT, SPLIT, MASK><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mm, p);
+  // programmatic stream serialization: the kernel's prologue (barriers,
+  // tensor memory, descriptor prefetch) may overlap the previous kernel on the
+  // stream; it waits for that kernel before any global-memory access
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa_fwd_kernel<D, DT, SPLIT, MASK>, mq, mk, mv, mm, p) != cudaSuccess)
+    return FA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

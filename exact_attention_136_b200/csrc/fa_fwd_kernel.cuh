@@ -1277,6 +1277,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if ((smem_u32(smem) & 1023u) != 0) {
     // 128-byte swizzled tiles need 1024-byte alignment; never expected.  The
     // CTA still counts itself finished, so the scratch is left at zero.
+    griddep_wait();
     if (threadIdx.x == 0) {
       atomicOr(p.status, ST_SMEM_MISALIGNED);
       cta_finished(p);
@@ -1331,6 +1332,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sh->tmem_base;
+  // the prologue above touches only this CTA's shared and tensor memory; the
+  // previous kernel on the stream (the scheduler counters it leaves at zero,
+  // any producer of Q, K, V) is complete from here on
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp < 4) {
     setmaxnreg_dec<REGS_LOAD_MMA>();

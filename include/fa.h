@@ -32,7 +32,11 @@
  * work-scheduler counters allocated once per device on the first call there
  * (one pair of counters per stream, left at zero by every launch).
  * Calls are asynchronous on `stream` (NULL = the legacy default stream);
- * outputs are ready when the stream's work completes.
+ * outputs are ready when the stream's work completes.  The forward kernel is
+ * launched with programmatic stream serialization: it may begin its
+ * on-chip prologue while the previous kernel on the stream finishes, and
+ * waits for that kernel to complete before it reads or writes any global
+ * memory, so stream order holds as for any launch.
  *
  * CUDA graphs: after one call on a stream (which sets kernel attributes and
  * takes the stream's counters), calls on that stream can be captured; a

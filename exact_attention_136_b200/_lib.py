@@ -24,6 +24,27 @@ FA_MASK_BOOL, FA_MASK_ADD = 1, 2
 _c_int, _c_float, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
 _fp = ctypes.POINTER(ctypes.c_float)
 
+class FwdArgs(ctypes.Structure):
+    """fa_fwd_args (include/fa.h), field for field."""
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("out", _vp), ("lse", _vp),
+                ("B", _c_int), ("N_q", _c_int), ("N_k", _c_int), ("H", _c_int), ("H_kv", _c_int), ("D", _c_int),
+                ("scale", _c_float), ("causal", _c_int), ("window_left", _c_int), ("window_right", _c_int),
+                ("dtype", _c_int), ("q_descale", _c_float), ("k_descale", _c_float), ("v_descale", _c_float),
+                ("cu_seqlens_q", _vp), ("cu_seqlens_k", _vp), ("total_q", _c_int), ("total_k", _c_int),
+                ("dropout_p", _c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint)]
+
+
+class BwdArgs(ctypes.Structure):
+    """fa_bwd_args (include/fa.h), field for field."""
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("out", _vp), ("dout", _vp), ("lse", _vp),
+                ("dq", _vp), ("dk", _vp), ("dv", _vp),
+                ("B", _c_int), ("N_q", _c_int), ("N_k", _c_int), ("H", _c_int), ("H_kv", _c_int), ("D", _c_int),
+                ("scale", _c_float), ("causal", _c_int), ("window_left", _c_int), ("window_right", _c_int),
+                ("dtype", _c_int), ("cu_seqlens_q", _vp), ("cu_seqlens_k", _vp), ("total_q", _c_int),
+                ("total_k", _c_int), ("dropout_p", _c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 SIGNATURES = {
     "fa_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                         _c_int, _c_int, _c_int, _vp]),
@@ -65,6 +86,8 @@ SIGNATURES = {
     "fa_bwd_dropout": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int,
                                 _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _c_float, ctypes.c_ulonglong,
                                 ctypes.c_uint, _vp, ctypes.c_size_t, _vp]),
+    "fa_fwd_ex": (_c_int, [ctypes.POINTER(FwdArgs), _vp]),
+    "fa_bwd_ex": (_c_int, [ctypes.POINTER(BwdArgs), _vp]),
     "fa_device_status": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "fa_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "fa_wait_probe": (_c_int, [ctypes.c_ulonglong, _vp]),

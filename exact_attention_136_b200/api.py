@@ -161,10 +161,10 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
     backward needs the same seed and offset.
     """
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
-    _check_right_window(window_right, attn_mask, num_splits, dropout_p)
+    _check_right_window(window_right, attn_mask, num_splits)
     if dropout_p:
         return _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, stream, num_splits,
-                                attn_mask, dropout_p, seed, offset)
+                                attn_mask, dropout_p, seed, offset, window_right)
     if num_splits == 0:
         # (a right window takes the one-launch path: no key-range slices)
         num_splits = 1 if window_right != -1 else auto_splits(B, n_q, n_k, H, q.device)
@@ -203,18 +203,53 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[f
     return out, lse
 
 
-def _check_right_window(window_right, attn_mask=None, num_splits=1, dropout_p=0.0):
+def _check_right_window(window_right, attn_mask=None, num_splits=1):
     if window_right == -1:
         return
     if window_right < -1:
         raise ValueError("window_right must be -1 (no bound) or >= 0")
-    if attn_mask is not None or num_splits not in (0, 1) or dropout_p:
-        raise ValueError("window_right is not combined with attn_mask, num_splits or dropout "
+    if attn_mask is not None or num_splits not in (0, 1):
+        raise ValueError("window_right is not combined with attn_mask or num_splits "
                          "(a boolean attn_mask expresses any window)")
 
 
+def _fwd_ex(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, window_right, dt, descales,
+            stream, packed=None, dropout=(0.0, 0, 0)):
+    """fa_fwd_ex: every combinable option in one call.  packed = (cu_q, cu_k, total_q, total_k) or None;
+    dropout = (p, seed, offset)."""
+    a = _lib.FwdArgs()
+    a.q, a.k, a.v, a.out = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
+    a.lse = lse.data_ptr() if lse is not None else None
+    a.B, a.N_q, a.N_k, a.H, a.H_kv, a.D = B, n_q, n_k, H, h_kv, D
+    a.scale, a.causal, a.window_left, a.window_right = scale, int(bool(causal)), int(window_left), int(window_right)
+    a.dtype = dt
+    a.q_descale, a.k_descale, a.v_descale = (float(x) for x in descales)
+    if packed is not None:
+        a.cu_seqlens_q, a.cu_seqlens_k = packed[0].data_ptr(), packed[1].data_ptr()
+        a.total_q, a.total_k = packed[2], packed[3]
+    a.dropout_p, a.seed, a.offset = float(dropout[0]), int(dropout[1]) & ((1 << 64) - 1), int(dropout[2]) & 0xFFFFFFFF
+    _lib.check(_lib.lib().fa_fwd_ex(ctypes.byref(a), stream.cuda_stream), "fa_fwd_ex")
+
+
+def _bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, B, n_q, n_k, H, h_kv, D, scale, causal, window_left,
+            window_right, dt, ws, nbytes, stream, packed=None, dropout=(0.0, 0, 0)):
+    """fa_bwd_ex: the backward of _fwd_ex with the same options."""
+    a = _lib.BwdArgs()
+    a.q, a.k, a.v, a.out, a.dout, a.lse = (t.data_ptr() for t in (q, k, v, out, dout, lse))
+    a.dq, a.dk, a.dv = dq.data_ptr(), dk.data_ptr(), dv.data_ptr()
+    a.B, a.N_q, a.N_k, a.H, a.H_kv, a.D = B, n_q, n_k, H, h_kv, D
+    a.scale, a.causal, a.window_left, a.window_right = scale, int(bool(causal)), int(window_left), int(window_right)
+    a.dtype = dt
+    if packed is not None:
+        a.cu_seqlens_q, a.cu_seqlens_k = packed[0].data_ptr(), packed[1].data_ptr()
+        a.total_q, a.total_k = packed[2], packed[3]
+    a.dropout_p, a.seed, a.offset = float(dropout[0]), int(dropout[1]) & ((1 << 64) - 1), int(dropout[2]) & 0xFFFFFFFF
+    a.workspace, a.workspace_bytes = ws.data_ptr(), nbytes
+    _lib.check(_lib.lib().fa_bwd_ex(ctypes.byref(a), stream.cuda_stream), "fa_bwd_ex")
+
+
 def _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, stream, num_splits, attn_mask,
-                     dropout_p, seed, offset):
+                     dropout_p, seed, offset, window_right=-1):
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
     if not (0.0 <= dropout_p < 1.0):
         raise ValueError("dropout_p must be in [0, 1)")
@@ -228,6 +263,10 @@ def _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, 
     out, lse = _outputs(q, B, n_q, H, D, out, lse, return_lse)
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        if window_right != -1:
+            _fwd_ex(q, k, v, out, lse, B, n_q, n_k, H, h_kv, D, scale, causal, window_left, window_right,
+                    _DT[q.dtype], (1.0, 1.0, 1.0), s, dropout=(dropout_p, seed, offset))
+            return out, lse
         rc = _lib.lib().fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                        lse.data_ptr() if lse is not None else None, B, n_q, n_k, H, h_kv, D, scale,
                                        int(bool(causal)), int(window_left), _DT[q.dtype], float(dropout_p),
@@ -239,11 +278,14 @@ def _dropout_forward(q, k, v, scale, causal, window_left, out, lse, return_lse, 
 def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
                    cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int, scale: Optional[float] = None,
                    causal: bool = False, window_left: int = -1, descales=(1.0, 1.0, 1.0),
-                   stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+                   stream: Optional[torch.cuda.Stream] = None, window_right: int = -1, dropout_p: float = 0.0,
+                   seed: Optional[int] = None, offset: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
     """Attention over a packed batch of sequences (fa_fwd_varlen): q [total_q,
     H, D], k, v [total_k, H_kv, D]; sequence b owns rows cu_seqlens_q[b] ..
     cu_seqlens_q[b+1] and keys cu_seqlens_k[b] .. cu_seqlens_k[b+1] (int32 CUDA
-    tensors of B + 1 entries).  Returns (out [total_q, H, D], lse [H, total_q])."""
+    tensors of B + 1 entries).  Returns (out [total_q, H, D], lse [H, total_q]).
+    window_right and dropout (p, seed, offset; sequence b draws as batch b
+    would) go through fa_fwd_ex."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor [total, heads, headdim]")
@@ -263,8 +305,17 @@ def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
     out_dtype = torch.float16 if q.dtype == torch.float16 else torch.bfloat16
     out = torch.empty((total_q, H, D), dtype=out_dtype, device=q.device)
     lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    _check_right_window(window_right)
+    if dropout_p and seed is None:
+        raise ValueError("dropout needs an explicit seed (and offset) so the backward can redraw the mask")
     with torch.cuda.device(q.device):
         s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        if window_right != -1 or dropout_p:
+            _fwd_ex(q, k, v, out, lse, B, int(max_seqlen_q), int(max_seqlen_k), H, h_kv, D, scale, causal,
+                    window_left, window_right, _DT[q.dtype], descales, s,
+                    packed=(cu_seqlens_q, cu_seqlens_k, total_q, total_k),
+                    dropout=(dropout_p, seed or 0, offset))
+            return out, lse
         rc = _lib.lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                       cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
                                       int(max_seqlen_k), total_q, total_k, H, h_kv, D, scale, int(bool(causal)),
@@ -277,10 +328,11 @@ def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
 def backward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
                     dout: torch.Tensor, cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, max_seqlen_q: int,
                     max_seqlen_k: int, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,
-                    stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+                    stream: Optional[torch.cuda.Stream] = None, window_right: int = -1, dropout_p: float = 0.0,
+                    seed: Optional[int] = None, offset: int = 0) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq [total_q, H, D], dk, dv [total_k, H_kv, D]) of forward_varlen over the same packed
     batch (fa_bwd_varlen), from its out and lse [H, total_q] (fp16 / bf16).  max_seqlen_q / max_seqlen_k
-    must bound every sequence's length."""
+    must bound every sequence's length.  window_right and dropout as given to the forward (fa_bwd_ex)."""
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         if not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor [total, heads, headdim]")
@@ -308,6 +360,17 @@ def backward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torc
         nbytes = int(_lib.lib().fa_bwd_workspace_bytes(1, total_q, H, D))
         with torch.cuda.stream(s):
             ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+        _check_right_window(window_right)
+        if dropout_p and seed is None:
+            raise ValueError("a dropout backward needs the forward's seed (and offset)")
+        if window_right != -1 or dropout_p:
+            _bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, B, int(max_seqlen_q), int(max_seqlen_k), H, h_kv, D, scale,
+                    causal, window_left, window_right, _DT[q.dtype], ws, nbytes, s,
+                    packed=(cu_seqlens_q, cu_seqlens_k, total_q, total_k), dropout=(dropout_p, seed or 0, offset))
+            if s != torch.cuda.current_stream(q.device):
+                for t in (dq, dk, dv):
+                    t.record_stream(s)
+            return dq, dk, dv
         rc = _lib.lib().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
                                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                       cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
@@ -380,7 +443,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
     B, n_q, n_k, H, h_kv, D = _check_inputs(q, k, v)
     if q.dtype not in (torch.float16, torch.bfloat16):
         raise ValueError("backward takes fp16 or bf16 inputs")
-    _check_right_window(window_right, dropout_p=dropout_p)
+    _check_right_window(window_right)
     for name, t in (("out", out), ("dout", dout)):
         if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous tensor like q")
@@ -393,7 +456,13 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tenso
         nbytes = int(_lib.lib().fa_bwd_workspace_bytes(B, n_q, H, D))
         with torch.cuda.stream(s):
             ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
-        if dropout_p:
+        if dropout_p and window_right != -1:
+            if seed is None:
+                raise ValueError("a dropout backward needs the forward's seed (and offset)")
+            _bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, B, n_q, n_k, H, h_kv, D, scale, causal, window_left,
+                    window_right, _DT[q.dtype], ws, nbytes, s, dropout=(dropout_p, seed, offset))
+            rc = _lib.FA_OK
+        elif dropout_p:
             if seed is None:
                 raise ValueError("a dropout backward needs the forward's seed (and offset)")
             rc = _lib.lib().fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),

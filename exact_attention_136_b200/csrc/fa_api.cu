@@ -208,6 +208,23 @@ int right_bound(int causal, int window_right, int Nq, int Nk, int* R) {
   return FA_OK;
 }
 
+// Sizes and pointers of a packed batch (fa_fwd_varlen, fa_bwd_varlen and the
+// struct entry points), checked on the host.  The forward's work units cover
+// max_q rows of every sequence; the backward's blocks also cover max_k keys.
+int packed_check(const int* cu_q, const int* cu_k, int B, int max_q, int max_k, int total_q, int total_k, int H,
+                 int H_kv, bool backward) {
+  if (B < 1 || total_q < 0 || total_k < 0 || max_q < 0 || max_k < 0) return FA_ERR_ARG;
+  if (!cu_q || !cu_k || (reinterpret_cast<uintptr_t>(cu_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_k) & 3u) != 0)
+    return FA_ERR_ARG;
+  if ((total_q > 0 && max_q < 1) || max_q > total_q || max_k > total_k) return FA_ERR_ARG;
+  if (backward && total_k > 0 && max_k < 1) return FA_ERR_ARG;
+  const int64_t units = static_cast<int64_t>((max_q + 2 * BLOCK_M - 1) / (2 * BLOCK_M)) * B * H;
+  const int64_t blocks_kv = static_cast<int64_t>((max_k + 127) / 128) * B * (H_kv > 0 ? H_kv : 1);
+  const int64_t blocks_q = static_cast<int64_t>((max_q + 127) / 128) * B * H;
+  if (units > 0x7fffffff || blocks_kv > 0x7fffffff || blocks_q > 0x7fffffff) return FA_ERR_ARG;
+  return FA_OK;
+}
+
 // Workspace of a split forward: fp32 O of every slice [splits, B, N_q, H, D]
 // followed by its LSE [splits, B, H, N_q].
 size_t splitkv_workspace_bytes(int B, int Nq, int H, int D, int splits) {
@@ -469,14 +486,9 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float*
                   const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int H,
                   int H_kv, int D, float scale, int causal, int window_left, int dtype, float q_descale,
                   float k_descale, float v_descale, fa_stream_t stream) {
-  if (B < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return FA_ERR_ARG;
-  if (!cu_seqlens_q || !cu_seqlens_k || (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 ||
-      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
-    return FA_ERR_ARG;
-  if ((total_q > 0 && max_seqlen_q < 1) || max_seqlen_q > total_q || max_seqlen_k > total_k) return FA_ERR_ARG;
-  // the work units cover max_seqlen_q rows of every sequence
-  const int64_t units = static_cast<int64_t>((max_seqlen_q + 2 * fa::BLOCK_M - 1) / (2 * fa::BLOCK_M)) * B * H;
-  if (units > 0x7fffffff) return FA_ERR_ARG;
+  const int rc = fa::packed_check(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, H,
+                                  H_kv, false);
+  if (rc != FA_OK) return rc;
   return fa::forward(q, k, v, out, lse, B, max_seqlen_q, max_seqlen_k, H, H_kv, D, scale, causal, window_left, dtype,
                      q_descale, k_descale, v_descale, reinterpret_cast<cudaStream_t>(stream), nullptr, 1, nullptr, 0,
                      nullptr, 0, 0, 0, 0, 0.f, 0, 0, cu_seqlens_q, cu_seqlens_k, total_q, total_k);
@@ -595,20 +607,42 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* out, 
                   int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int H, int H_kv, int D, float scale,
                   int causal, int window_left, int dtype, void* workspace, size_t workspace_bytes,
                   fa_stream_t stream) {
-  if (B < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return FA_ERR_ARG;
-  if (!cu_seqlens_q || !cu_seqlens_k || (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 ||
-      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
-    return FA_ERR_ARG;
-  // every row and key of a sequence lies in a launched block
-  if ((total_q > 0 && max_seqlen_q < 1) || (total_k > 0 && max_seqlen_k < 1) || max_seqlen_q > total_q ||
-      max_seqlen_k > total_k)
-    return FA_ERR_ARG;
-  const int64_t blocks_kv = static_cast<int64_t>((max_seqlen_k + 127) / 128) * B * (H_kv > 0 ? H_kv : 1);
-  const int64_t blocks_q = static_cast<int64_t>((max_seqlen_q + 127) / 128) * B * H;
-  if (blocks_kv > 0x7fffffff || blocks_q > 0x7fffffff) return FA_ERR_ARG;
+  // (every row and key of a sequence lies in a launched block)
+  const int rc = fa::packed_check(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, H,
+                                  H_kv, true);
+  if (rc != FA_OK) return rc;
   return fa::backward(q, k, v, out, dout, lse, dq, dk, dv, B, max_seqlen_q, max_seqlen_k, H, H_kv, D, scale, causal,
                       window_left, dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), 0.f, 0,
                       0, -1, cu_seqlens_q, cu_seqlens_k, total_q, total_k);
+}
+
+int fa_fwd_ex(const fa_fwd_args* a, fa_stream_t stream) {
+  if (!a || (a->cu_seqlens_q == nullptr) != (a->cu_seqlens_k == nullptr)) return FA_ERR_ARG;
+  const bool packed = a->cu_seqlens_q != nullptr;
+  if (packed) {
+    const int rc = fa::packed_check(a->cu_seqlens_q, a->cu_seqlens_k, a->B, a->N_q, a->N_k, a->total_q, a->total_k,
+                                    a->H, a->H_kv, false);
+    if (rc != FA_OK) return rc;
+  }
+  return fa::forward(a->q, a->k, a->v, a->out, a->lse, a->B, a->N_q, a->N_k, a->H, a->H_kv, a->D, a->scale,
+                     a->causal, a->window_left, a->dtype, a->q_descale, a->k_descale, a->v_descale,
+                     reinterpret_cast<cudaStream_t>(stream), nullptr, 1, nullptr, 0, nullptr, 0, 0, 0, 0, a->dropout_p,
+                     a->seed, a->offset, a->cu_seqlens_q, a->cu_seqlens_k, packed ? a->total_q : 0,
+                     packed ? a->total_k : 0, a->window_right);
+}
+
+int fa_bwd_ex(const fa_bwd_args* a, fa_stream_t stream) {
+  if (!a || (a->cu_seqlens_q == nullptr) != (a->cu_seqlens_k == nullptr)) return FA_ERR_ARG;
+  const bool packed = a->cu_seqlens_q != nullptr;
+  if (packed) {
+    const int rc = fa::packed_check(a->cu_seqlens_q, a->cu_seqlens_k, a->B, a->N_q, a->N_k, a->total_q, a->total_k,
+                                    a->H, a->H_kv, true);
+    if (rc != FA_OK) return rc;
+  }
+  return fa::backward(a->q, a->k, a->v, a->out, a->dout, a->lse, a->dq, a->dk, a->dv, a->B, a->N_q, a->N_k, a->H,
+                      a->H_kv, a->D, a->scale, a->causal, a->window_left, a->dtype, a->workspace, a->workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), a->dropout_p, a->seed, a->offset, a->window_right,
+                      a->cu_seqlens_q, a->cu_seqlens_k, packed ? a->total_q : 0, packed ? a->total_k : 0);
 }
 
 int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out, const void* dout,

@@ -67,7 +67,6 @@ int backward(const void* q, const void* k, const void* v, const void* out, const
   if (dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;
   if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_ARG;
   const bool drop = dropout_p > 0.f;
-  if (cu_q && drop) return FA_ERR_ARG;
   if ((rNq > 0 && (!dout || !lse || !dq)) || (rNk > 0 && (!dk || !dv))) return FA_ERR_ARG;
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)

@@ -14,8 +14,7 @@ Readings (the pages leave these open):
   i - left <= j <= i + right, -1 meaning no bound on that side
   (fa_fwd_window).  With ``causal=True`` the right window is zero whatever
   ``right`` says (the page pairs causal=True with a two-sided window, which
-  contradict each other; causal wins).  A right window without causal is
-  not combined with dropout.
+  contradict each other; causal wins).
 - ``dropout_p``: the usual attention dropout, each softmax probability kept
   with probability 1 - p and scaled by 1 / (1 - p) (fa_fwd_dropout).  The
   pages name no random generator; each call draws a 64-bit seed from
@@ -33,16 +32,12 @@ import torch
 from .api import backward, forward
 
 
-def _window(causal: bool, window_size: Tuple[int, int], dropout_p: float) -> Tuple[int, int]:
+def _window(causal: bool, window_size: Tuple[int, int]) -> Tuple[int, int]:
     """(left, right) as forward / backward take them; right -1 under causal."""
     left, right = (int(window_size[0]), int(window_size[1]))
     if left < -1 or right < -1:
         raise ValueError("window_size entries are -1 (unlimited) or >= 0")
-    if causal:
-        return left, -1
-    if right != -1 and dropout_p:
-        raise NotImplementedError("a right window without causal=True is not combined with dropout")
-    return left, right
+    return (left, -1) if causal else (left, right)
 
 
 class _FlashAttn(torch.autograd.Function):
@@ -51,7 +46,8 @@ class _FlashAttn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, scale, causal, window_left, window_right, dropout_p, seed):
         if dropout_p:
-            out, lse = forward(q, k, v, scale, causal, window_left, dropout_p=dropout_p, seed=seed)
+            out, lse = forward(q, k, v, scale, causal, window_left, dropout_p=dropout_p, seed=seed,
+                               window_right=window_right)
         else:
             out, lse = forward(q, k, v, scale, causal, window_left, window_right=window_right)
         ctx.save_for_backward(q, k, v, out, lse)
@@ -67,7 +63,7 @@ class _FlashAttn(torch.autograd.Function):
         q, k, v, out, lse = ctx.saved_tensors
         if ctx.dropout_p:
             dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left,
-                                  dropout_p=ctx.dropout_p, seed=ctx.seed)
+                                  dropout_p=ctx.dropout_p, seed=ctx.seed, window_right=ctx.window_right)
         else:
             dq, dk, dv = backward(q, k, v, out, lse, dout.contiguous(), ctx.scale, ctx.causal, ctx.window_left,
                                   window_right=ctx.window_right)
@@ -87,14 +83,14 @@ def flash_attn_func(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dropout_p
     dropout_p = float(dropout_p)
     if not (0.0 <= dropout_p < 1.0):
         raise ValueError("dropout_p must be in [0, 1)")
-    wl, wr = _window(bool(causal), window_size, dropout_p)
+    wl, wr = _window(bool(causal), window_size)
     scale = float(softmax_scale) if softmax_scale is not None else q.shape[-1] ** -0.5
     seed = int(torch.randint(0, 2 ** 62, (1,)).item()) if dropout_p > 0.0 else 0
     needs_grad = torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v))
     if needs_grad:
         out, lse = _FlashAttn.apply(q, k, v, scale, bool(causal), wl, wr, dropout_p, seed)
     elif dropout_p > 0.0:
-        out, lse = forward(q, k, v, scale, bool(causal), wl, dropout_p=dropout_p, seed=seed)
+        out, lse = forward(q, k, v, scale, bool(causal), wl, dropout_p=dropout_p, seed=seed, window_right=wr)
     else:
         out, lse = forward(q, k, v, scale, bool(causal), wl, window_right=wr)
     return (out, lse) if return_lse else out

@@ -381,6 +381,74 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out,
                    size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_fwd_ex / fa_bwd_ex -- one call with every option of the pages'
+ * flash_attn_func that can be combined (Flash Attention | Hermes Skill,
+ * Workflow 2, Steps 2-3: dropout_p, causal, window_size=(left, right),
+ * K/V with fewer heads), over a padded or a packed batch.  The fields take
+ * the meanings of the entry points above:
+ *   q ... lse, B, N_q, N_k, H, H_kv, D, scale, causal, window_left, dtype and
+ *     the descales as fa_fwd_gqa; window_right as fa_fwd_window;
+ *   cu_seqlens_q / cu_seqlens_k (both NULL: the padded batch [B, N_q / N_k,
+ *     ...]; both set: the packed batch of fa_fwd_varlen, B sequences, N_q /
+ *     N_k the longest (fa_bwd_ex: every sequence at most that long), total_q
+ *     / total_k the packed rows);
+ *   dropout_p, seed, offset as fa_fwd_dropout (0 = no dropout; FA_FP16 /
+ *     FA_BF16 only); in a packed batch sequence b draws as batch b would.
+ * fa_bwd_ex adds out, dout, dq, dk, dv and the workspace of fa_bwd
+ * (fa_bwd_workspace_bytes(B, N_q, H, D), or (1, total_q, H, D) for a packed
+ * batch) and takes the forward's options unchanged; FA_E4M3 is refused
+ * there.  A mask or a split key range is not an option here (fa_fwd_mask,
+ * fa_fwd_splitkv).  Validation, ownership and return values as the entry
+ * points whose fields they are; FA_ERR_ARG also for a NULL args pointer or
+ * only one of the two cu_seqlens pointers.
+ */
+typedef struct fa_fwd_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  int B, N_q, N_k, H, H_kv, D;
+  float scale;
+  int causal, window_left, window_right;
+  int dtype;
+  float q_descale, k_descale, v_descale;
+  const int* cu_seqlens_q;
+  const int* cu_seqlens_k;
+  int total_q, total_k;
+  float dropout_p;
+  unsigned long long seed;
+  unsigned offset;
+} fa_fwd_args;
+
+typedef struct fa_bwd_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* out;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  int B, N_q, N_k, H, H_kv, D;
+  float scale;
+  int causal, window_left, window_right;
+  int dtype;
+  const int* cu_seqlens_q;
+  const int* cu_seqlens_k;
+  int total_q, total_k;
+  float dropout_p;
+  unsigned long long seed;
+  unsigned offset;
+  void* workspace;
+  size_t workspace_bytes;
+} fa_bwd_args;
+
+int fa_fwd_ex(const fa_fwd_args* args, fa_stream_t stream);
+int fa_bwd_ex(const fa_bwd_args* args, fa_stream_t stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * device status word that kernels set when a wait times out.  Returns FA_OK,
  * FA_ERR_TIMEOUT (and the raw flag bits in *flags when flags != NULL) or

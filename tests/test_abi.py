@@ -330,3 +330,57 @@ def test_varlen_backward_arguments_validated(kw, expect):
     assert f(A, A, A, A, A, A, A, A, A, a["cu_q"], a["cu_k"], a["B"], a["max_q"], a["max_k"], a["total_q"],
              a["total_k"], a["H"], a["H_kv"], a["D"], 0.1, a["causal"], a["wl"], a["dt"], A, a["ws_bytes"],
              None) == expect
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes structures of fa_fwd_args / fa_bwd_args have the C compiler's size and field offsets."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lines = []
+    for cname, py in (("fa_fwd_args", _lib.FwdArgs), ("fa_bwd_args", _lib.BwdArgs)):
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in py._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"fa.h\"\nint main(void) {\n"
+                   + "\n".join(lines) + "\n  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    res = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o",
+                          str(exe)], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60).stdout.split("\n")
+    got = {(ln.split()[0], ln.split()[1]): int(ln.split()[2]) for ln in out if ln.strip()}
+    for cname, py in (("fa_fwd_args", _lib.FwdArgs), ("fa_bwd_args", _lib.BwdArgs)):
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for field, _ in py._fields_:
+            assert got[(cname, field)] == getattr(py, field).offset, (cname, field)
+
+
+@pytest.mark.parametrize("kw, expect", [
+    (dict(cu_q=A), _lib.FA_ERR_ARG),                 # one of the two packed-batch pointers
+    (dict(wr=-2), _lib.FA_ERR_ARG),
+    (dict(p=1.0), _lib.FA_ERR_ARG),
+    (dict(p=0.1, dt=_lib.FA_E4M3, D=128), _lib.FA_ERR_UNSUPPORTED),
+    (dict(cu_q=A, cu_k=A, total_q=150, total_k=150, Nq=0), _lib.FA_ERR_ARG),   # packed rows, no launched block
+    (dict(D=96), _lib.FA_ERR_UNSUPPORTED),
+])
+def test_struct_entry_points_validated(kw, expect):
+    """fa_fwd_ex / fa_bwd_ex check their arguments on the host, before any GPU work."""
+    a = dict(B=2, Nq=100, Nk=100, H=2, D=64, wl=-1, wr=3, dt=_lib.FA_FP16, p=0.0, cu_q=None, cu_k=None,
+             total_q=0, total_k=0)
+    a.update(kw)
+    f = _lib.FwdArgs(q=A, k=A, v=A, out=A, lse=None, B=a["B"], N_q=a["Nq"], N_k=a["Nk"], H=a["H"], H_kv=a["H"],
+                     D=a["D"], scale=0.1, causal=0, window_left=a["wl"], window_right=a["wr"], dtype=a["dt"],
+                     q_descale=1.0, k_descale=1.0, v_descale=1.0, cu_seqlens_q=a["cu_q"], cu_seqlens_k=a["cu_k"],
+                     total_q=a["total_q"], total_k=a["total_k"], dropout_p=a["p"], seed=1, offset=0)
+    assert _lib.lib().fa_fwd_ex(ctypes.byref(f), None) == expect
+    b = _lib.BwdArgs(q=A, k=A, v=A, out=A, dout=A, lse=A, dq=A, dk=A, dv=A, B=a["B"], N_q=a["Nq"], N_k=a["Nk"],
+                     H=a["H"], H_kv=a["H"], D=a["D"], scale=0.1, causal=0, window_left=a["wl"],
+                     window_right=a["wr"], dtype=a["dt"], cu_seqlens_q=a["cu_q"], cu_seqlens_k=a["cu_k"],
+                     total_q=a["total_q"], total_k=a["total_k"], dropout_p=a["p"], seed=1, offset=0, workspace=A,
+                     workspace_bytes=1 << 30)
+    assert _lib.lib().fa_bwd_ex(ctypes.byref(b), None) == expect
+    assert _lib.lib().fa_fwd_ex(None, None) == _lib.FA_ERR_ARG

@@ -86,8 +86,6 @@ def test_rejected_arguments(oracle_backend):
     for bad_p in (-0.1, 1.0):
         with pytest.raises(ValueError):
             itf.flash_attn_func(q, q, q, dropout_p=bad_p)
-    with pytest.raises(NotImplementedError):
-        itf.flash_attn_func(q, q, q, causal=False, window_size=(2, 2), dropout_p=0.1)
     with pytest.raises(ValueError):
         itf.flash_attn_func(q, q, q, window_size=(-2, -1))
     assert oracle_backend == []
@@ -127,3 +125,15 @@ def test_dropout_gradients_and_seed_plumbing(oracle_backend):
     assert torch.allclose(out, ref, atol=1e-12)
     for a, b in ((q.grad, q2.grad), (k.grad, k2.grad), (v.grad, v2.grad)):
         assert torch.allclose(a, b, atol=1e-12)
+
+
+def test_dropout_with_two_sided_window_reaches_both_calls(oracle_backend):
+    """dropout_p with a non-causal window_size=(left, right): the forward and the backward get the same
+    seed and both window entries."""
+    g = torch.Generator().manual_seed(13)
+    q, k, v = (torch.randn(1, 12, 2, 4, generator=g, dtype=torch.float64, requires_grad=True) for _ in range(3))
+    itf.flash_attn_func(q, k, v, dropout_p=0.2, window_size=(3, 2)).sum().backward()
+    (f, bw) = oracle_backend
+    assert f[0] == "fwd" and bw[0] == "bwd"
+    assert f[1:] == bw[1:] and f[3] == 3 and f[4] == 0.2 and f[6] == 0 and f[7] == 2
+    assert all(t.grad is not None and torch.isfinite(t.grad).all() for t in (q, k, v))

@@ -157,8 +157,6 @@ def test_window_rejected_combinations():
     with pytest.raises(ValueError):
         forward(q, q, q, 0.1, False, -1, window_right=4, attn_mask=torch.ones(128, 128, dtype=torch.bool,
                                                                               device=DEV))
-    with pytest.raises(ValueError):
-        forward(q, q, q, 0.1, False, -1, window_right=4, dropout_p=0.1, seed=1)
 
 
 def test_right_window_with_automatic_slices_keeps_the_window():

@@ -11,7 +11,7 @@ include/fa.h); this package only marshals arguments.
 
 from .api import (auto_splits, backward, backward_varlen, device_status, forward, forward_fp8, forward_host,
                   forward_varlen, set_wait_limit_ns, wait_probe)
-from .interface import flash_attn_func
+from .interface import flash_attn_func, flash_attn_varlen_func
 
 __all__ = ["forward", "forward_fp8", "forward_host", "forward_varlen", "backward", "backward_varlen",
-           "flash_attn_func", "auto_splits", "device_status", "set_wait_limit_ns", "wait_probe"]
+           "flash_attn_func", "flash_attn_varlen_func", "auto_splits", "device_status", "set_wait_limit_ns", "wait_probe"]

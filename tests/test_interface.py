@@ -137,3 +137,65 @@ def test_dropout_with_two_sided_window_reaches_both_calls(oracle_backend):
     assert f[0] == "fwd" and bw[0] == "bwd"
     assert f[1:] == bw[1:] and f[3] == 3 and f[4] == 0.2 and f[6] == 0 and f[7] == 2
     assert all(t.grad is not None and torch.isfinite(t.grad).all() for t in (q, k, v))
+
+
+@pytest.fixture
+def packed_backend(monkeypatch):
+    """forward_varlen / backward_varlen replaced by the oracle run on each sequence (CPU tensors)."""
+    calls = []
+
+    def seqs(cu):
+        c = cu.tolist()
+        return [(c[i], c[i + 1]) for i in range(len(c) - 1)]
+
+    def fwd(q, k, v, cu_q, cu_k, max_q, max_k, scale, causal, wl, window_right=-1, dropout_p=0.0, seed=None,
+            offset=0):
+        calls.append(("fwd", max_q, max_k, scale, causal, wl, window_right, dropout_p))
+        out = torch.zeros(q.shape, dtype=torch.float64)
+        lse = torch.zeros((q.shape[1], q.shape[0]), dtype=torch.float64)
+        for (q0, q1), (k0, k1) in zip(seqs(cu_q), seqs(cu_k)):
+            o, l = attention_ref(q[None, q0:q1].detach().numpy(), k[None, k0:k1].detach().numpy(),
+                                 v[None, k0:k1].detach().numpy(), scale, causal, wl, window_right=window_right)
+            out[q0:q1], lse[:, q0:q1] = torch.from_numpy(o[0]), torch.from_numpy(l[0])
+        return out, lse
+
+    def bwd(q, k, v, out, lse, dout, cu_q, cu_k, max_q, max_k, scale, causal, wl, window_right=-1, dropout_p=0.0,
+            seed=None, offset=0):
+        calls.append(("bwd", max_q, max_k, scale, causal, wl, window_right, dropout_p))
+        grads = [torch.zeros(t.shape, dtype=torch.float64) for t in (q, k, v)]
+        for (q0, q1), (k0, k1) in zip(seqs(cu_q), seqs(cu_k)):
+            g = attention_backward_ref(q[None, q0:q1].detach().numpy(), k[None, k0:k1].detach().numpy(),
+                                       v[None, k0:k1].detach().numpy(), dout[None, q0:q1].numpy(), scale, causal, wl,
+                                       window_right=window_right)
+            grads[0][q0:q1] = torch.from_numpy(g[0][0])
+            grads[1][k0:k1] = torch.from_numpy(g[1][0])
+            grads[2][k0:k1] = torch.from_numpy(g[2][0])
+        return tuple(grads)
+
+    monkeypatch.setattr(itf, "forward_varlen", fwd)
+    monkeypatch.setattr(itf, "backward_varlen", bwd)
+    return calls
+
+
+@pytest.mark.parametrize("causal, window", [(True, (-1, -1)), (False, (2, 3))])
+def test_packed_call_gradients_match_torch_autograd(packed_backend, causal, window):
+    """flash_attn_varlen_func: gradients of the packed call equal torch autograd's of plain attention run
+    on each sequence alone, and the options reach the packed forward and backward unchanged."""
+    g = torch.Generator().manual_seed(21)
+    lens = [5, 1, 8]
+    total = sum(lens)
+    q, k, v = (torch.randn(total, 2, 4, generator=g, dtype=torch.float64, requires_grad=True) for _ in range(3))
+    do = torch.randn(total, 2, 4, generator=g, dtype=torch.float64)
+    cu = torch.tensor([0, 5, 6, 14], dtype=torch.int32)
+    out = itf.flash_attn_varlen_func(q, k, v, cu, cu, 8, 8, causal=causal, window_size=window)
+    out.backward(do)
+    wl, wr = window[0], (-1 if causal else window[1])
+    q2, k2, v2 = (t.detach().clone().requires_grad_() for t in (q, k, v))
+    refs = []
+    for a, b in ((0, 5), (5, 6), (6, 14)):
+        refs.append(_plain_attention(q2[None, a:b], k2[None, a:b], v2[None, a:b], 0.5, causal, wl, wr)[0])
+    torch.cat(refs).backward(do)
+    assert torch.allclose(out, torch.cat(refs), atol=1e-12)
+    for a_, b_ in ((q.grad, q2.grad), (k.grad, k2.grad), (v.grad, v2.grad)):
+        assert torch.allclose(a_, b_, atol=1e-12)
+    assert packed_backend == [("fwd", 8, 8, 0.5, causal, wl, wr, 0.0), ("bwd", 8, 8, 0.5, causal, wl, wr, 0.0)]

@@ -171,3 +171,22 @@ def test_varlen_backward_rejects_bad_sizes():
         backward_varlen(t, t, t, t, lse, t, cu, cu, 0, 128)       # rows but max_seqlen_q 0
     with pytest.raises(_lib.FAError):
         backward_varlen(t, t, t, t, lse, t, cu, cu, 128, 300)     # longer than the packed keys
+
+
+def test_packed_call_with_autograd_equals_the_direct_calls():
+    """flash_attn_varlen_func (autograd over the packed batch) gives the outputs and gradients of
+    forward_varlen / backward_varlen bit for bit."""
+    from exact_attention_136_b200 import backward_varlen, flash_attn_varlen_func
+    lens_q = [300, 1, 517]
+    qkv, q, k, v, cu_q, cu_k = _packed(lens_q, lens_q, 4, 2, 128, "bf16", 880)
+    do = inputs.make_qkv(1, sum(lens_q), 1, 4, 128, "bf16", seeds=(884, 885, 886)).q[0].to(DEV)
+    qd, kd, vd = (t.contiguous().to(DEV).requires_grad_() for t in (q, k, v))
+    cq, ck = cu_q.to(DEV), cu_k.to(DEV)
+    out = flash_attn_varlen_func(qd, kd, vd, cq, ck, 517, 517, causal=True, window_size=(100, 0))
+    out.backward(do)
+    o2, l2 = forward_varlen(qd.detach(), kd.detach(), vd.detach(), cq, ck, 517, 517, 128 ** -0.5, True, 100)
+    g2 = backward_varlen(qd.detach(), kd.detach(), vd.detach(), o2, l2, do, cq, ck, 517, 517, 128 ** -0.5, True, 100)
+    torch.cuda.synchronize()
+    assert torch.equal(out.detach(), o2)
+    for got, want in zip((qd.grad, kd.grad, vd.grad), g2):
+        assert torch.equal(got, want)

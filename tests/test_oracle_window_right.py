@@ -151,3 +151,23 @@ def test_backward_right_window_matches_finite_differences():
         want = _fd_grads(q, k, v, do, 0.6, wl, wr)
         for g, w in zip(got, want):
             assert np.allclose(g, w, rtol=1e-6, atol=1e-7), float(np.max(np.abs(g - w)))
+
+
+def test_right_window_with_dropout_reduces_to_causal_and_to_unbounded():
+    """With dropout the right window still means j <= i + r: r = 0 gives the causal dropout forward and
+    backward, r >= N_k the unbounded ones (the keep bits do not depend on the window)."""
+    q, k, v = _rand((2, 9, 2, 4), 800), _rand((2, 9, 2, 4), 801), _rand((2, 9, 2, 4), 802)
+    do = _rand((2, 9, 2, 4), 803)
+    kw = dict(dropout_p=0.3, seed=12345, offset=7)
+    for wl in (-1, 2):
+        o1, l1 = attention_ref(q, k, v, 0.6, False, wl, window_right=0, **kw)
+        o2, l2 = attention_ref(q, k, v, 0.6, True, wl, **kw)
+        np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+        g1 = attention_backward_ref(q, k, v, do, 0.6, False, wl, window_right=0, **kw)
+        g2 = attention_backward_ref(q, k, v, do, 0.6, True, wl, **kw)
+        for a, b in zip(g1, g2):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+        o3, _ = attention_ref(q, k, v, 0.6, False, wl, window_right=9, **kw)
+        o4, _ = attention_ref(q, k, v, 0.6, False, wl, **kw)
+        np.testing.assert_allclose(o3, o4, rtol=0, atol=1e-13)
